@@ -1,0 +1,147 @@
+/*
+ * int8mm.h -- C ABI of the B200 (sm_100a) LLM.int8() linear layer, libint8mm.so.
+ *
+ * The layer (Y = X . W^T with vector-wise int8 quantization and mixed-precision
+ * decomposition) is defined on two pages, cited below by title and section:
+ *   [P5] "PyTorch 2.9 支持 LLM.int8()：大模型低比特推理的工程突破" (yongjin360.com/news/208476)
+ *   [P2] "8位量化实战：离群值处理与显存优化避坑指南" (zwxr.cn/news/257102)
+ *
+ * Conventions for every entry point:
+ *   - Matrices are row-major with K (the input-feature axis) contiguous.
+ *   - Half-precision data is IEEE binary16 (passed as void*; the ABI has no half type).
+ *   - Every pointer is a caller-owned DEVICE pointer on the current CUDA device, unless
+ *     stated otherwise; the library allocates nothing and keeps no state between calls.
+ *     Matrix and vector pointers must be 16-byte aligned.
+ *   - K must be a multiple of 16 (each row must start on a 16-byte boundary for the
+ *     tensor-memory-access unit); 1 <= M, N and K <= INT8MM_MAX_K.
+ *   - Work is enqueued on `stream` (NULL = the legacy default stream) and the call
+ *     returns without waiting; the return value reports argument and launch errors only.
+ *     Kernel-side failures (a bounded wait that gave up) are written as a negative code
+ *     to a device status word and read with int8_read_device_status().
+ *   - Results are deterministic: the same inputs give the same bits on every call.
+ */
+#ifndef INT8MM_H
+#define INT8MM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *int8mm_stream_t; /* the same type as cudaStream_t */
+
+#define INT8MM_MAX_K 65536
+
+/* status codes */
+#define INT8MM_OK 0
+#define INT8MM_ERR_NULL (-1)         /* a required pointer is NULL */
+#define INT8MM_ERR_SHAPE (-2)        /* M, N or K out of range */
+#define INT8MM_ERR_ALIGN (-3)        /* K % 16 != 0, or a pointer not 16-byte aligned */
+#define INT8MM_ERR_THRESHOLD (-4)    /* threshold is NaN */
+#define INT8MM_ERR_WORKSPACE (-5)    /* workspace NULL, misaligned or too small */
+#define INT8MM_ERR_CUDA (-6)         /* a CUDA runtime or launch error */
+#define INT8MM_ERR_DEVICE (-7)       /* the current device is not sm_100 */
+#define INT8MM_ERR_TIMEOUT (-8)      /* device side: a bounded wait gave up */
+#define INT8MM_ERR_OVERFLOW (-9)     /* device side: an outlier count beyond K */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *int8_status_string(int status);
+
+/*
+ * Per-output-channel weight quantization, done once when the layer is loaded.
+ * [P5] section "LLM.int8() 是怎么做到几乎无损的", item 1:
+ *   w_scale[n] = max_k |W[n,k]| / 127;  Wq[n,k] = round(W[n,k] / w_scale[n]).
+ * The scale is a float32 IEEE division; round is to nearest, ties to even; the result is
+ * clamped to [-127, 127]; an all-zero channel gets scale 0 and all-zero codes.
+ *   W        [in]  binary16 [N, K]
+ *   Wq       [out] int8     [N, K]
+ *   w_scale  [out] float32  [N]
+ */
+int int8_quant_weight(const void *W, int N, int K, int8_t *Wq, float *w_scale,
+                      int8mm_stream_t stream);
+
+/*
+ * Bytes of device workspace int8_linear_forward and int8_quantize_rows need for an
+ * [M, K] x [N, K]^T layer.  The workspace holds the device status word (its first int32),
+ * the outlier-column mask and list, the row scales, the int8 activations and the fp16
+ * outlier operands, sized for the worst case (every column an outlier).  Zero it once
+ * before first use (kernels only ever write a nonzero code into the status word).
+ * Returns 0 for out-of-range sizes.
+ */
+size_t int8_linear_workspace_size(int M, int N, int K);
+
+/*
+ * The LLM.int8() linear layer, [P2] section 2.3 with [P5] items 1-3:
+ *   O   = { j : max_i |X[i,j]| > threshold }          (outlier feature columns)
+ *   sx  = per row i, max over j not in O of |X[i,j]|, divided by 127 (float32)
+ *   Xq  = round(X / sx) on the regular columns, 0 on O   (ties to even, [-127,127])
+ *   Y   = fp16( (Xq . Wq^T)[i,n] * sx[i] * w_scale[n]         (int8 x int8 -> int32)
+ *               + sum_{j in O} X[i,j] * W_hat[n,j]             (fp16 operands, fp32 sum)
+ *               + bias[n] )
+ * with W_hat = fp16(Wq * w_scale): the layer keeps no fp16 weights ([P5] section
+ * "如何在 PyTorch 2.9 中启用 LLM.int8 推理", has_fp16_weights=False).
+ *   X          [in]  binary16 [M, K]
+ *   Wq, w_scale[in]  from int8_quant_weight, int8 [N, K] and float32 [N]
+ *   bias       [in]  binary16 [N], or NULL for none
+ *   threshold  [in]  outlier threshold (the pages' default is 6.0); a negative value acts
+ *                    as 0 (every column holding a nonzero value is an outlier); +inf turns
+ *                    the fp16 term off; NaN is rejected
+ *   Y          [out] binary16 [M, N]
+ *   workspace  [in/out] ws_bytes >= int8_linear_workspace_size(M, N, K), 256-byte aligned
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+int int8_linear_forward(const void *X, int M, int K, const int8_t *Wq, const float *w_scale,
+                        const void *bias, int N, float threshold, void *Y, void *workspace,
+                        size_t ws_bytes, int8mm_stream_t stream);
+
+/*
+ * Diagnostic: the quantization half of the layer alone (outlier detection and per-row
+ * activation quantization, [P2] section 2.3 and [P5] item 2, as in int8_linear_forward).
+ *   X            [in]  binary16 [M, K]
+ *   Xq           [out] int8     [M, K] (0 in outlier columns)
+ *   row_scale    [out] float32  [M]
+ *   outlier_cols [out] int32    [K]: the outlier columns in ascending order, first
+ *                      *n_outliers entries valid
+ *   n_outliers   [out] int32    [1] (device memory)
+ *   workspace    as for int8_linear_forward with N = 1
+ */
+int int8_quantize_rows(const void *X, int M, int K, float threshold, int8_t *Xq,
+                       float *row_scale, int32_t *outlier_cols, int32_t *n_outliers,
+                       void *workspace, size_t ws_bytes, int8mm_stream_t stream);
+
+/*
+ * Diagnostic: the int8 product alone, C[i,n] = sum_k Xq[i,k] * Wq[n,k], exact int32
+ * (the int8 matrix multiplication of [P2] section 2.3, run on the tensor cores).
+ *   Xq [in] int8 [M, K];  Wq [in] int8 [N, K];  C [out] int32 [M, N]
+ *   dev_status [in/out] one int32 of device memory that receives a negative code if a
+ *              bounded wait gives up (zero it before the first call)
+ */
+int int8_gemm_i32(const int8_t *Xq, const int8_t *Wq, int M, int N, int K, int32_t *C,
+                  int32_t *dev_status, int8mm_stream_t stream);
+
+/*
+ * Diagnostic: the fp16 outlier weights alone,
+ *   W_hat[n, r] = fp16(float(Wq[n, cols[r]]) * w_scale[n])   for r < *n_outliers
+ * (the layer keeps no fp16 weights: [P5] section "如何在 PyTorch 2.9 中启用 LLM.int8 推理",
+ * has_fp16_weights=False).  The product is rounded to float32, then to binary16 (ties to
+ * even).
+ *   outlier_cols, n_outliers [in] device int32, as written by int8_quantize_rows
+ *   W_hat [out] binary16 [N, K] with row stride K; entries r >= *n_outliers are untouched
+ */
+int int8_outlier_weights(const int8_t *Wq, const float *w_scale, int N, int K,
+                         const int32_t *outlier_cols, const int32_t *n_outliers, void *W_hat,
+                         int8mm_stream_t stream);
+
+/*
+ * Waits for `stream`, then returns the device status word at dev_status (for the forward
+ * and int8_quantize_rows, the word is the first int32 of the workspace): 0, or the
+ * negative code a kernel wrote.  Returns INT8MM_ERR_CUDA if the stream itself failed.
+ */
+int int8_read_device_status(const int32_t *dev_status, int8mm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,250 @@
+"""B200 (sm_100a) LLM.int8() linear layer: a thin Python binding over libint8mm.so.
+
+Every computation runs in the library's CUDA kernels; this module only marshals torch
+tensors (device memory and the current stream) into the C ABI of include/int8mm.h and
+raises on a nonzero status.  There is no CPU fallback: if the library has not been
+built, importing the binding's functions raises.
+
+Functions keep the C names:
+    int8_quant_weight, int8_linear_workspace_size, int8_linear_forward,
+    int8_quantize_rows, int8_gemm_i32, int8_outlier_weights, int8_read_device_status,
+    int8_status_string
+and ``Int8Linear`` bundles them the way the pages use the layer
+(``Linear8bitLt(in, out, bias, has_fp16_weights=False, threshold=6.0)``).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "Int8mmError", "load_library", "library_path",
+    "int8_quant_weight", "int8_linear_workspace_size", "int8_linear_forward",
+    "int8_quantize_rows", "int8_gemm_i32", "int8_outlier_weights",
+    "int8_read_device_status", "int8_status_string", "Int8Linear", "DEFAULT_THRESHOLD",
+]
+
+DEFAULT_THRESHOLD = 6.0
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libint8mm.so")
+_lib = None
+_lock = threading.Lock()
+
+
+class Int8mmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: status {status} ({int8_status_string(status)})")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libint8mm.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                              "`python -m int8_mixed_precision_absmax_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        p, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.int8_status_string.argtypes = [i]
+        lib.int8_status_string.restype = ctypes.c_char_p
+        lib.int8_quant_weight.argtypes = [p, i, i, p, p, p]
+        lib.int8_linear_workspace_size.argtypes = [i, i, i]
+        lib.int8_linear_workspace_size.restype = sz
+        lib.int8_linear_forward.argtypes = [p, i, i, p, p, p, i, f, p, p, sz, p]
+        lib.int8_quantize_rows.argtypes = [p, i, i, f, p, p, p, p, p, sz, p]
+        lib.int8_gemm_i32.argtypes = [p, p, i, i, i, p, p, p]
+        lib.int8_outlier_weights.argtypes = [p, p, i, i, p, p, p, p]
+        lib.int8_read_device_status.argtypes = [p, p]
+        for name in ("int8_quant_weight", "int8_linear_forward", "int8_quantize_rows",
+                     "int8_gemm_i32", "int8_outlier_weights", "int8_read_device_status"):
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def int8_status_string(status: int) -> str:
+    return load_library().int8_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise Int8mmError(status, what)
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, dims: int | None = None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dims is not None and t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dimensions")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def int8_linear_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load_library().int8_linear_workspace_size(M, N, K))
+
+
+def new_workspace(M: int, N: int, K: int, device) -> torch.Tensor:
+    """A zeroed workspace tensor (uint8) for an [M,K] x [N,K]^T layer."""
+    n = int8_linear_workspace_size(M, N, K)
+    if n == 0:
+        raise ValueError(f"unsupported layer shape M={M} N={N} K={K}")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def int8_quant_weight(W: torch.Tensor, Wq: torch.Tensor | None = None,
+                      w_scale: torch.Tensor | None = None, stream=None):
+    """Per-output-channel int8 weights and float32 scales of an fp16 [N, K] weight."""
+    _need(W, torch.float16, "W", 2)
+    N, K = W.shape
+    if Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if w_scale is None:
+        w_scale = torch.empty(N, dtype=torch.float32, device=W.device)
+    _need(Wq, torch.int8, "Wq", 2)
+    _need(w_scale, torch.float32, "w_scale", 1)
+    _check(load_library().int8_quant_weight(_ptr(W), N, K, _ptr(Wq), _ptr(w_scale),
+                                            ctypes.c_void_p(_stream(stream, W.device))),
+           "int8_quant_weight")
+    return Wq, w_scale
+
+
+def int8_linear_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                        bias: torch.Tensor | None, threshold: float = DEFAULT_THRESHOLD,
+                        Y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """Y = LLM.int8()(X, Wq, w_scale, bias, threshold), fp16 [M, N]."""
+    _need(X, torch.float16, "X", 2)
+    _need(Wq, torch.int8, "Wq", 2)
+    _need(w_scale, torch.float32, "w_scale", 1)
+    M, K = X.shape
+    N = Wq.shape[0]
+    if bias is not None:
+        _need(bias, torch.float16, "bias", 1)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    _need(Y, torch.float16, "Y", 2)
+    if workspace is None:
+        workspace = new_workspace(M, N, K, X.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    _check(load_library().int8_linear_forward(
+        _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(bias), N, float(threshold), _ptr(Y),
+        _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream, X.device))),
+        "int8_linear_forward")
+    return Y
+
+
+def int8_quantize_rows(X: torch.Tensor, threshold: float = DEFAULT_THRESHOLD,
+                       workspace: torch.Tensor | None = None, stream=None):
+    """(Xq int8 [M,K], row_scale f32 [M], outlier_cols i32 [K], n_outliers i32 [1]) on device.
+
+    Only the first n_outliers entries of outlier_cols are meaningful."""
+    _need(X, torch.float16, "X", 2)
+    M, K = X.shape
+    dev = X.device
+    Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sx = torch.empty(M, dtype=torch.float32, device=dev)
+    cols = torch.empty(K, dtype=torch.int32, device=dev)
+    n = torch.zeros(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(M, 1, K, dev)
+    _check(load_library().int8_quantize_rows(
+        _ptr(X), M, K, float(threshold), _ptr(Xq), _ptr(sx), _ptr(cols), _ptr(n),
+        _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream, dev))),
+        "int8_quantize_rows")
+    return Xq, sx, cols, n
+
+
+def int8_gemm_i32(Xq: torch.Tensor, Wq: torch.Tensor, C: torch.Tensor | None = None,
+                  dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """C = Xq . Wq^T exactly, int32 [M, N], on the tensor cores."""
+    _need(Xq, torch.int8, "Xq", 2)
+    _need(Wq, torch.int8, "Wq", 2)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=Xq.device)
+    _check(load_library().int8_gemm_i32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(C), _ptr(dev_status),
+                                        ctypes.c_void_p(_stream(stream, Xq.device))),
+           "int8_gemm_i32")
+    return C
+
+
+def int8_outlier_weights(Wq: torch.Tensor, w_scale: torch.Tensor, cols: torch.Tensor,
+                         n_outliers: torch.Tensor, W_hat: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """fp16 [N, K] whose first n_outliers columns are fp16(Wq[:, cols] * w_scale)."""
+    _need(Wq, torch.int8, "Wq", 2)
+    N, K = Wq.shape
+    if W_hat is None:
+        W_hat = torch.zeros((N, K), dtype=torch.float16, device=Wq.device)
+    _check(load_library().int8_outlier_weights(
+        _ptr(Wq), _ptr(w_scale), N, K, _ptr(cols), _ptr(n_outliers), _ptr(W_hat),
+        ctypes.c_void_p(_stream(stream, Wq.device))), "int8_outlier_weights")
+    return W_hat
+
+
+def int8_read_device_status(dev_status: torch.Tensor, stream=None) -> int:
+    """Wait for the stream and return the device status word (0 or a negative code)."""
+    return int(load_library().int8_read_device_status(
+        _ptr(dev_status), ctypes.c_void_p(_stream(stream, dev_status.device))))
+
+
+class Int8Linear:
+    """An LLM.int8() linear layer holding int8 weights only (no fp16 copy).
+
+    Mirrors ``Linear8bitLt(in_features, out_features, bias, has_fp16_weights=False,
+    threshold)``: the fp16 weight is quantized once per output channel at construction,
+    then every call quantizes its activations per row on the fly and routes the columns
+    whose magnitude exceeds ``threshold`` through fp16.
+    """
+
+    def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None,
+                 threshold: float = DEFAULT_THRESHOLD):
+        if math.isnan(threshold):
+            raise ValueError("threshold is NaN")
+        self.out_features, self.in_features = weight.shape
+        self.Wq, self.w_scale = int8_quant_weight(weight.contiguous())
+        self.bias = None if bias is None else bias.to(torch.float16).contiguous()
+        self.threshold = float(threshold)
+        self._workspace = None
+        self._ws_rows = 0
+
+    def _ws(self, M: int, device) -> torch.Tensor:
+        if self._workspace is None or self._ws_rows < M:
+            self._workspace = new_workspace(M, self.out_features, self.in_features, device)
+            self._ws_rows = M
+        return self._workspace
+
+    def __call__(self, X: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+        lead = X.shape[:-1]
+        X2 = X.reshape(-1, self.in_features).contiguous()
+        ws = self._ws(X2.shape[0], X2.device)
+        Y = int8_linear_forward(X2, self.Wq, self.w_scale, self.bias, self.threshold, Y=out,
+                                workspace=ws)
+        return Y.reshape(*lead, self.out_features)

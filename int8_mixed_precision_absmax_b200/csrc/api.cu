@@ -1,0 +1,225 @@
+// api.cu -- the extern "C" entry points of libint8mm.so (declared in include/int8mm.h):
+// argument checks, workspace carving, tensor-map encoding and kernel launches.  No entry
+// point allocates memory or synchronizes, except int8_read_device_status (documented).
+#include <cmath>
+#include <cstdint>
+
+#include "kernels.cuh"
+
+using namespace i8mm;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+int check_shape(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0 || K > INT8MM_MAX_K) return INT8MM_ERR_SHAPE;
+  if (K % 16 != 0) return INT8MM_ERR_ALIGN;
+  return INT8MM_OK;
+}
+
+// The kernels are built for sm_100a only.
+int check_device() {
+  static int checked_device = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return INT8MM_ERR_CUDA;
+  if (dev == checked_device) return INT8MM_OK;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return INT8MM_ERR_CUDA;
+  if (major != 10 || minor != 0) return INT8MM_ERR_DEVICE;
+  checked_device = dev;
+  return INT8MM_OK;
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? INT8MM_OK : INT8MM_ERR_CUDA; }
+
+float effective_threshold(float t) { return t < 0.0f ? 0.0f : t; }
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* int8_status_string(int status) {
+  switch (status) {
+    case INT8MM_OK: return "ok";
+    case INT8MM_ERR_NULL: return "a required pointer is NULL";
+    case INT8MM_ERR_SHAPE: return "M, N or K out of range";
+    case INT8MM_ERR_ALIGN: return "K is not a multiple of 16 or a pointer is not 16-byte aligned";
+    case INT8MM_ERR_THRESHOLD: return "threshold is NaN";
+    case INT8MM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case INT8MM_ERR_CUDA: return "CUDA runtime or launch error";
+    case INT8MM_ERR_DEVICE: return "the current device is not sm_100";
+    case INT8MM_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case INT8MM_ERR_OVERFLOW: return "outlier count out of range";
+    default: return "unknown status";
+  }
+}
+
+int int8_quant_weight(const void* W, int N, int K, int8_t* Wq, float* w_scale,
+                      int8mm_stream_t stream) {
+  if (!W || !Wq || !w_scale) return INT8MM_ERR_NULL;
+  int rc = check_shape(1, N, K);
+  if (rc) return rc;
+  if (!aligned16(W) || !aligned16(Wq) || !aligned16(w_scale)) return INT8MM_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_status(launch_quant_weight(static_cast<const __half*>(W), N, K, Wq, w_scale,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t int8_linear_workspace_size(int M, int N, int K) {
+  if (check_shape(M, N, K) != INT8MM_OK) return 0;
+  return workspace_layout(M, N, K).total;
+}
+
+int int8_linear_forward(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+                        const void* bias, int N, float threshold, void* Y, void* workspace,
+                        size_t ws_bytes, int8mm_stream_t stream_) {
+  if (!X || !Wq || !w_scale || !Y) return INT8MM_ERR_NULL;
+  int rc = check_shape(M, N, K);
+  if (rc) return rc;
+  if (!aligned16(X) || !aligned16(Wq) || !aligned16(w_scale) || !aligned16(Y) ||
+      (bias && !aligned16(bias)))
+    return INT8MM_ERR_ALIGN;
+  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
+  const WorkspaceLayout L = workspace_layout(M, N, K);
+  if (!workspace || !aligned256(workspace) || ws_bytes < L.total) return INT8MM_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+
+  int32_t* header = at<int32_t>(workspace, L.header);
+  uint32_t* mask = at<uint32_t>(workspace, L.mask);
+  int8_t* xq = at<int8_t>(workspace, L.xq);
+  float* xscale = at<float>(workspace, L.xscale);
+  __half* xo = at<__half>(workspace, L.xo);
+  __half* wo = at<__half>(workspace, L.wo);
+
+  GemmMaps maps;
+  if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, M, K, kBKBytes, kBM) ||
+      !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kBN) ||
+      !encode_tmap_2d(&maps.xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xo, L.ldo, M, L.ldo * 2ull,
+                      kBKBytes / 2, kBM) ||
+      !encode_tmap_2d(&maps.wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, L.ldo, N, L.ldo * 2ull,
+                      kBKBytes / 2, kBN))
+    return INT8MM_ERR_CUDA;
+
+  if ((rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
+                                         effective_threshold(threshold), mask, stream, true))))
+    return rc;
+  RowQuantArgs rq;
+  rq.X = static_cast<const __half*>(X);
+  rq.M = M;
+  rq.K = K;
+  rq.mask = mask;
+  rq.xq = xq;
+  rq.xscale = xscale;
+  rq.xo = xo;
+  rq.ldo = L.ldo;
+  rq.cols = at<int32_t>(workspace, L.cols);
+  rq.n_out = header + 1;
+  rq.Wq = Wq;
+  rq.w_scale = w_scale;
+  rq.wo = wo;
+  rq.N = N;
+  rq.status = header;
+  if ((rc = launch_status(launch_rowquant(rq, stream, true)))) return rc;
+  GemmArgs g;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.xscale = xscale;
+  g.w_scale = w_scale;
+  g.bias = static_cast<const __half*>(bias);
+  g.Y = static_cast<__half*>(Y);
+  g.C = nullptr;
+  g.n_out = header + 1;
+  g.status = header;
+  return launch_status(launch_gemm(maps, g, stream, true));
+}
+
+int int8_quantize_rows(const void* X, int M, int K, float threshold, int8_t* Xq,
+                       float* row_scale, int32_t* outlier_cols, int32_t* n_outliers,
+                       void* workspace, size_t ws_bytes, int8mm_stream_t stream_) {
+  if (!X || !Xq || !row_scale || !outlier_cols || !n_outliers) return INT8MM_ERR_NULL;
+  int rc = check_shape(M, 1, K);
+  if (rc) return rc;
+  if (!aligned16(X) || !aligned16(Xq)) return INT8MM_ERR_ALIGN;
+  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
+  const WorkspaceLayout L = workspace_layout(M, 1, K);
+  if (!workspace || !aligned256(workspace) || ws_bytes < L.total) return INT8MM_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  uint32_t* mask = at<uint32_t>(workspace, L.mask);
+  if ((rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
+                                         effective_threshold(threshold), mask, stream, false))))
+    return rc;
+  RowQuantArgs rq = {};
+  rq.X = static_cast<const __half*>(X);
+  rq.M = M;
+  rq.K = K;
+  rq.mask = mask;
+  rq.xq = Xq;
+  rq.xscale = row_scale;
+  rq.xo = nullptr;
+  rq.ldo = L.ldo;
+  rq.cols = outlier_cols;
+  rq.n_out = n_outliers;
+  rq.wo = nullptr;
+  rq.status = at<int32_t>(workspace, L.header);
+  return launch_status(launch_rowquant(rq, stream, true));
+}
+
+int int8_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K, int32_t* C,
+                  int32_t* dev_status, int8mm_stream_t stream_) {
+  if (!Xq || !Wq || !C || !dev_status) return INT8MM_ERR_NULL;
+  int rc = check_shape(M, N, K);
+  if (rc) return rc;
+  if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(C)) return INT8MM_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  GemmMaps maps;
+  if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K, M, K, kBKBytes, kBM) ||
+      !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kBN))
+    return INT8MM_ERR_CUDA;
+  maps.xo = maps.xq;  // unused: no outlier columns
+  maps.wo = maps.wq;
+  GemmArgs g = {};
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.C = C;
+  g.n_out = nullptr;
+  g.status = dev_status;
+  return launch_status(launch_gemm(maps, g, reinterpret_cast<cudaStream_t>(stream_), false));
+}
+
+int int8_outlier_weights(const int8_t* Wq, const float* w_scale, int N, int K,
+                         const int32_t* outlier_cols, const int32_t* n_outliers, void* W_hat,
+                         int8mm_stream_t stream) {
+  if (!Wq || !w_scale || !outlier_cols || !n_outliers || !W_hat) return INT8MM_ERR_NULL;
+  int rc = check_shape(1, N, K);
+  if (rc) return rc;
+  if (!aligned16(Wq) || !aligned16(W_hat)) return INT8MM_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_status(launch_outlier_weights(Wq, w_scale, N, K, outlier_cols, n_outliers,
+                                              static_cast<__half*>(W_hat),
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int int8_read_device_status(const int32_t* dev_status, int8mm_stream_t stream) {
+  if (!dev_status) return INT8MM_ERR_NULL;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return INT8MM_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, dev_status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return INT8MM_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

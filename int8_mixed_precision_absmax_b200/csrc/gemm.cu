@@ -1,0 +1,328 @@
+// gemm.cu -- the tensor-core half of the LLM.int8() layer on sm_100a.
+//
+// One persistent, warp-specialised kernel computes, per 128 x 256 output tile,
+//   A = Xq . Wq^T         int8 x int8 -> int32   tcgen05.mma kind::i8, TMEM accumulator
+//   P = X_O . W_hat_O^T   fp16 x fp16 -> fp32    tcgen05.mma kind::f16, second accumulator
+// and the fused epilogue Y = fp16(A * sx[i] * w_scale[n] + P + bias[n])
+// ([P2] "8位量化实战：离群值处理与显存优化避坑指南" section 2.3: the int8 and fp16 products
+// are computed separately and summed; [P5] "PyTorch 2.9 支持 LLM.int8()" item 3: the
+// results are merged at the end).  The dequantization by the outer product of the row
+// and column scales undoes x ~ q * sx and w ~ q * w_scale of [P5] items 1 and 2.
+//
+// Roles (192 threads): warp 0 issues TMA loads into a 4-stage shared-memory ring, warp 1
+// allocates tensor memory and issues the MMAs (one thread), warps 2-5 drain the
+// accumulators (each warp owns the 32 TMEM lanes of its quadrant).  With both products
+// present the 512 TMEM columns hold one int32 and one fp32 accumulator; with only one of
+// them, two accumulator slots alternate so the epilogue of a tile overlaps the next
+// tile's main loop.  Every wait is bounded (ptx.cuh); a wait that gives up writes
+// INT8MM_ERR_TIMEOUT to the status word, and the block drains its in-flight copies and
+// MMAs, frees its tensor memory and exits.
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace i8mm {
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBKBytes;  // 16 KB
+constexpr int kBBytes = kBN * kBKBytes;  // 32 KB
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kIdescI8 = idesc_i8_s32(kBM, kBN);
+constexpr uint32_t kIdescF16 = idesc_f16_f32(kBM, kBN);
+
+struct GemmShared {
+  uint8_t a[kStages][kABytes];
+  uint8_t b[kStages][kBBytes];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemBytes = sizeof(GemmShared) + 1024;  // + alignment slack
+
+struct TileSchedule {
+  int m_tiles, tiles;
+  __device__ void coords(int tile, int& m0, int& n0) const {
+    m0 = (tile % m_tiles) * kBM;  // consecutive blocks share the weight tile
+    n0 = (tile / m_tiles) * kBN;
+  }
+};
+
+__device__ __forceinline__ void report(int32_t* status, int code) {
+  if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
+}
+
+__device__ __forceinline__ void store_half32(__half* dst, const float (&y)[32], int valid,
+                                             bool vec_ok) {
+  if (vec_ok && valid == 32) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __half2 h = __floats2half2_rn(y[v * 8 + 2 * e], y[v * 8 + 2 * e + 1]);
+        w[e] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(dst)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < valid) dst[j] = __float2half_rn(y[j]);
+  }
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
+                const __grid_constant__ CUtensorMap map_xo, const __grid_constant__ CUtensorMap map_wo,
+                const GemmArgs args) {
+  extern __shared__ uint8_t gemm_smem_raw[];
+  GemmShared& S = *reinterpret_cast<GemmShared*>(
+      (reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.tmem_full[b], 1);
+      mbar_init(&S.tmem_empty[b], 128);
+    }
+    mbar_init(&S.drain, 1);
+    S.abort = 0;
+    fence_mbarrier_init();
+  }
+  if (threadIdx.x == 32) {
+    prefetch_tmap(&map_xq);
+    prefetch_tmap(&map_wq);
+    prefetch_tmap(&map_xo);
+    prefetch_tmap(&map_wo);
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // Everything above overlaps the previous kernel; inputs are read only after this.
+  grid_dependency_wait();
+
+  const int M = args.M, N = args.N, K = args.K;
+  const int n_out = args.n_out ? *args.n_out : 0;
+  const int kb_i8 = (n_out >= K) ? 0 : (K + kBKBytes - 1) / kBKBytes;  // Xq == 0 if all outliers
+  const int kb_f16 = (n_out + 63) / 64;
+  const int kb_total = kb_i8 + kb_f16;
+  const bool both = kb_i8 > 0 && kb_f16 > 0;
+  const int nslots = both ? 1 : 2;
+  TileSchedule sched;
+  sched.m_tiles = (M + kBM - 1) / kBM;
+  sched.tiles = sched.m_tiles * ((N + kBN - 1) / kBN);
+  const uint32_t tmem = S.tmem_base;
+  volatile int* abort = &S.abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ producer: TMA into the ring
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < sched.tiles; tile += gridDim.x) {
+        int m0, n0;
+        sched.coords(tile, m0, n0);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait_bounded(&S.empty[stage], phase ^ 1u, abort)) { ok = false; break; }
+          mbar_arrive_expect_tx(&S.full[stage], kABytes + kBBytes);
+          if (kb < kb_i8) {
+            tma_load_2d(&map_xq, S.a[stage], &S.full[stage], kb * kBKBytes, m0);
+            tma_load_2d(&map_wq, S.b[stage], &S.full[stage], kb * kBKBytes, n0);
+          } else {
+            const int k = (kb - kb_i8) * 64;
+            tma_load_2d(&map_xo, S.a[stage], &S.full[stage], k, m0);
+            tma_load_2d(&map_wo, S.b[stage], &S.full[stage], k, n0);
+          }
+          ++issued;
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // let every issued copy land before the block can exit (bounded, abort ignored)
+      int dummy = 0;
+      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+        mbar_wait_bounded(&S.full[j % kStages], static_cast<uint32_t>(j / kStages) & 1u, &dummy);
+      if (!ok) report(args.status, INT8MM_ERR_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < sched.tiles; tile += gridDim.x, ++it) {
+        const int slot = (nslots == 1) ? 0 : (it & 1);
+        const uint32_t use = (nslots == 1) ? it : (it >> 1);
+        if (!mbar_wait_bounded(&S.tmem_empty[slot], (use & 1u) ^ 1u, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_i8 = tmem + (both ? 0u : slot * 256u);
+        const uint32_t d_f32 = tmem + (both ? 256u : slot * 256u);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait_bounded(&S.full[stage], phase, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_addr(S.a[stage]);
+          const uint32_t b0 = smem_addr(S.b[stage]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // 4 x 32 bytes along K per stage
+            const uint64_t ad = sw128_kmajor_desc(a0 + 32u * k);
+            const uint64_t bd = sw128_kmajor_desc(b0 + 32u * k);
+            if (kb < kb_i8)
+              mma_i8(d_i8, ad, bd, kIdescI8, (kb > 0 || k > 0) ? 1u : 0u);
+            else
+              mma_f16(d_f32, ad, bd, kIdescF16, (kb > kb_i8 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&S.empty[stage]);  // frees the stage once these MMAs have read it
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&S.tmem_full[slot]);
+      }
+      // every MMA issued so far must finish before tensor memory is freed
+      mma_commit(&S.drain);
+      int dummy = 0;
+      mbar_wait_bounded(&S.drain, 0, &dummy);
+      if (!ok) report(args.status, INT8MM_ERR_TIMEOUT);
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2..5)
+    const int quad = warp & 3;
+    const bool vec_ok = (N % 8) == 0;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < sched.tiles; tile += gridDim.x, ++it) {
+      const int slot = (nslots == 1) ? 0 : (it & 1);
+      const uint32_t use = (nslots == 1) ? it : (it >> 1);
+      if (!mbar_wait_bounded(&S.tmem_full[slot], use & 1u, abort)) {
+        report(args.status, INT8MM_ERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      int m0, n0;
+      sched.coords(tile, m0, n0);
+      const int row = m0 + quad * 32 + lane;
+      const bool row_ok = row < M;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+      const uint32_t t_i8 = lane_base + (both ? 0u : slot * 256u);
+      const uint32_t t_f32 = lane_base + (both ? 256u : slot * 256u);
+      const float sx = (args.Y && row_ok) ? args.xscale[row] : 0.0f;
+      for (int c = 0; c < kBN; c += 32) {
+        uint32_t ra[32], rp[32];
+        __syncwarp();  // the tensor-memory loads are warp-collective
+        if (kb_i8 > 0) tmem_ld_32x32b_x32(t_i8 + c, ra);
+        if (kb_f16 > 0) tmem_ld_32x32b_x32(t_f32 + c, rp);
+        tmem_ld_wait();
+        const int n = n0 + c;
+        const int valid = min(32, N - n);
+        if (!row_ok || valid <= 0) {
+        } else if (args.C) {
+          int32_t* dst = args.C + static_cast<size_t>(row) * N + n;
+          if (valid == 32 && (N % 4) == 0) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              reinterpret_cast<int4*>(dst)[v] =
+                  make_int4(kb_i8 ? ra[4 * v] : 0, kb_i8 ? ra[4 * v + 1] : 0,
+                            kb_i8 ? ra[4 * v + 2] : 0, kb_i8 ? ra[4 * v + 3] : 0);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < valid) dst[j] = kb_i8 ? static_cast<int32_t>(ra[j]) : 0;
+          }
+        } else {
+          float y[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int nn = min(n + j, N - 1);
+            float acc = 0.0f;
+            if (kb_i8 > 0) acc = static_cast<float>(static_cast<int32_t>(ra[j])) * sx * args.w_scale[nn];
+            if (kb_f16 > 0) acc += __uint_as_float(rp[j]);
+            if (args.bias) acc += __half2float(args.bias[nn]);
+            y[j] = acc;
+          }
+          store_half32(args.Y + static_cast<size_t>(row) * N + n, y, valid, vec_ok);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&S.tmem_empty[slot]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                    uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
+                    uint32_t box_inner, uint32_t box_outer) {
+  using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn encode = nullptr;
+  if (encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return false;
+    encode = reinterpret_cast<EncodeFn>(fn);
+  }
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  return encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream, bool pdl) {
+  static int configured_device = -1;
+  static int num_sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (configured_device != dev) {
+    e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  const int tiles = ((a.M + kBM - 1) / kBM) * ((a.N + kBN - 1) / kBN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles < num_sms ? tiles : num_sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemm_kernel, maps.xq, maps.wq, maps.xo, maps.wo, a);
+}
+
+}  // namespace i8mm

@@ -1,0 +1,105 @@
+// kernels.cuh -- internal interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "int8mm.h"
+
+namespace i8mm {
+
+// ---------------------------------------------------------------- workspace layout
+//
+// One contiguous device buffer, every region 256-byte aligned:
+//   header   int32[64]      [0] status word, [1] outlier count
+//   mask     uint32[ceil(K/32)]    bit j%32 of word j/32 set <=> column j is an outlier
+//   cols     int32[K]       outlier columns, ascending
+//   xscale   float[M]       per-row activation scale
+//   xq       int8[M*K]      quantized activations (0 in outlier columns)
+//   xo       half[M*ldo]    outlier activations, compacted, zero-padded to a multiple of 64
+//   wo       half[N*ldo]    outlier weights fp16(Wq*w_scale), compacted, zero-padded
+// ldo = K rounded up to 64 (the fp16 operand tiles are 64 elements deep).
+struct WorkspaceLayout {
+  size_t header, mask, cols, xscale, xq, xo, wo, total;
+  int ldo;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+inline WorkspaceLayout workspace_layout(int M, int N, int K) {
+  WorkspaceLayout L;
+  L.ldo = (K + 63) / 64 * 64;
+  size_t off = 0;
+  L.header = off; off = align256(off + 64 * sizeof(int32_t));
+  L.mask = off;   off = align256(off + static_cast<size_t>((K + 31) / 32) * sizeof(uint32_t));
+  L.cols = off;   off = align256(off + static_cast<size_t>(K) * sizeof(int32_t));
+  L.xscale = off; off = align256(off + static_cast<size_t>(M) * sizeof(float));
+  L.xq = off;     off = align256(off + static_cast<size_t>(M) * K);
+  L.xo = off;     off = align256(off + static_cast<size_t>(M) * L.ldo * sizeof(__half));
+  L.wo = off;     off = align256(off + static_cast<size_t>(N) * L.ldo * sizeof(__half));
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- launches
+// Each returns cudaSuccess or the launch error; `pdl` lets the launch start while the
+// previous kernel on the stream drains (the kernel waits on griddepcontrol before
+// touching its inputs).
+
+cudaError_t launch_quant_weight(const __half* W, int N, int K, int8_t* Wq, float* w_scale,
+                                cudaStream_t stream);
+
+cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint32_t* mask,
+                           cudaStream_t stream, bool pdl);
+
+cudaError_t launch_outlier_weights(const int8_t* Wq, const float* w_scale, int N, int K,
+                                   const int32_t* cols, const int32_t* n_out, __half* W_hat,
+                                   cudaStream_t stream);
+
+struct RowQuantArgs {
+  const __half* X;
+  int M, K;
+  const uint32_t* mask;
+  int8_t* xq;
+  float* xscale;
+  __half* xo;           // nullable: skip the outlier-activation gather
+  int ldo;
+  int32_t* cols;        // written by block 0
+  int32_t* n_out;       // written by block 0
+  // outlier-weight gather (extra blocks after the M row blocks); wo nullable
+  const int8_t* Wq;
+  const float* w_scale;
+  __half* wo;
+  int N;
+  int32_t* status;
+};
+cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl);
+
+struct GemmArgs {
+  int M, N, K;
+  const float* xscale;   // [M]
+  const float* w_scale;  // [N]
+  const __half* bias;    // [N] or null
+  __half* Y;             // fused epilogue output [M,N], or null
+  int32_t* C;            // raw int32 output [M,N], or null (exactly one of Y, C)
+  const int32_t* n_out;  // device outlier count, or null for none
+  int32_t* status;
+};
+struct GemmMaps {
+  CUtensorMap xq, wq, xo, wo;
+};
+// Host-side tensor-map encoding (driver entry point fetched through the runtime).
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                    uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
+                    uint32_t box_inner, uint32_t box_outer);
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream, bool pdl);
+
+// GEMM tile shape (shared with the host for map boxes)
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBKBytes = 128;  // one 128-byte swizzle row: 128 int8 or 64 fp16 per stage
+
+}  // namespace i8mm

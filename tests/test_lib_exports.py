@@ -1,0 +1,89 @@
+"""The C-ABI library builds, loads without a GPU and exports every declared entry point.
+
+No compute call is made here: only host-side queries and argument checks that return
+before any device work (the pointers passed are never dereferenced).
+"""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import int8_mixed_precision_absmax_b200 as i8
+from int8_mixed_precision_absmax_b200 import build as lib_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "int8mm.h")
+FAKE = ctypes.c_void_p(0x10000)  # aligned, never dereferenced: validation fails first
+
+
+def declared_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(int8_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lib_build.build()
+    return i8.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("int8_quant_weight", "int8_linear_forward", "int8_linear_workspace_size",
+                     "int8_quantize_rows", "int8_gemm_i32", "int8_outlier_weights",
+                     "int8_read_device_status", "int8_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(-9, 1):
+        assert i8.int8_status_string(code) not in ("", "unknown status")
+    assert i8.int8_status_string(-1234) == "unknown status"
+
+
+def test_workspace_size_is_worst_case_and_rejects_bad_shapes(lib):
+    M, N, K = 2048, 11008, 4096
+    ws = i8.int8_linear_workspace_size(M, N, K)
+    # at least: Xq (M*K) + fp16 outlier activations (M*K*2) + fp16 outlier weights (N*K*2)
+    assert ws >= M * K + 2 * M * K + 2 * N * K
+    assert i8.int8_linear_workspace_size(16, 16, 40) == 0      # K % 16 != 0
+    assert i8.int8_linear_workspace_size(0, 16, 32) == 0
+    assert i8.int8_linear_workspace_size(16, 16, 65536 + 16) == 0
+
+
+def test_argument_checks_need_no_device(lib):
+    L = lib
+    null = None
+    # NULL pointers
+    assert L.int8_linear_forward(null, 4, 32, FAKE, FAKE, null, 8, 6.0, FAKE, FAKE, 1 << 20,
+                                 null) == -1
+    # shapes
+    assert L.int8_linear_forward(FAKE, 0, 32, FAKE, FAKE, null, 8, 6.0, FAKE, FAKE, 1 << 20,
+                                 null) == -2
+    assert L.int8_linear_forward(FAKE, 4, 40, FAKE, FAKE, null, 8, 6.0, FAKE, FAKE, 1 << 20,
+                                 null) == -3
+    # misaligned pointer
+    assert L.int8_linear_forward(ctypes.c_void_p(0x10002), 4, 32, FAKE, FAKE, null, 8, 6.0, FAKE,
+                                 FAKE, 1 << 20, null) == -3
+    # NaN threshold
+    assert L.int8_linear_forward(FAKE, 4, 32, FAKE, FAKE, null, 8, math.nan, FAKE, FAKE,
+                                 1 << 20, null) == -4
+    # workspace too small / misaligned
+    assert L.int8_linear_forward(FAKE, 4, 32, FAKE, FAKE, null, 8, 6.0, FAKE, FAKE, 16,
+                                 null) == -5
+    assert L.int8_linear_forward(FAKE, 4, 32, FAKE, FAKE, null, 8, 6.0, FAKE,
+                                 ctypes.c_void_p(0x10010), 1 << 20, null) == -5
+    assert L.int8_gemm_i32(FAKE, FAKE, 4, 8, 40, FAKE, FAKE, null) == -3
+    assert L.int8_gemm_i32(FAKE, FAKE, 4, 8, 32, FAKE, null, null) == -1
+    assert L.int8_quant_weight(FAKE, 8, 0, FAKE, FAKE, null) == -2
+    assert L.int8_quantize_rows(FAKE, 4, 32, math.nan, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20,
+                                null) == -4
+    assert L.int8_read_device_status(null, null) == -1
