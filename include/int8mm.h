@@ -97,6 +97,26 @@ int int8_linear_forward(const void *X, int M, int K, const int8_t *Wq, const flo
                         size_t ws_bytes, int8mm_stream_t stream);
 
 /*
+ * The two halves of int8_linear_forward, for callers that time or schedule them apart
+ * (int8_linear_forward is exactly int8_linear_quantize followed by int8_linear_matmul on
+ * the same workspace and stream).
+ *
+ * int8_linear_quantize: the activation side -- outlier columns, per-row scales, int8
+ *   activations, and the compacted fp16 outlier operands (activations and
+ *   W_hat = fp16(Wq * w_scale)) -- written into the workspace.  Arguments as for
+ *   int8_linear_forward.
+ * int8_linear_matmul: the tensor-core side -- the int8 and fp16 products and the fused
+ *   epilogue -- reading the workspace the previous int8_linear_quantize call on the same
+ *   layer shape and weights filled.
+ */
+int int8_linear_quantize(const void *X, int M, int K, const int8_t *Wq, const float *w_scale,
+                         int N, float threshold, void *workspace, size_t ws_bytes,
+                         int8mm_stream_t stream);
+int int8_linear_matmul(int M, int K, const int8_t *Wq, const float *w_scale, const void *bias,
+                       int N, void *Y, void *workspace, size_t ws_bytes,
+                       int8mm_stream_t stream);
+
+/*
  * Diagnostic: the quantization half of the layer alone (outlier detection and per-row
  * activation quantization, [P2] section 2.3 and [P5] item 2, as in int8_linear_forward).
  *   X            [in]  binary16 [M, K]

@@ -79,69 +79,130 @@ size_t int8_linear_workspace_size(int M, int N, int K) {
   return workspace_layout(M, N, K).total;
 }
 
-int int8_linear_forward(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
-                        const void* bias, int N, float threshold, void* Y, void* workspace,
-                        size_t ws_bytes, int8mm_stream_t stream_) {
-  if (!X || !Wq || !w_scale || !Y) return INT8MM_ERR_NULL;
+}  // extern "C"
+
+namespace {
+
+struct ForwardPlan {
+  WorkspaceLayout L;
+  int32_t* header;
+  uint32_t* mask;
+  int8_t* xq;
+  float* xscale;
+  __half* xo;
+  __half* wo;
+};
+
+int plan_forward(int M, int N, int K, const int8_t* Wq, const float* w_scale, void* workspace,
+                 size_t ws_bytes, ForwardPlan& p) {
+  if (!Wq || !w_scale) return INT8MM_ERR_NULL;
   int rc = check_shape(M, N, K);
   if (rc) return rc;
-  if (!aligned16(X) || !aligned16(Wq) || !aligned16(w_scale) || !aligned16(Y) ||
-      (bias && !aligned16(bias)))
-    return INT8MM_ERR_ALIGN;
-  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
-  const WorkspaceLayout L = workspace_layout(M, N, K);
-  if (!workspace || !aligned256(workspace) || ws_bytes < L.total) return INT8MM_ERR_WORKSPACE;
+  if (!aligned16(Wq) || !aligned16(w_scale)) return INT8MM_ERR_ALIGN;
+  p.L = workspace_layout(M, N, K);
+  if (!workspace || !aligned256(workspace) || ws_bytes < p.L.total) return INT8MM_ERR_WORKSPACE;
   if ((rc = check_device())) return rc;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  p.header = at<int32_t>(workspace, p.L.header);
+  p.mask = at<uint32_t>(workspace, p.L.mask);
+  p.xq = at<int8_t>(workspace, p.L.xq);
+  p.xscale = at<float>(workspace, p.L.xscale);
+  p.xo = at<__half>(workspace, p.L.xo);
+  p.wo = at<__half>(workspace, p.L.wo);
+  return INT8MM_OK;
+}
 
-  int32_t* header = at<int32_t>(workspace, L.header);
-  uint32_t* mask = at<uint32_t>(workspace, L.mask);
-  int8_t* xq = at<int8_t>(workspace, L.xq);
-  float* xscale = at<float>(workspace, L.xscale);
-  __half* xo = at<__half>(workspace, L.xo);
-  __half* wo = at<__half>(workspace, L.wo);
-
-  GemmMaps maps;
-  if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, M, K, kBKBytes, kBM) ||
-      !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kBN) ||
-      !encode_tmap_2d(&maps.xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xo, L.ldo, M, L.ldo * 2ull,
-                      kBKBytes / 2, kBM) ||
-      !encode_tmap_2d(&maps.wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, L.ldo, N, L.ldo * 2ull,
-                      kBKBytes / 2, kBN))
-    return INT8MM_ERR_CUDA;
-
-  if ((rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
-                                         effective_threshold(threshold), mask, stream, true))))
-    return rc;
+int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale, int N,
+                 float threshold, void* workspace, const ForwardPlan& p, cudaStream_t stream,
+                 bool pdl_first) {
+  int rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
+                                        effective_threshold(threshold), p.mask, stream,
+                                        pdl_first));
+  if (rc) return rc;
   RowQuantArgs rq;
   rq.X = static_cast<const __half*>(X);
   rq.M = M;
   rq.K = K;
-  rq.mask = mask;
-  rq.xq = xq;
-  rq.xscale = xscale;
-  rq.xo = xo;
-  rq.ldo = L.ldo;
-  rq.cols = at<int32_t>(workspace, L.cols);
-  rq.n_out = header + 1;
+  rq.mask = p.mask;
+  rq.xq = p.xq;
+  rq.xscale = p.xscale;
+  rq.xo = p.xo;
+  rq.ldo = p.L.ldo;
+  rq.cols = at<int32_t>(workspace, p.L.cols);
+  rq.n_out = p.header + 1;
   rq.Wq = Wq;
   rq.w_scale = w_scale;
-  rq.wo = wo;
+  rq.wo = p.wo;
   rq.N = N;
-  rq.status = header;
-  if ((rc = launch_status(launch_rowquant(rq, stream, true)))) return rc;
+  rq.status = p.header;
+  return launch_status(launch_rowquant(rq, stream, true));
+}
+
+int run_matmul(int M, int K, const int8_t* Wq, const float* w_scale, const void* bias, int N,
+               void* Y, const ForwardPlan& p, cudaStream_t stream, bool pdl) {
+  GemmMaps maps;
+  if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.xq, K, M, K, kBKBytes, kBM) ||
+      !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kBN) ||
+      !encode_tmap_2d(&maps.xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.xo, p.L.ldo, M,
+                      p.L.ldo * 2ull, kBKBytes / 2, kBM) ||
+      !encode_tmap_2d(&maps.wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.wo, p.L.ldo, N,
+                      p.L.ldo * 2ull, kBKBytes / 2, kBN))
+    return INT8MM_ERR_CUDA;
   GemmArgs g;
   g.M = M;
   g.N = N;
   g.K = K;
-  g.xscale = xscale;
+  g.xscale = p.xscale;
   g.w_scale = w_scale;
   g.bias = static_cast<const __half*>(bias);
   g.Y = static_cast<__half*>(Y);
   g.C = nullptr;
-  g.n_out = header + 1;
-  g.status = header;
-  return launch_status(launch_gemm(maps, g, stream, true));
+  g.n_out = p.header + 1;
+  g.status = p.header;
+  return launch_status(launch_gemm(maps, g, stream, pdl));
+}
+
+}  // namespace
+
+extern "C" {
+
+int int8_linear_forward(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+                        const void* bias, int N, float threshold, void* Y, void* workspace,
+                        size_t ws_bytes, int8mm_stream_t stream_) {
+  if (!X || !Y) return INT8MM_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Y) || (bias && !aligned16(bias))) return INT8MM_ERR_ALIGN;
+  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
+  ForwardPlan p;
+  int rc = plan_forward(M, N, K, Wq, w_scale, workspace, ws_bytes, p);
+  if (rc) return rc;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if ((rc = run_quantize(X, M, K, Wq, w_scale, N, threshold, workspace, p, stream, true)))
+    return rc;
+  return run_matmul(M, K, Wq, w_scale, bias, N, Y, p, stream, true);
+}
+
+int int8_linear_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+                         int N, float threshold, void* workspace, size_t ws_bytes,
+                         int8mm_stream_t stream) {
+  if (!X) return INT8MM_ERR_NULL;
+  if (!aligned16(X)) return INT8MM_ERR_ALIGN;
+  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
+  ForwardPlan p;
+  int rc = plan_forward(M, N, K, Wq, w_scale, workspace, ws_bytes, p);
+  if (rc) return rc;
+  return run_quantize(X, M, K, Wq, w_scale, N, threshold, workspace, p,
+                      reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+int int8_linear_matmul(int M, int K, const int8_t* Wq, const float* w_scale, const void* bias,
+                       int N, void* Y, void* workspace, size_t ws_bytes,
+                       int8mm_stream_t stream) {
+  if (!Y) return INT8MM_ERR_NULL;
+  if (!aligned16(Y) || (bias && !aligned16(bias))) return INT8MM_ERR_ALIGN;
+  ForwardPlan p;
+  int rc = plan_forward(M, N, K, Wq, w_scale, workspace, ws_bytes, p);
+  if (rc) return rc;
+  return run_matmul(M, K, Wq, w_scale, bias, N, Y, p, reinterpret_cast<cudaStream_t>(stream),
+                    true);
 }
 
 int int8_quantize_rows(const void* X, int M, int K, float threshold, int8_t* Xq,
