@@ -97,24 +97,34 @@ int int8_linear_forward(const void *X, int M, int K, const int8_t *Wq, const flo
                         size_t ws_bytes, int8mm_stream_t stream);
 
 /*
- * The two halves of int8_linear_forward, for callers that time or schedule them apart
- * (int8_linear_forward is exactly int8_linear_quantize followed by int8_linear_matmul on
- * the same workspace and stream).
+ * The two halves of int8_linear_forward, for callers that time or schedule them apart:
+ * int8_linear_forward is exactly int8_linear_quantize followed by int8_linear_matmul with
+ * the same arguments, workspace and stream.  Arguments are as for int8_linear_forward.
  *
- * int8_linear_quantize: the activation side -- outlier columns, per-row scales, int8
- *   activations, and the compacted fp16 outlier operands (activations and
- *   W_hat = fp16(Wq * w_scale)) -- written into the workspace.  Arguments as for
- *   int8_linear_forward.
- * int8_linear_matmul: the tensor-core side -- the int8 and fp16 products and the fused
- *   epilogue -- reading the workspace the previous int8_linear_quantize call on the same
- *   layer shape and weights filled.
+ * int8_linear_quantize: the activation statistics.  For M > 16: outlier columns, per-row
+ *   scales, int8 activations and the compacted fp16 outlier operands (activations and
+ *   W_hat = fp16(Wq * w_scale)), written into the workspace.  For M <= 16 (few tokens, the
+ *   weight-streaming regime): the outlier mask and per-strip row maxima only; the int8
+ *   activations are formed inside the matmul kernel, next to the tensor cores.
+ * int8_linear_matmul: the rest -- the int8 and fp16 products and the fused epilogue --
+ *   reading what int8_linear_quantize left in the workspace.
  */
 int int8_linear_quantize(const void *X, int M, int K, const int8_t *Wq, const float *w_scale,
                          int N, float threshold, void *workspace, size_t ws_bytes,
                          int8mm_stream_t stream);
-int int8_linear_matmul(int M, int K, const int8_t *Wq, const float *w_scale, const void *bias,
-                       int N, void *Y, void *workspace, size_t ws_bytes,
-                       int8mm_stream_t stream);
+int int8_linear_matmul(const void *X, int M, int K, const int8_t *Wq, const float *w_scale,
+                       const void *bias, int N, float threshold, void *Y, void *workspace,
+                       size_t ws_bytes, int8mm_stream_t stream);
+
+/*
+ * Diagnostic: int8_linear_forward that also writes the int32 accumulators
+ * acc[i,n] = sum_k Xq[i,k] * Wq[n,k] (the int8 product of [P2] section 2.3 before
+ * dequantization), int32 [M, N], 16-byte aligned.  Y is as for int8_linear_forward.
+ */
+int int8_linear_forward_acc(const void *X, int M, int K, const int8_t *Wq,
+                            const float *w_scale, const void *bias, int N, float threshold,
+                            void *Y, int32_t *acc, void *workspace, size_t ws_bytes,
+                            int8mm_stream_t stream);
 
 /*
  * Diagnostic: the quantization half of the layer alone (outlier detection and per-row

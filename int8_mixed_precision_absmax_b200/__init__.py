@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "Int8mmError", "load_library", "library_path",
     "int8_quant_weight", "int8_linear_workspace_size", "int8_linear_forward",
-    "int8_linear_quantize", "int8_linear_matmul",
+    "int8_linear_quantize", "int8_linear_matmul", "int8_linear_forward_acc",
     "int8_quantize_rows", "int8_gemm_i32", "int8_outlier_weights",
     "int8_read_device_status", "int8_status_string", "Int8Linear", "DEFAULT_THRESHOLD",
 ]
@@ -64,13 +64,14 @@ def load_library():
         lib.int8_linear_workspace_size.restype = sz
         lib.int8_linear_forward.argtypes = [p, i, i, p, p, p, i, f, p, p, sz, p]
         lib.int8_linear_quantize.argtypes = [p, i, i, p, p, i, f, p, sz, p]
-        lib.int8_linear_matmul.argtypes = [i, i, p, p, p, i, p, p, sz, p]
+        lib.int8_linear_matmul.argtypes = [p, i, i, p, p, p, i, f, p, p, sz, p]
+        lib.int8_linear_forward_acc.argtypes = [p, i, i, p, p, p, i, f, p, p, p, sz, p]
         lib.int8_quantize_rows.argtypes = [p, i, i, f, p, p, p, p, p, sz, p]
         lib.int8_gemm_i32.argtypes = [p, p, i, i, i, p, p, p]
         lib.int8_outlier_weights.argtypes = [p, p, i, i, p, p, p, p]
         lib.int8_read_device_status.argtypes = [p, p]
         for name in ("int8_quant_weight", "int8_linear_forward", "int8_linear_quantize",
-                     "int8_linear_matmul", "int8_quantize_rows",
+                     "int8_linear_matmul", "int8_linear_forward_acc", "int8_quantize_rows",
                      "int8_gemm_i32", "int8_outlier_weights", "int8_read_device_status"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
@@ -175,18 +176,40 @@ def int8_linear_quantize(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tenso
         workspace.numel(), ctypes.c_void_p(_stream(stream, X.device))), "int8_linear_quantize")
 
 
-def int8_linear_matmul(M: int, Wq: torch.Tensor, w_scale: torch.Tensor,
-                       bias: torch.Tensor | None, Y: torch.Tensor, workspace: torch.Tensor,
-                       stream=None) -> torch.Tensor:
-    """The tensor-core side of the forward, from `workspace` (see int8_linear_forward)."""
+def int8_linear_matmul(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                       bias: torch.Tensor | None, threshold: float, Y: torch.Tensor,
+                       workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """The second half of the forward, from `workspace` (see int8_linear_forward)."""
+    _need(X, torch.float16, "X", 2)
     _need(Wq, torch.int8, "Wq", 2)
     _need(Y, torch.float16, "Y", 2)
     _need(workspace, torch.uint8, "workspace", 1)
-    N, K = Wq.shape
+    M, K = X.shape
+    N = Wq.shape[0]
     _check(load_library().int8_linear_matmul(
-        M, K, _ptr(Wq), _ptr(w_scale), _ptr(bias), N, _ptr(Y), _ptr(workspace),
-        workspace.numel(), ctypes.c_void_p(_stream(stream, Y.device))), "int8_linear_matmul")
+        _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(bias), N, float(threshold), _ptr(Y),
+        _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream, X.device))),
+        "int8_linear_matmul")
     return Y
+
+
+def int8_linear_forward_acc(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                            bias: torch.Tensor | None, threshold: float = DEFAULT_THRESHOLD,
+                            workspace: torch.Tensor | None = None, stream=None):
+    """(Y fp16 [M,N], int32 accumulators [M,N]) of one forward."""
+    _need(X, torch.float16, "X", 2)
+    _need(Wq, torch.int8, "Wq", 2)
+    M, K = X.shape
+    N = Wq.shape[0]
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=X.device)
+    if workspace is None:
+        workspace = new_workspace(M, N, K, X.device)
+    _check(load_library().int8_linear_forward_acc(
+        _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(bias), N, float(threshold), _ptr(Y),
+        _ptr(acc), _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream, X.device))),
+        "int8_linear_forward_acc")
+    return Y, acc
 
 
 def int8_quantize_rows(X: torch.Tensor, threshold: float = DEFAULT_THRESHOLD,

@@ -36,6 +36,24 @@ int check_device() {
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? INT8MM_OK : INT8MM_ERR_CUDA; }
 
+}  // namespace
+
+int i8mm::device_sm_count() {
+  static int cached_device = -1, cached_sms = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev != cached_device) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+    cached_sms = sms;
+    cached_device = dev;
+  }
+  return cached_sms;
+}
+
+namespace {
+
 float effective_threshold(float t) { return t < 0.0f ? 0.0f : t; }
 
 template <typename T>
@@ -111,9 +129,38 @@ int plan_forward(int M, int N, int K, const int8_t* Wq, const float* w_scale, vo
   return INT8MM_OK;
 }
 
+SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+                     const void* bias, int N, float threshold, void* Y, int32_t* acc,
+                     void* workspace, const ForwardPlan& p, const SmallPlan& sp) {
+  SmallArgs a;
+  a.X = static_cast<const __half*>(X);
+  a.M = M;
+  a.K = K;
+  a.N = N;
+  a.threshold = effective_threshold(threshold);
+  a.mask = p.mask;
+  a.rowmax_part = at<float>(workspace, p.L.rowmax);
+  a.Wq = Wq;
+  a.w_scale = w_scale;
+  a.bias = static_cast<const __half*>(bias);
+  a.Y = static_cast<__half*>(Y);
+  a.acc = acc;
+  a.partials = at<int32_t>(workspace, p.L.partials);
+  a.counters = at<uint32_t>(workspace, p.L.counters);
+  a.splits = sp.splits;
+  a.status = p.header;
+  return a;
+}
+
 int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale, int N,
                  float threshold, void* workspace, const ForwardPlan& p, cudaStream_t stream,
                  bool pdl_first) {
+  if (p.L.small) {
+    const SmallPlan sp = plan_small(M, N, K, device_sm_count());
+    const SmallArgs a = small_args(X, M, K, Wq, w_scale, nullptr, N, threshold, nullptr, nullptr,
+                                   workspace, p, sp);
+    return launch_status(launch_small_stats(a, sp, stream, pdl_first));
+  }
   int rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
                                         effective_threshold(threshold), p.mask, stream,
                                         pdl_first));
@@ -137,8 +184,18 @@ int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_s
   return launch_status(launch_rowquant(rq, stream, true));
 }
 
-int run_matmul(int M, int K, const int8_t* Wq, const float* w_scale, const void* bias, int N,
-               void* Y, const ForwardPlan& p, cudaStream_t stream, bool pdl) {
+int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+               const void* bias, int N, float threshold, void* Y, int32_t* acc,
+               void* workspace, const ForwardPlan& p, cudaStream_t stream, bool pdl) {
+  if (p.L.small) {
+    const SmallPlan sp = plan_small(M, N, K, device_sm_count());
+    const SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace,
+                                   p, sp);
+    CUtensorMap map;
+    if (!encode_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kSmallBN))
+      return INT8MM_ERR_CUDA;
+    return launch_status(launch_small_gemm(map, a, sp, stream, pdl));
+  }
   GemmMaps maps;
   if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.xq, K, M, K, kBKBytes, kBM) ||
       !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kBN) ||
@@ -155,10 +212,25 @@ int run_matmul(int M, int K, const int8_t* Wq, const float* w_scale, const void*
   g.w_scale = w_scale;
   g.bias = static_cast<const __half*>(bias);
   g.Y = static_cast<__half*>(Y);
-  g.C = nullptr;
+  g.C = acc;
   g.n_out = p.header + 1;
   g.status = p.header;
   return launch_status(launch_gemm(maps, g, stream, pdl));
+}
+
+int forward_impl(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+                 const void* bias, int N, float threshold, void* Y, int32_t* acc,
+                 void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!X || !Y) return INT8MM_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Y) || (bias && !aligned16(bias)) || (acc && !aligned16(acc)))
+    return INT8MM_ERR_ALIGN;
+  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
+  ForwardPlan p;
+  int rc = plan_forward(M, N, K, Wq, w_scale, workspace, ws_bytes, p);
+  if (rc) return rc;
+  if ((rc = run_quantize(X, M, K, Wq, w_scale, N, threshold, workspace, p, stream, true)))
+    return rc;
+  return run_matmul(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace, p, stream, true);
 }
 
 }  // namespace
@@ -167,17 +239,18 @@ extern "C" {
 
 int int8_linear_forward(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                         const void* bias, int N, float threshold, void* Y, void* workspace,
-                        size_t ws_bytes, int8mm_stream_t stream_) {
-  if (!X || !Y) return INT8MM_ERR_NULL;
-  if (!aligned16(X) || !aligned16(Y) || (bias && !aligned16(bias))) return INT8MM_ERR_ALIGN;
-  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
-  ForwardPlan p;
-  int rc = plan_forward(M, N, K, Wq, w_scale, workspace, ws_bytes, p);
-  if (rc) return rc;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  if ((rc = run_quantize(X, M, K, Wq, w_scale, N, threshold, workspace, p, stream, true)))
-    return rc;
-  return run_matmul(M, K, Wq, w_scale, bias, N, Y, p, stream, true);
+                        size_t ws_bytes, int8mm_stream_t stream) {
+  return forward_impl(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, workspace, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int int8_linear_forward_acc(const void* X, int M, int K, const int8_t* Wq,
+                            const float* w_scale, const void* bias, int N, float threshold,
+                            void* Y, int32_t* acc, void* workspace, size_t ws_bytes,
+                            int8mm_stream_t stream) {
+  if (!acc) return INT8MM_ERR_NULL;
+  return forward_impl(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 int int8_linear_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
@@ -193,16 +266,17 @@ int int8_linear_quantize(const void* X, int M, int K, const int8_t* Wq, const fl
                       reinterpret_cast<cudaStream_t>(stream), true);
 }
 
-int int8_linear_matmul(int M, int K, const int8_t* Wq, const float* w_scale, const void* bias,
-                       int N, void* Y, void* workspace, size_t ws_bytes,
-                       int8mm_stream_t stream) {
-  if (!Y) return INT8MM_ERR_NULL;
-  if (!aligned16(Y) || (bias && !aligned16(bias))) return INT8MM_ERR_ALIGN;
+int int8_linear_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+                       const void* bias, int N, float threshold, void* Y, void* workspace,
+                       size_t ws_bytes, int8mm_stream_t stream) {
+  if (!X || !Y) return INT8MM_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Y) || (bias && !aligned16(bias))) return INT8MM_ERR_ALIGN;
+  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
   ForwardPlan p;
   int rc = plan_forward(M, N, K, Wq, w_scale, workspace, ws_bytes, p);
   if (rc) return rc;
-  return run_matmul(M, K, Wq, w_scale, bias, N, Y, p, reinterpret_cast<cudaStream_t>(stream),
-                    true);
+  return run_matmul(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, workspace, p,
+                    reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 int int8_quantize_rows(const void* X, int M, int K, float threshold, int8_t* Xq,

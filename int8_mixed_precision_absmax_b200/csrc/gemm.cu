@@ -229,8 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         const int n = n0 + c;
         const int valid = min(32, N - n);
-        if (!row_ok || valid <= 0) {
-        } else if (args.C) {
+        if (row_ok && valid > 0 && args.C) {
           int32_t* dst = args.C + static_cast<size_t>(row) * N + n;
           if (valid == 32 && (N % 4) == 0) {
 #pragma unroll
@@ -243,7 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j)
               if (j < valid) dst[j] = kb_i8 ? static_cast<int32_t>(ra[j]) : 0;
           }
-        } else {
+        }
+        if (row_ok && valid > 0 && args.Y) {
           float y[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {

@@ -22,9 +22,19 @@ namespace i8mm {
 //   xo       half[M*ldo]    outlier activations, compacted, zero-padded to a multiple of 64
 //   wo       half[N*ldo]    outlier weights fp16(Wq*w_scale), compacted, zero-padded
 // ldo = K rounded up to 64 (the fp16 operand tiles are 64 elements deep).
+// The small-M path (M <= kSmallMP) adds: per-strip row maxima float[ceil(K/256)*16],
+// split-K partial sums int32[tiles*kSmallMaxSplits*128*16] and per-tile counters
+// uint32[tiles] (zero between calls: the last CTA of a tile resets its counter).
+constexpr int kSmallMP = 16;             // tokens per MMA (N of the swapped product)
+constexpr int kSmallBN = 128;            // output channels per CTA (M of the MMA)
+constexpr int kSmallMaxSplits = 16;
+constexpr int kSmallMaxKbPerSplit = 32;  // 128-byte k-blocks of Xq one CTA keeps in smem
+constexpr int kSmallStrip = 256;         // columns per stats block
+
 struct WorkspaceLayout {
-  size_t header, mask, cols, xscale, xq, xo, wo, total;
+  size_t header, mask, cols, xscale, xq, xo, wo, rowmax, partials, counters, total;
   int ldo;
+  bool small;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -40,6 +50,14 @@ inline WorkspaceLayout workspace_layout(int M, int N, int K) {
   L.xq = off;     off = align256(off + static_cast<size_t>(M) * K);
   L.xo = off;     off = align256(off + static_cast<size_t>(M) * L.ldo * sizeof(__half));
   L.wo = off;     off = align256(off + static_cast<size_t>(N) * L.ldo * sizeof(__half));
+  L.small = M <= kSmallMP;
+  L.rowmax = L.partials = L.counters = off;
+  if (L.small) {
+    const size_t tiles = static_cast<size_t>((N + kSmallBN - 1) / kSmallBN);
+    L.rowmax = off;   off = align256(off + static_cast<size_t>((K + kSmallStrip - 1) / kSmallStrip) * kSmallMP * sizeof(float));
+    L.partials = off; off = align256(off + tiles * kSmallMaxSplits * kSmallBN * kSmallMP * sizeof(int32_t));
+    L.counters = off; off = align256(off + tiles * sizeof(uint32_t));
+  }
   L.total = off;
   return L;
 }
@@ -78,13 +96,39 @@ struct RowQuantArgs {
 };
 cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl);
 
+struct SmallArgs {
+  const __half* X;
+  int M, K, N;
+  float threshold;
+  uint32_t* mask;
+  float* rowmax_part;
+  const int8_t* Wq;
+  const float* w_scale;
+  const __half* bias;
+  __half* Y;
+  int32_t* acc;          // nullable: also write the int32 accumulators
+  int32_t* partials;
+  uint32_t* counters;
+  int splits;
+  int32_t* status;
+};
+struct SmallPlan {
+  int tiles, splits, kb_per_split, strips;
+};
+SmallPlan plan_small(int M, int N, int K, int num_sms);
+cudaError_t launch_small_stats(const SmallArgs& a, const SmallPlan& p, cudaStream_t stream,
+                               bool pdl);
+cudaError_t launch_small_gemm(const CUtensorMap& map_wq, const SmallArgs& a, const SmallPlan& p,
+                              cudaStream_t stream, bool pdl);
+int device_sm_count();
+
 struct GemmArgs {
   int M, N, K;
   const float* xscale;   // [M]
   const float* w_scale;  // [N]
   const __half* bias;    // [N] or null
   __half* Y;             // fused epilogue output [M,N], or null
-  int32_t* C;            // raw int32 output [M,N], or null (exactly one of Y, C)
+  int32_t* C;            // raw int32 accumulators [M,N], or null (at least one of Y, C)
   const int32_t* n_out;  // device outlier count, or null for none
   int32_t* status;
 };

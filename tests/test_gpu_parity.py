@@ -197,3 +197,68 @@ def test_175b_sweep_narrow(frac, t):
     g_cols = check_full_size(w, X, W, b, t, n_rows=4)
     if t == math.inf:
         assert g_cols.size == 0
+
+
+# ------------------------------------------------------------------ accumulators and few tokens
+
+def check_forward_acc(X, W, b, t, rows=None):
+    """Y and the int32 accumulators of int8_linear_forward_acc against the oracle."""
+    Xd = to_dev(X)
+    Wq_d, sw_d = i8.int8_quant_weight(to_dev(W))
+    ws = i8.new_workspace(X.shape[0], W.shape[0], X.shape[1], Xd.device)
+    Y, acc = i8.int8_linear_forward_acc(Xd, Wq_d, sw_d, None if b is None else to_dev(b), t,
+                                        workspace=ws)
+    assert i8.int8_read_device_status(ws[:4].view(torch.int32)) == 0
+    Y, acc = to_np(Y), to_np(acc)
+    Wq, sw = to_np(Wq_d), to_np(sw_d)
+    if rows is None:
+        rows = np.arange(X.shape[0])
+    Y_ref, A_ref = oracle.linear_forward_rows(X, Wq, sw, b, t, rows)
+    np.testing.assert_array_equal(acc[rows], A_ref)
+    assert_y_close(Y[rows], Y_ref)
+    # the forward without accumulators gives the same Y bits
+    Y2 = to_np(i8.int8_linear_forward(Xd, Wq_d, sw_d, None if b is None else to_dev(b), t,
+                                      workspace=ws))
+    np.testing.assert_array_equal(f16_bits(Y2), f16_bits(Y))
+    return Y, acc
+
+
+@pytest.mark.parametrize("M,K,N,n_out,t", [
+    (1, 16, 1, 0, 6.0),
+    (1, 4096, 4096, 3, 6.0),
+    (3, 1040, 300, 2, 6.0),     # ragged K and N on the few-token path
+    (8, 4096, 4096, 6, 6.0),    # the decode shape
+    (16, 2048, 640, 5, 6.0),    # the largest few-token batch
+    (16, 256, 128, 0, math.inf),
+    (7, 512, 384, 0, 0.0),      # every column an outlier: int8 product is zero
+    (5, 20000, 200, 4, 6.0),    # long rows: many splits
+    (17, 512, 300, 3, 6.0),     # one row past the few-token path
+    (200, 1040, 600, 5, 6.0),   # the tiled path
+])
+def test_forward_accumulators_and_y(M, K, N, n_out, t):
+    X, W, b = random_case(M, K, N, n_out, seed=M + 3 * K + 7 * N)
+    Y, acc = check_forward_acc(X, W, b, t)
+    if t == 0.0:
+        assert not acc.any()
+
+
+def test_decode_workload_full_forward():
+    w, X, W, b, _ = workload_inputs("decode_q_proj")
+    Y, acc = check_forward_acc(X, W, b, w.threshold)
+    # repeated calls reuse the split-K counters: same bits every time
+    Y2, acc2 = check_forward_acc(X, W, b, w.threshold)
+    np.testing.assert_array_equal(acc, acc2)
+    np.testing.assert_array_equal(f16_bits(Y), f16_bits(Y2))
+
+
+def test_few_token_path_many_calls_one_workspace():
+    X, W, b = random_case(8, 1024, 1024, 3, seed=21)
+    Xd = to_dev(X)
+    Wq_d, sw_d = i8.int8_quant_weight(to_dev(W))
+    ws = i8.new_workspace(8, 1024, 1024, Xd.device)
+    first = to_np(i8.int8_linear_forward(Xd, Wq_d, sw_d, to_dev(b), 6.0, workspace=ws))
+    Ys = [i8.int8_linear_forward(Xd, Wq_d, sw_d, to_dev(b), 6.0, workspace=ws) for _ in range(50)]
+    torch.cuda.synchronize()
+    for Y in Ys:
+        np.testing.assert_array_equal(f16_bits(to_np(Y)), f16_bits(first))
+    assert i8.int8_read_device_status(ws[:4].view(torch.int32)) == 0
