@@ -146,6 +146,7 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
   a.Y = static_cast<__half*>(Y);
   a.acc = acc;
   a.partials = at<int32_t>(workspace, p.L.partials);
+  a.fpartials = at<float>(workspace, p.L.fpartials);
   a.counters = at<uint32_t>(workspace, p.L.counters);
   a.splits = sp.splits;
   a.status = p.header;

@@ -23,7 +23,8 @@ namespace i8mm {
 //   wo       half[N*ldo]    outlier weights fp16(Wq*w_scale), compacted, zero-padded
 // ldo = K rounded up to 64 (the fp16 operand tiles are 64 elements deep).
 // The small-M path (M <= kSmallMP) adds: per-strip row maxima float[ceil(K/256)*16],
-// split-K partial sums int32[tiles*kSmallMaxSplits*128*16] and per-tile counters
+// split-K partial sums int32[tiles*kSmallMaxSplits*128*16] and their fp32 outlier-term
+// counterparts float[tiles*kSmallMaxSplits*128*16], and per-tile counters
 // uint32[tiles] (zero between calls: the last CTA of a tile resets its counter).
 constexpr int kSmallMP = 16;             // tokens per MMA (N of the swapped product)
 constexpr int kSmallBN = 128;            // output channels per CTA (M of the MMA)
@@ -32,7 +33,7 @@ constexpr int kSmallMaxKbPerSplit = 32;  // 128-byte k-blocks of Xq one CTA keep
 constexpr int kSmallStrip = 256;         // columns per stats block
 
 struct WorkspaceLayout {
-  size_t header, mask, cols, xscale, xq, xo, wo, rowmax, partials, counters, total;
+  size_t header, mask, cols, xscale, xq, xo, wo, rowmax, partials, fpartials, counters, total;
   int ldo;
   bool small;
 };
@@ -51,11 +52,12 @@ inline WorkspaceLayout workspace_layout(int M, int N, int K) {
   L.xo = off;     off = align256(off + static_cast<size_t>(M) * L.ldo * sizeof(__half));
   L.wo = off;     off = align256(off + static_cast<size_t>(N) * L.ldo * sizeof(__half));
   L.small = M <= kSmallMP;
-  L.rowmax = L.partials = L.counters = off;
+  L.rowmax = L.partials = L.fpartials = L.counters = off;
   if (L.small) {
     const size_t tiles = static_cast<size_t>((N + kSmallBN - 1) / kSmallBN);
     L.rowmax = off;   off = align256(off + static_cast<size_t>((K + kSmallStrip - 1) / kSmallStrip) * kSmallMP * sizeof(float));
     L.partials = off; off = align256(off + tiles * kSmallMaxSplits * kSmallBN * kSmallMP * sizeof(int32_t));
+    L.fpartials = off; off = align256(off + tiles * kSmallMaxSplits * kSmallBN * kSmallMP * sizeof(float));
     L.counters = off; off = align256(off + tiles * sizeof(uint32_t));
   }
   L.total = off;
@@ -107,7 +109,8 @@ struct SmallArgs {
   const __half* bias;
   __half* Y;
   int32_t* acc;          // nullable: also write the int32 accumulators
-  int32_t* partials;
+  int32_t* partials;     // split-K int32 partial sums
+  float* fpartials;      // split-K partial fp16-outlier terms
   uint32_t* counters;
   int splits;
   int32_t* status;

@@ -148,6 +148,7 @@ struct SmallShared {
   int epi_ok;
   float sx[kSmallMP];
   int zero_row[kSmallMP];
+  float psum[kSmallBN][kSmallMP + 1];  // this CTA's outlier term per channel (+1: no bank clash)
   uint32_t mask[kSmallMaxKbPerSplit * 4];
 };
 
@@ -156,7 +157,7 @@ size_t small_gemm_smem_bytes(int kb_per_split) {
          static_cast<size_t>(kb_per_split) * kBBytesPerKb + sizeof(SmallShared);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     small_gemm_kernel(const __grid_constant__ CUtensorMap map_wq, const SmallArgs a) {
   extern __shared__ uint8_t small_smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
@@ -296,9 +297,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_arrive(&sh.xq_ready);
 
     if (warp >= 4) {
-      // ---- epilogue: warps 4..7 own TMEM lane quadrants 0..3 (channels 32q .. 32q+31)
+      // ---- warps 4..7 own TMEM lane quadrants 0..3, i.e. channels 32q .. 32q+31
       const int quad = warp & 3;
       const int n = quad * 32 + lane, gn = n0 + n;
+      // The fp16 outlier term of the outlier columns inside this CTA's K-slice, computed
+      // while the MMAs run: P[i] = sum_j X[i,j] * fp16(Wq[gn,j] * w_scale[gn]).
+      {
+        float P[kSmallMP];
+#pragma unroll
+        for (int i = 0; i < kSmallMP; ++i) P[i] = 0.0f;
+        if (gn < a.N) {
+          const float sw_n = a.w_scale[gn];
+          const int8_t* wrow = a.Wq + static_cast<size_t>(gn) * a.K;
+          for (int w = 0; w < nkb * 4; ++w) {
+            uint32_t bits = sh.mask[w];
+            while (bits) {
+              const int j = kb_begin * kBKBytes + w * 32 + __ffs(bits) - 1;
+              bits &= bits - 1u;
+              const float wv = __half2float(__float2half_rn(static_cast<float>(wrow[j]) * sw_n));
+#pragma unroll
+              for (int i = 0; i < kSmallMP; ++i)
+                if (i < a.M) P[i] += wv * __half2float(a.X[static_cast<size_t>(i) * a.K + j]);
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kSmallMP; ++i) sh.psum[n][i] = P[i];
+      }
       int32_t acc[kSmallMP];
       mbar_wait_bounded(&sh.tmem_full, 0, abort);
       // one decision for all 128 epilogue threads, so the barriers below cannot split
@@ -316,11 +341,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool finish = ok;
       if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
       if (ok && S > 1) {
-        int4* part = reinterpret_cast<int4*>(
-            a.partials + ((static_cast<size_t>(tile) * S + split) * kSmallBN + n) * kSmallMP);
+        const size_t slot = ((static_cast<size_t>(tile) * S + split) * kSmallBN + n) * kSmallMP;
+        int4* ip = reinterpret_cast<int4*>(a.partials + slot);
+        float4* fp = reinterpret_cast<float4*>(a.fpartials + slot);
 #pragma unroll
-        for (int v = 0; v < kSmallMP / 4; ++v)
-          __stcg(part + v, make_int4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]));
+        for (int v = 0; v < kSmallMP / 4; ++v) {
+          __stcg(ip + v, make_int4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]));
+          __stcg(fp + v, make_float4(sh.psum[n][4 * v], sh.psum[n][4 * v + 1],
+                                     sh.psum[n][4 * v + 2], sh.psum[n][4 * v + 3]));
+        }
         __threadfence();
         named_barrier(2, 128);
         if (threadIdx.x == 128) {
@@ -333,46 +362,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         finish = sh.last != 0;
         if (finish) {
           __threadfence();
+          float P[kSmallMP];
 #pragma unroll
-          for (int i = 0; i < kSmallMP; ++i) acc[i] = 0;
+          for (int i = 0; i < kSmallMP; ++i) {
+            acc[i] = 0;
+            P[i] = 0.0f;
+          }
           for (int s2 = 0; s2 < S; ++s2) {  // fixed order: the same bits on every call
-            const int4* p = reinterpret_cast<const int4*>(
-                a.partials + ((static_cast<size_t>(tile) * S + s2) * kSmallBN + n) * kSmallMP);
+            const size_t o = ((static_cast<size_t>(tile) * S + s2) * kSmallBN + n) * kSmallMP;
+            const int4* ip2 = reinterpret_cast<const int4*>(a.partials + o);
+            const float4* fp2 = reinterpret_cast<const float4*>(a.fpartials + o);
 #pragma unroll
             for (int v = 0; v < kSmallMP / 4; ++v) {
-              const int4 t = __ldcg(p + v);
+              const int4 t = __ldcg(ip2 + v);
+              const float4 f = __ldcg(fp2 + v);
               acc[4 * v] += t.x;
               acc[4 * v + 1] += t.y;
               acc[4 * v + 2] += t.z;
               acc[4 * v + 3] += t.w;
+              P[4 * v] += f.x;
+              P[4 * v + 1] += f.y;
+              P[4 * v + 2] += f.z;
+              P[4 * v + 3] += f.w;
             }
           }
+#pragma unroll
+          for (int i = 0; i < kSmallMP; ++i) sh.psum[n][i] = P[i];
         }
       }
       if (finish && gn < a.N) {
-        // fp16 outlier term on the CUDA cores: P[i] = sum_j X[i,j] * fp16(Wq[gn,j] * w_scale[gn])
-        const float swn = a.w_scale[gn];
-        float P[kSmallMP];
-#pragma unroll
-        for (int i = 0; i < kSmallMP; ++i) P[i] = 0.0f;
-        const int words = (a.K + 31) / 32;
-        const int8_t* wrow = a.Wq + static_cast<size_t>(gn) * a.K;
-        for (int w = 0; w < words; ++w) {
-          uint32_t bits = __ldcg(a.mask + w);
-          while (bits) {
-            const int j = w * 32 + __ffs(bits) - 1;
-            bits &= bits - 1u;
-            const float wv = __half2float(__float2half_rn(static_cast<float>(wrow[j]) * swn));
-#pragma unroll
-            for (int i = 0; i < kSmallMP; ++i)
-              if (i < a.M) P[i] += wv * __half2float(a.X[static_cast<size_t>(i) * a.K + j]);
-          }
-        }
         const float b = a.bias ? __half2float(a.bias[gn]) : 0.0f;
+        const float swn = a.w_scale[gn];
 #pragma unroll
         for (int i = 0; i < kSmallMP; ++i) {
           if (i < a.M) {
-            const float y = static_cast<float>(acc[i]) * sh.sx[i] * swn + P[i] + b;
+            const float y = static_cast<float>(acc[i]) * sh.sx[i] * swn + sh.psum[n][i] + b;
             a.Y[static_cast<size_t>(i) * a.N + gn] = __float2half_rn(y);
             if (a.acc) a.acc[static_cast<size_t>(i) * a.N + gn] = acc[i];
           }
