@@ -101,11 +101,11 @@ int int8_linear_forward(const void *X, int M, int K, const int8_t *Wq, const flo
  * int8_linear_forward is exactly int8_linear_quantize followed by int8_linear_matmul with
  * the same arguments, workspace and stream.  Arguments are as for int8_linear_forward.
  *
- * int8_linear_quantize: the activation statistics.  For M > 16: outlier columns, per-row
- *   scales, int8 activations and the compacted fp16 outlier operands (activations and
+ * int8_linear_quantize: the activation side.  For M > 16: outlier columns, per-row scales,
+ *   int8 activations and the compacted fp16 outlier operands (activations and
  *   W_hat = fp16(Wq * w_scale)), written into the workspace.  For M <= 16 (few tokens, the
- *   weight-streaming regime): the outlier mask and per-strip row maxima only; the int8
- *   activations are formed inside the matmul kernel, next to the tensor cores.
+ *   weight-streaming regime, K <= 32768) it enqueues nothing: one kernel in
+ *   int8_linear_matmul quantizes the activations next to the tensor cores.
  * int8_linear_matmul: the rest -- the int8 and fp16 products and the fused epilogue --
  *   reading what int8_linear_quantize left in the workspace.
  */

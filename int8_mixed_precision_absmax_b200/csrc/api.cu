@@ -36,24 +36,6 @@ int check_device() {
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? INT8MM_OK : INT8MM_ERR_CUDA; }
 
-}  // namespace
-
-int i8mm::device_sm_count() {
-  static int cached_device = -1, cached_sms = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev != cached_device) {
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-      sms = 148;
-    cached_sms = sms;
-    cached_device = dev;
-  }
-  return cached_sms;
-}
-
-namespace {
-
 float effective_threshold(float t) { return t < 0.0f ? 0.0f : t; }
 
 template <typename T>
@@ -131,23 +113,18 @@ int plan_forward(int M, int N, int K, const int8_t* Wq, const float* w_scale, vo
 
 SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                      const void* bias, int N, float threshold, void* Y, int32_t* acc,
-                     void* workspace, const ForwardPlan& p, const SmallPlan& sp) {
+                     const ForwardPlan& p, const SmallPlan& sp) {
   SmallArgs a;
   a.X = static_cast<const __half*>(X);
   a.M = M;
   a.K = K;
   a.N = N;
   a.threshold = effective_threshold(threshold);
-  a.mask = p.mask;
-  a.rowmax_part = at<float>(workspace, p.L.rowmax);
   a.Wq = Wq;
   a.w_scale = w_scale;
   a.bias = static_cast<const __half*>(bias);
   a.Y = static_cast<__half*>(Y);
   a.acc = acc;
-  a.partials = at<int32_t>(workspace, p.L.partials);
-  a.fpartials = at<float>(workspace, p.L.fpartials);
-  a.counters = at<uint32_t>(workspace, p.L.counters);
   a.splits = sp.splits;
   a.status = p.header;
   return a;
@@ -156,12 +133,7 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
 int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale, int N,
                  float threshold, void* workspace, const ForwardPlan& p, cudaStream_t stream,
                  bool pdl_first) {
-  if (p.L.small) {
-    const SmallPlan sp = plan_small(M, N, K, device_sm_count());
-    const SmallArgs a = small_args(X, M, K, Wq, w_scale, nullptr, N, threshold, nullptr, nullptr,
-                                   workspace, p, sp);
-    return launch_status(launch_small_stats(a, sp, stream, pdl_first));
-  }
+  if (small_path_fits(M, K)) return INT8MM_OK;  // one kernel does everything: see run_matmul
   int rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
                                         effective_threshold(threshold), p.mask, stream,
                                         pdl_first));
@@ -188,14 +160,13 @@ int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_s
 int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                const void* bias, int N, float threshold, void* Y, int32_t* acc,
                void* workspace, const ForwardPlan& p, cudaStream_t stream, bool pdl) {
-  if (p.L.small) {
-    const SmallPlan sp = plan_small(M, N, K, device_sm_count());
-    const SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace,
-                                   p, sp);
+  if (small_path_fits(M, K)) {
+    const SmallPlan sp = plan_small(N, K);
+    const SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p, sp);
     CUtensorMap map;
     if (!encode_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kSmallBN))
       return INT8MM_ERR_CUDA;
-    return launch_status(launch_small_gemm(map, a, sp, stream, pdl));
+    return launch_status(launch_small(map, a, sp, stream, pdl));
   }
   GemmMaps maps;
   if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.xq, K, M, K, kBKBytes, kBM) ||

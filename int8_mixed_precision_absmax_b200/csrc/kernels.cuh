@@ -22,20 +22,16 @@ namespace i8mm {
 //   xo       half[M*ldo]    outlier activations, compacted, zero-padded to a multiple of 64
 //   wo       half[N*ldo]    outlier weights fp16(Wq*w_scale), compacted, zero-padded
 // ldo = K rounded up to 64 (the fp16 operand tiles are 64 elements deep).
-// The small-M path (M <= kSmallMP) adds: per-strip row maxima float[ceil(K/256)*16],
-// split-K partial sums int32[tiles*kSmallMaxSplits*128*16] and their fp32 outlier-term
-// counterparts float[tiles*kSmallMaxSplits*128*16], and per-tile counters
-// uint32[tiles] (zero between calls: the last CTA of a tile resets its counter).
+// The few-token path (M <= kSmallMP) runs in one cluster kernel (small.cu) and keeps its
+// intermediates in shared memory; it uses only the status word of the workspace.
 constexpr int kSmallMP = 16;             // tokens per MMA (N of the swapped product)
-constexpr int kSmallBN = 128;            // output channels per CTA (M of the MMA)
-constexpr int kSmallMaxSplits = 16;
+constexpr int kSmallBN = 128;            // output channels per tile (M of the MMA)
+constexpr int kSmallMaxSplits = 8;       // CTAs per cluster (portable cluster size)
 constexpr int kSmallMaxKbPerSplit = 32;  // 128-byte k-blocks of Xq one CTA keeps in smem
-constexpr int kSmallStrip = 256;         // columns per stats block
 
 struct WorkspaceLayout {
-  size_t header, mask, cols, xscale, xq, xo, wo, rowmax, partials, fpartials, counters, total;
+  size_t header, mask, cols, xscale, xq, xo, wo, total;
   int ldo;
-  bool small;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -51,15 +47,6 @@ inline WorkspaceLayout workspace_layout(int M, int N, int K) {
   L.xq = off;     off = align256(off + static_cast<size_t>(M) * K);
   L.xo = off;     off = align256(off + static_cast<size_t>(M) * L.ldo * sizeof(__half));
   L.wo = off;     off = align256(off + static_cast<size_t>(N) * L.ldo * sizeof(__half));
-  L.small = M <= kSmallMP;
-  L.rowmax = L.partials = L.fpartials = L.counters = off;
-  if (L.small) {
-    const size_t tiles = static_cast<size_t>((N + kSmallBN - 1) / kSmallBN);
-    L.rowmax = off;   off = align256(off + static_cast<size_t>((K + kSmallStrip - 1) / kSmallStrip) * kSmallMP * sizeof(float));
-    L.partials = off; off = align256(off + tiles * kSmallMaxSplits * kSmallBN * kSmallMP * sizeof(int32_t));
-    L.fpartials = off; off = align256(off + tiles * kSmallMaxSplits * kSmallBN * kSmallMP * sizeof(float));
-    L.counters = off; off = align256(off + tiles * sizeof(uint32_t));
-  }
   L.total = off;
   return L;
 }
@@ -101,29 +88,22 @@ cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl
 struct SmallArgs {
   const __half* X;
   int M, K, N;
-  float threshold;
-  uint32_t* mask;
-  float* rowmax_part;
+  float threshold;       // already clamped to >= 0
   const int8_t* Wq;
   const float* w_scale;
   const __half* bias;
   __half* Y;
   int32_t* acc;          // nullable: also write the int32 accumulators
-  int32_t* partials;     // split-K int32 partial sums
-  float* fpartials;      // split-K partial fp16-outlier terms
-  uint32_t* counters;
-  int splits;
+  int splits;            // CTAs per cluster, each owning a K-slice
   int32_t* status;
 };
 struct SmallPlan {
-  int tiles, splits, kb_per_split, strips;
+  int tiles, splits, kb_per_split;
 };
-SmallPlan plan_small(int M, int N, int K, int num_sms);
-cudaError_t launch_small_stats(const SmallArgs& a, const SmallPlan& p, cudaStream_t stream,
-                               bool pdl);
-cudaError_t launch_small_gemm(const CUtensorMap& map_wq, const SmallArgs& a, const SmallPlan& p,
-                              cudaStream_t stream, bool pdl);
-int device_sm_count();
+SmallPlan plan_small(int N, int K);
+bool small_path_fits(int M, int K);
+cudaError_t launch_small(const CUtensorMap& map_wq, const SmallArgs& a, const SmallPlan& p,
+                         cudaStream_t stream, bool pdl);
 
 struct GemmArgs {
   int M, N, K;

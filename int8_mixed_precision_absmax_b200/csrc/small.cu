@@ -1,26 +1,35 @@
-// small.cu -- the LLM.int8() layer for a few tokens (M <= 16: the decode regime).
+// small.cu -- the LLM.int8() layer for a few tokens (M <= 16: the decode regime), in one
+// kernel launch.
 //
-// With so few rows the layer is a weight-streaming problem (read Wq once at HBM speed), so
-// the 128 x 256 tiles of gemm.cu would leave most SMs idle.  This path uses two kernels:
+// With so few rows the layer is a weight-streaming problem: every byte of Wq must be read
+// once at HBM speed and everything else hidden behind that stream.  Each output tile of
+// 128 channels is computed by a thread-block cluster of S CTAs that split K (split-K).
+// Each CTA of a cluster:
+//   1. starts the TMA stream of its Wq slice [128 channels x K/S] into a 4-stage ring;
+//   2. reads its K-slice of X for all M rows and finds, per column, whether any |x|
+//      exceeds the threshold (the outlier columns of [P2] "8位量化实战：离群值处理与显存
+//      优化避坑指南" section 2.3 -- complete per slice, since every row is present) and,
+//      per row, the largest |x| over the slice's regular columns;
+//   3. after a cluster barrier, reads the other CTAs' row maxima from their shared memory
+//      (distributed shared memory) to form the row scale sx = max / 127 over all of K
+//      ([P5] "PyTorch 2.9 支持 LLM.int8()" item 2, taken over X_R), identical in every CTA;
+//   4. quantizes its slice, q = rne(x / sx) clamped to [-127, 127] and 0 in outlier
+//      columns, straight into the 128-byte-swizzled shared-memory layout of the MMA's B
+//      operand, and one thread issues tcgen05.mma kind::i8 (M = 128 channels, N = 16
+//      tokens, int32 accumulator in tensor memory);
+//   5. meanwhile computes the fp16 outlier term of the outlier columns in its slice,
+//      sum_j X[i,j] * fp16(Wq[n,j] * w_scale[n]) ([P5] "如何在 PyTorch 2.9 中启用 LLM.int8
+//      推理": no fp16 weights are kept);
+//   6. after a second cluster barrier, sums the S partial int32 accumulators and outlier
+//      terms of its share of the channels from the cluster's shared memory, in rank order
+//      (deterministic), and writes Y = fp16(acc * sx * w_scale + P + bias).
+// No CTA waits on another except through the cluster's hardware barrier; the kernel keeps
+// no state in global memory between calls.
 //
-//   small_stats_kernel  one block per 256-column strip of X: the strip's outlier-mask words
-//                       ([P2] "8位量化实战：离群值处理与显存优化避坑指南" section 2.3) and, per
-//                       row, the maximum |x| over the strip's regular columns (the
-//                       vector-wise absmax of [P5] "PyTorch 2.9 支持 LLM.int8()" item 2,
-//                       taken over X_R).  All <= 16 rows of a strip live in one block, so
-//                       both results are complete per strip: no atomics, no cross-block wait.
-//   small_gemm_kernel   swap-AB tensor-core product with split-K.  Each CTA owns 128 output
-//                       channels and a slice of K.  Its TMA warp streams the Wq slice before
-//                       waiting on the stats kernel (the weights do not depend on it); six
-//                       warps meanwhile quantize the CTA's K-slice of X (row scale = max of
-//                       the strip maxima / 127, q = rne(x / s), 0 in outlier columns) straight
-//                       into the 128-byte-swizzled shared-memory layout of the MMA's B
-//                       operand; one thread issues tcgen05.mma kind::i8 (M = 128 channels,
-//                       N = 16 tokens, int32 accumulator in TMEM).  The CTA writes its int32
-//                       partial sums; the last CTA of a channel tile to finish (an atomic
-//                       count it resets itself) adds the partials in split order (exact),
-//                       the fp16 outlier term sum_j X[i,j] * fp16(Wq[n,j] * w_scale[n]) and
-//                       the bias, and writes Y.  No CTA ever waits for another.
+// Quantization arithmetic, exact to the IEEE quotient: v = x * r with r = 1/sx rounded to
+// nearest is within 2^-16 of x/sx (for |x/sx| <= 127), and the rounded quotient fl(x/sx) is
+// within 2^-18 of it, so round-to-nearest-even of v equals that of fl(x/sx) unless v lies
+// within 2^-15 of a half-integer; there the quotient itself (__fdiv_rn) is rounded.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -29,29 +38,46 @@ namespace i8mm {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kStripCols = kSmallStrip;
 constexpr int kStages = 4;
-constexpr int kABytes = kSmallBN * kBKBytes;   // 16 KB of Wq per stage
+constexpr int kABytes = kSmallBN * kBKBytes;       // 16 KB of Wq per stage
 constexpr int kBBytesPerKb = kSmallMP * kBKBytes;  // 2 KB of Xq per k-block
 constexpr uint32_t kTmemCols = 32;
 constexpr uint32_t kIdesc = idesc_i8_s32(kSmallBN, kSmallMP);
-
-__device__ __forceinline__ int quantize_value(float x, float s) {
-  const int q = __float2int_rn(__fdiv_rn(x, s));
-  return max(-127, min(127, q));
-}
-
-__device__ __forceinline__ float habs_f(uint32_t word, int hi) {
-  const unsigned short b = static_cast<unsigned short>(hi ? (word >> 16) : (word & 0xFFFFu));
-  return fabsf(__half2float(__ushort_as_half(b)));
-}
+constexpr int kQuantThreads = 192;  // warps 2..7
 
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
-
 __device__ __forceinline__ void fence_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Split cluster barrier (per thread, not warp-collective): every thread of every CTA of
+// the cluster arrives once per phase and waits before arriving again.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -68,73 +94,22 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
 }
 
-}  // namespace
-
-// ------------------------------------------------------------------ stats
-
-__global__ void __launch_bounds__(kThreads) small_stats_kernel(const SmallArgs a) {
-  __shared__ __half2 red[8][32][4];
-  __shared__ uint32_t flags[32];
-  grid_dependency_wait();
-  grid_launch_dependents();
-  const int strip = blockIdx.x;
-  const int chunk = threadIdx.x & 31;  // 8 columns each
-  const int rg = threadIdx.x >> 5;     // rows rg and rg + 8
-  const int col0 = strip * kStripCols + chunk * 8;
-  const bool valid = col0 < a.K;
-  uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-  if (valid && rg < a.M)
-    v0 = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(rg) * a.K + col0));
-  if (valid && rg + 8 < a.M)
-    v1 = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(rg + 8) * a.K + col0));
-  const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w};
-  const uint32_t w1[4] = {v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    __half2 h0 = *reinterpret_cast<const __half2*>(&w0[e]);
-    __half2 h1 = *reinterpret_cast<const __half2*>(&w1[e]);
-    red[rg][chunk][e] = __hmax2(__habs2(h0), __habs2(h1));
-  }
-  __syncthreads();
-  if (rg == 0) {
-    uint32_t bits8 = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      __half2 m = red[0][chunk][e];
-#pragma unroll
-      for (int r = 1; r < 8; ++r) m = __hmax2(m, red[r][chunk][e]);
-      if (__low2float(m) > a.threshold) bits8 |= 1u << (2 * e);
-      if (__high2float(m) > a.threshold) bits8 |= 1u << (2 * e + 1);
-    }
-    flags[chunk] = bits8;
-    uint32_t word = bits8 << (8 * (chunk & 3));
-    word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    word |= __shfl_xor_sync(0xffffffffu, word, 2);
-    const int w = strip * (kStripCols / 32) + chunk / 4;
-    if ((chunk & 3) == 0 && w < (a.K + 31) / 32) a.mask[w] = word;
-  }
-  __syncthreads();
-  const uint32_t bits8 = flags[chunk];
-  float r0 = 0.0f, r1 = 0.0f;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    if (!((bits8 >> e) & 1u)) {
-      r0 = fmaxf(r0, habs_f(w0[e / 2], e & 1));
-      r1 = fmaxf(r1, habs_f(w1[e / 2], e & 1));
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    r0 = fmaxf(r0, __shfl_xor_sync(0xffffffffu, r0, o));
-    r1 = fmaxf(r1, __shfl_xor_sync(0xffffffffu, r1, o));
-  }
-  if (chunk == 0) {
-    a.rowmax_part[strip * kSmallMP + rg] = r0;
-    a.rowmax_part[strip * kSmallMP + rg + 8] = r1;
-  }
+__device__ __forceinline__ float half_bits_to_float(uint32_t word, int hi) {
+  return __half2float(
+      __ushort_as_half(static_cast<unsigned short>(hi ? (word >> 16) : (word & 0xFFFFu))));
 }
 
-// ------------------------------------------------------------------ fused quantize + product
+// rne(fl(x / s)) clamped to [-127, 127]; rcp = 1/s rounded to nearest (see file comment)
+__device__ __forceinline__ int quantize_exact(float x, float s, float rcp) {
+  float v = x * rcp;
+  const float av = fabsf(v);
+  const float frac = av - floorf(av);
+  if (fabsf(frac - 0.5f) <= 0x1p-15f) v = __fdiv_rn(x, s);
+  const int q = __float2int_rn(v);
+  return max(-127, min(127, q));
+}
+
+}  // namespace
 
 struct SmallShared {
   uint64_t full[kStages];
@@ -144,34 +119,39 @@ struct SmallShared {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  int last;
   int epi_ok;
+  float rowmax_local[kSmallMP];  // read by the other CTAs of the cluster
+  float red[kQuantThreads / 32][kSmallMP];
   float sx[kSmallMP];
+  float rcp[kSmallMP];
   int zero_row[kSmallMP];
-  float psum[kSmallBN][kSmallMP + 1];  // this CTA's outlier term per channel (+1: no bank clash)
-  uint32_t mask[kSmallMaxKbPerSplit * 4];
+  uint8_t flags[kSmallMaxKbPerSplit * 16];  // outlier bits, 8 columns per byte
+  int32_t acc[kSmallBN][kSmallMP];          // this CTA's partial sums, read cluster-wide
+  float psum[kSmallBN][kSmallMP];           // this CTA's outlier term, read cluster-wide
 };
 
-size_t small_gemm_smem_bytes(int kb_per_split) {
+size_t small_smem_bytes(int kb_per_split) {
   return 1024 + static_cast<size_t>(kStages) * kABytes +
-         static_cast<size_t>(kb_per_split) * kBBytesPerKb + sizeof(SmallShared);
+         static_cast<size_t>(kb_per_split) * kBBytesPerKb + sizeof(SmallShared) + 16;
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
-    small_gemm_kernel(const __grid_constant__ CUtensorMap map_wq, const SmallArgs a) {
+    small_fused_kernel(const __grid_constant__ CUtensorMap map_wq, const SmallArgs a) {
   extern __shared__ uint8_t small_smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(small_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* a_stage = base;                                   // kStages x 16 KB
-  uint8_t* xq_tiles = base + kStages * kABytes;              // nkb x 2 KB
+  uint8_t* a_stage = base;                       // kStages x 16 KB
+  uint8_t* xq_tiles = base + kStages * kABytes;  // kb_max x 2 KB
   const int S = a.splits;
-  const int tile = blockIdx.x / S, split = blockIdx.x % S;
+  const int split = static_cast<int>(cluster_rank());
+  const int tile = blockIdx.x / S;
   const int n0 = tile * kSmallBN;
   const int kb_total = (a.K + kBKBytes - 1) / kBKBytes;
   const int kb_begin = static_cast<int>(static_cast<long long>(split) * kb_total / S);
   const int kb_end = static_cast<int>(static_cast<long long>(split + 1) * kb_total / S);
   const int nkb = kb_end - kb_begin;
-  SmallShared& sh = *reinterpret_cast<SmallShared*>(xq_tiles + nkb * kBBytesPerKb);
+  const int kb_max = (kb_total + S - 1) / S;  // the same in every CTA: a common smem layout
+  SmallShared& sh = *reinterpret_cast<SmallShared*>(xq_tiles + kb_max * kBBytesPerKb);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort = &sh.abort;
 
@@ -180,11 +160,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], 1);
     }
-    mbar_init(&sh.xq_ready, 192);
+    mbar_init(&sh.xq_ready, kQuantThreads);
     mbar_init(&sh.tmem_full, 1);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
-    sh.last = 0;
     fence_mbarrier_init();
   }
   if (threadIdx.x == 32) prefetch_tmap(&map_wq);
@@ -196,34 +175,38 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
+  // The inputs may be written by the previous launch on the stream: wait for it before
+  // the first read (everything above overlapped its tail).
+  grid_dependency_wait();
 
   if (warp == 0) {
+    cluster_arrive();  // phase 1 (row maxima) needs nothing from this warp
     if (lane == 0) {
-      // ---- Wq stream: starts before the stats kernel has finished (weights are constant)
+      // ---- TMA producer: the Wq slice, 128 channels x 128 bytes per stage
       bool ok = true;
+      int issued = 0;
       for (int j = 0; j < nkb; ++j) {
         const int s = j % kStages;
         if (j >= kStages &&
-            !mbar_wait_bounded(&sh.empty[s], static_cast<uint32_t>((j / kStages) - 1) & 1u, abort)) {
+            !mbar_wait_bounded(&sh.empty[s], static_cast<uint32_t>((j / kStages) - 1) & 1u,
+                               abort)) {
           ok = false;
-          int dummy = 0;
-          for (int d = j - kStages; d < j; ++d)  // let the copies in flight land
-            mbar_wait_bounded(&sh.full[d % kStages], static_cast<uint32_t>(d / kStages) & 1u,
-                              &dummy);
           break;
         }
         mbar_arrive_expect_tx(&sh.full[s], kABytes);
         tma_load_2d(&map_wq, a_stage + s * kABytes, &sh.full[s], (kb_begin + j) * kBKBytes, n0);
+        ++issued;
       }
+      int dummy = 0;  // every issued copy lands before the block may exit
+      for (int d = issued > kStages ? issued - kStages : 0; d < issued; ++d)
+        mbar_wait_bounded(&sh.full[d % kStages], static_cast<uint32_t>(d / kStages) & 1u, &dummy);
       if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
-      if (ok) {  // let every copy land before the block may exit
-        int dummy = 0;
-        for (int d = nkb > kStages ? nkb - kStages : 0; d < nkb; ++d)
-          mbar_wait_bounded(&sh.full[d % kStages], static_cast<uint32_t>(d / kStages) & 1u, &dummy);
-      }
     }
+    cluster_wait();
+    cluster_arrive();  // phase 2 (partial sums)
+    cluster_wait();
   } else if (warp == 1) {
-    grid_dependency_wait();
+    cluster_arrive();
     if (lane == 0) {
       // ---- MMA issuer
       bool ok = mbar_wait_bounded(&sh.xq_ready, 0, abort);
@@ -240,171 +223,190 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint32_t b0 = smem_addr(xq_tiles + j * kBBytesPerKb);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_i8(tmem, sw128_kmajor_desc(a0 + 32u * k), sw128_kmajor_desc(b0 + 32u * k), kIdesc,
-                   (j > 0 || k > 0) ? 1u : 0u);
+            mma_i8(tmem, sw128_kmajor_desc(a0 + 32u * k), sw128_kmajor_desc(b0 + 32u * k),
+                   kIdesc, (j > 0 || k > 0) ? 1u : 0u);
           mma_commit(&sh.empty[s]);
         }
         if (ok) mma_commit(&sh.tmem_full);
       }
-      mma_commit(&sh.drain);
+      mma_commit(&sh.drain);  // every MMA issued must finish before TMEM is freed
       int dummy = 0;
       mbar_wait_bounded(&sh.drain, 0, &dummy);
       if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
     }
+    cluster_wait();
+    cluster_arrive();
+    cluster_wait();
   } else {
-    // ---- warps 2..7: quantize this CTA's K-slice of X into the B operand
-    grid_dependency_wait();
+    // ---- warps 2..7: statistics and quantization of this K-slice of X
     const int tq = threadIdx.x - 64;  // 0..191
-    const int strips = (a.K + kStripCols - 1) / kStripCols;
+    const int col_begin = kb_begin * kBKBytes;
+    const int chunks = nkb * (kBKBytes / 8);  // 8 columns per chunk
+    float rmax[kSmallMP];
+#pragma unroll
+    for (int i = 0; i < kSmallMP; ++i) rmax[i] = 0.0f;
+    for (int c = tq; c < chunks; c += kQuantThreads) {
+      const int k = col_begin + c * 8;
+      uint4 v[kSmallMP];
+      __half2 cm[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cm[e] = __float2half2_rn(0.0f);
+#pragma unroll
+      for (int i = 0; i < kSmallMP; ++i) {
+        v[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < a.M && k < a.K)
+          v[i] = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * a.K + k));
+      }
+#pragma unroll
+      for (int i = 0; i < kSmallMP; ++i) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          cm[e] = __hmax2(cm[e], __habs2(*reinterpret_cast<const __half2*>(&w[e])));
+      }
+      uint32_t bits = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (__low2float(cm[e]) > a.threshold) bits |= 1u << (2 * e);
+        if (__high2float(cm[e]) > a.threshold) bits |= 1u << (2 * e + 1);
+      }
+      sh.flags[c] = static_cast<uint8_t>(bits);
+#pragma unroll
+      for (int i = 0; i < kSmallMP; ++i) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (!((bits >> e) & 1u))
+            rmax[i] = fmaxf(rmax[i], fabsf(half_bits_to_float(w[e / 2], e & 1)));
+      }
+    }
+    // row maxima of this slice: warp then block reduction
+#pragma unroll
+    for (int i = 0; i < kSmallMP; ++i) {
+      float m = rmax[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      rmax[i] = m;
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < kSmallMP; ++i) sh.red[warp - 2][i] = rmax[i];
+    }
+    named_barrier(1, kQuantThreads);
     if (tq < kSmallMP) {
-      float rm = 0.0f;
-      for (int s = 0; s < strips; ++s) rm = fmaxf(rm, __ldcg(a.rowmax_part + s * kSmallMP + tq));
-      sh.sx[tq] = (tq < a.M) ? __fdiv_rn(rm, 127.0f) : 0.0f;
-      sh.zero_row[tq] = (tq >= a.M) || rm == 0.0f;
+      float m = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kQuantThreads / 32; ++w) m = fmaxf(m, sh.red[w][tq]);
+      sh.rowmax_local[tq] = m;
     }
-    const int words = (a.K + 31) / 32;
-    for (int w = tq; w < nkb * 4; w += 192) {
-      const int gw = kb_begin * 4 + w;
-      sh.mask[w] = gw < words ? __ldcg(a.mask + gw) : 0u;
+    cluster_arrive();  // phase 1: every CTA's rowmax_local is written
+    cluster_wait();
+    if (tq < kSmallMP) {
+      float m = 0.0f;
+      const uint32_t local = smem_addr(&sh.rowmax_local[tq]);
+      for (int r = 0; r < S; ++r) m = fmaxf(m, ld_cluster_f32(map_rank(local, r)));
+      const float s = __fdiv_rn(m, 127.0f);
+      sh.sx[tq] = (tq < a.M) ? s : 0.0f;
+      sh.rcp[tq] = (tq < a.M && m > 0.0f) ? __frcp_rn(s) : 0.0f;
+      sh.zero_row[tq] = (tq >= a.M) || m == 0.0f;
     }
-    named_barrier(1, 192);
-    const int chunks_per_row = nkb * (kBKBytes / 8);  // 8 int8 codes per chunk
-    for (int u = tq; u < kSmallMP * chunks_per_row; u += 192) {
-      const int r = u / chunks_per_row, c = u % chunks_per_row;
-      const int k = kb_begin * kBKBytes + c * 8;
+    named_barrier(1, kQuantThreads);
+    // quantize into the B operand: row i, k-block kbl, byte kk at
+    //   kbl*2048 + (i/8)*1024 + (i%8)*128 + ((kk/16) ^ (i%8))*16 + kk%16
+    for (int u = tq; u < kSmallMP * chunks; u += kQuantThreads) {
+      const int i = u / chunks, c = u % chunks;
+      const int k = col_begin + c * 8;
       uint2 q = make_uint2(0u, 0u);
-      if (r < a.M && k < a.K && !sh.zero_row[r]) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(r) * a.K + k));
-        const uint32_t bits = (sh.mask[(c * 8) >> 5] >> ((c * 8) & 31)) & 0xFFu;
+      if (!sh.zero_row[i] && k < a.K) {
+        const uint4 v =
+            __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * a.K + k));
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        const float s = sh.sx[r];
+        const uint32_t bits = sh.flags[c];
+        const float s = sh.sx[i], r = sh.rcp[i];
         uint32_t p[2] = {0u, 0u};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           if ((bits >> e) & 1u) continue;
-          const unsigned short hb = static_cast<unsigned short>((w[e / 2] >> (16 * (e & 1))) & 0xFFFFu);
-          const int qv = quantize_value(__half2float(__ushort_as_half(hb)), s);
+          const int qv = quantize_exact(half_bits_to_float(w[e / 2], e & 1), s, r);
           p[e / 4] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
         }
         q = make_uint2(p[0], p[1]);
       }
       const int kbl = c / 16, kk = (c % 16) * 8;
-      uint8_t* dst = xq_tiles + kbl * kBBytesPerKb + (r / 8) * 1024 + (r % 8) * 128 +
-                     (((kk / 16) ^ (r % 8)) * 16) + (kk % 16);
+      uint8_t* dst = xq_tiles + kbl * kBBytesPerKb + (i / 8) * 1024 + (i % 8) * 128 +
+                     (((kk / 16) ^ (i % 8)) * 16) + (kk % 16);
       *reinterpret_cast<uint2*>(dst) = q;
     }
     fence_async_shared();
     mbar_arrive(&sh.xq_ready);
 
     if (warp >= 4) {
-      // ---- warps 4..7 own TMEM lane quadrants 0..3, i.e. channels 32q .. 32q+31
+      // ---- warps 4..7: TMEM lane quadrant q <-> channels 32q .. 32q+31
       const int quad = warp & 3;
       const int n = quad * 32 + lane, gn = n0 + n;
-      // The fp16 outlier term of the outlier columns inside this CTA's K-slice, computed
-      // while the MMAs run: P[i] = sum_j X[i,j] * fp16(Wq[gn,j] * w_scale[gn]).
-      {
-        float P[kSmallMP];
+      // fp16 outlier term of the outlier columns in this slice, while the MMAs run
+      float P[kSmallMP];
 #pragma unroll
-        for (int i = 0; i < kSmallMP; ++i) P[i] = 0.0f;
-        if (gn < a.N) {
-          const float sw_n = a.w_scale[gn];
-          const int8_t* wrow = a.Wq + static_cast<size_t>(gn) * a.K;
-          for (int w = 0; w < nkb * 4; ++w) {
-            uint32_t bits = sh.mask[w];
-            while (bits) {
-              const int j = kb_begin * kBKBytes + w * 32 + __ffs(bits) - 1;
-              bits &= bits - 1u;
-              const float wv = __half2float(__float2half_rn(static_cast<float>(wrow[j]) * sw_n));
+      for (int i = 0; i < kSmallMP; ++i) P[i] = 0.0f;
+      if (gn < a.N) {
+        const float sw_n = a.w_scale[gn];
+        const int8_t* wrow = a.Wq + static_cast<size_t>(gn) * a.K;
+        for (int c = 0; c < chunks; ++c) {
+          uint32_t bits = sh.flags[c];
+          while (bits) {
+            const int j = col_begin + c * 8 + __ffs(bits) - 1;
+            bits &= bits - 1u;
+            const float wv = __half2float(__float2half_rn(static_cast<float>(wrow[j]) * sw_n));
 #pragma unroll
-              for (int i = 0; i < kSmallMP; ++i)
-                if (i < a.M) P[i] += wv * __half2float(a.X[static_cast<size_t>(i) * a.K + j]);
-            }
+            for (int i = 0; i < kSmallMP; ++i)
+              if (i < a.M) P[i] += wv * __half2float(a.X[static_cast<size_t>(i) * a.K + j]);
           }
         }
-#pragma unroll
-        for (int i = 0; i < kSmallMP; ++i) sh.psum[n][i] = P[i];
       }
-      int32_t acc[kSmallMP];
+#pragma unroll
+      for (int i = 0; i < kSmallMP; ++i) sh.psum[n][i] = P[i];
       mbar_wait_bounded(&sh.tmem_full, 0, abort);
-      // one decision for all 128 epilogue threads, so the barriers below cannot split
+      // one decision for the 128 epilogue threads
       named_barrier(2, 128);
       if (threadIdx.x == 128) sh.epi_ok = (*abort == 0);
       named_barrier(2, 128);
-      const bool ok = sh.epi_ok != 0;
       tc_fence_after();
       uint32_t r[16];
       __syncwarp();
       tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16), r);
       tmem_ld_wait();
+      const bool ok = sh.epi_ok != 0;
 #pragma unroll
-      for (int i = 0; i < kSmallMP; ++i) acc[i] = ok ? static_cast<int32_t>(r[i]) : 0;
-      bool finish = ok;
+      for (int i = 0; i < kSmallMP; ++i) sh.acc[n][i] = ok ? static_cast<int32_t>(r[i]) : 0;
       if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
-      if (ok && S > 1) {
-        const size_t slot = ((static_cast<size_t>(tile) * S + split) * kSmallBN + n) * kSmallMP;
-        int4* ip = reinterpret_cast<int4*>(a.partials + slot);
-        float4* fp = reinterpret_cast<float4*>(a.fpartials + slot);
-#pragma unroll
-        for (int v = 0; v < kSmallMP / 4; ++v) {
-          __stcg(ip + v, make_int4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]));
-          __stcg(fp + v, make_float4(sh.psum[n][4 * v], sh.psum[n][4 * v + 1],
-                                     sh.psum[n][4 * v + 2], sh.psum[n][4 * v + 3]));
-        }
-        __threadfence();
-        named_barrier(2, 128);
-        if (threadIdx.x == 128) {
-          const unsigned old = atomicAdd(a.counters + tile, 1u);
-          const int last = old == static_cast<unsigned>(S - 1);
-          if (last) atomicExch(a.counters + tile, 0u);  // ready for the next call
-          sh.last = last;
-        }
-        named_barrier(2, 128);
-        finish = sh.last != 0;
-        if (finish) {
-          __threadfence();
-          float P[kSmallMP];
-#pragma unroll
-          for (int i = 0; i < kSmallMP; ++i) {
-            acc[i] = 0;
-            P[i] = 0.0f;
-          }
-          for (int s2 = 0; s2 < S; ++s2) {  // fixed order: the same bits on every call
-            const size_t o = ((static_cast<size_t>(tile) * S + s2) * kSmallBN + n) * kSmallMP;
-            const int4* ip2 = reinterpret_cast<const int4*>(a.partials + o);
-            const float4* fp2 = reinterpret_cast<const float4*>(a.fpartials + o);
-#pragma unroll
-            for (int v = 0; v < kSmallMP / 4; ++v) {
-              const int4 t = __ldcg(ip2 + v);
-              const float4 f = __ldcg(fp2 + v);
-              acc[4 * v] += t.x;
-              acc[4 * v + 1] += t.y;
-              acc[4 * v + 2] += t.z;
-              acc[4 * v + 3] += t.w;
-              P[4 * v] += f.x;
-              P[4 * v + 1] += f.y;
-              P[4 * v + 2] += f.z;
-              P[4 * v + 3] += f.w;
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < kSmallMP; ++i) sh.psum[n][i] = P[i];
-        }
+    }
+    cluster_arrive();  // phase 2: every CTA's partial sums are in its shared memory
+    cluster_wait();
+    // ---- sum the S partials of this CTA's share of the output, in rank order
+    const int outs = kSmallBN * a.M;
+    const int per = (outs + S - 1) / S;
+    const int o_begin = split * per, o_end = min(outs, o_begin + per);
+    for (int o = o_begin + tq; o < o_end; o += kQuantThreads) {
+      const int n = o / a.M, i = o % a.M, gn = n0 + n;
+      if (gn >= a.N) continue;
+      const uint32_t acc_l = smem_addr(&sh.acc[n][i]);
+      const uint32_t p_l = smem_addr(&sh.psum[n][i]);
+      int32_t acc = 0;
+      float P = 0.0f;
+      for (int r = 0; r < S; ++r) {
+        acc += ld_cluster_s32(map_rank(acc_l, r));
+        P += ld_cluster_f32(map_rank(p_l, r));
       }
-      if (finish && gn < a.N) {
-        const float b = a.bias ? __half2float(a.bias[gn]) : 0.0f;
-        const float swn = a.w_scale[gn];
-#pragma unroll
-        for (int i = 0; i < kSmallMP; ++i) {
-          if (i < a.M) {
-            const float y = static_cast<float>(acc[i]) * sh.sx[i] * swn + sh.psum[n][i] + b;
-            a.Y[static_cast<size_t>(i) * a.N + gn] = __float2half_rn(y);
-            if (a.acc) a.acc[static_cast<size_t>(i) * a.N + gn] = acc[i];
-          }
-        }
-      }
+      const float b = a.bias ? __half2float(a.bias[gn]) : 0.0f;
+      const float y = static_cast<float>(acc) * sh.sx[i] * a.w_scale[gn] + P + b;
+      a.Y[static_cast<size_t>(i) * a.N + gn] = __float2half_rn(y);
+      if (a.acc) a.acc[static_cast<size_t>(i) * a.N + gn] = acc;
     }
   }
 
+  // no CTA may leave while the others can still read its shared memory
+  cluster_arrive();
+  cluster_wait();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -415,59 +417,46 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 // ------------------------------------------------------------------ host side
 
-SmallPlan plan_small(int M, int N, int K, int num_sms) {
+SmallPlan plan_small(int N, int K) {
   SmallPlan p;
   p.tiles = (N + kSmallBN - 1) / kSmallBN;
   const int kb_total = (K + kBKBytes - 1) / kBKBytes;
-  int S = static_cast<int>((2.0 * num_sms) / p.tiles + 0.5);
-  S = S < 1 ? 1 : S;
-  const int need = (kb_total + kSmallMaxKbPerSplit - 1) / kSmallMaxKbPerSplit;
-  if (S < need) S = need;
-  if (S > kb_total) S = kb_total;
-  if (S > kSmallMaxSplits) S = kSmallMaxSplits;
-  p.splits = S;
-  p.kb_per_split = (kb_total + S - 1) / S;
-  p.strips = (K + kStripCols - 1) / kStripCols;
-  (void)M;
+  p.splits = kb_total < kSmallMaxSplits ? kb_total : kSmallMaxSplits;
+  p.kb_per_split = (kb_total + p.splits - 1) / p.splits;
   return p;
 }
 
-cudaError_t launch_small_stats(const SmallArgs& a, const SmallPlan& p, cudaStream_t stream,
-                               bool pdl) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.strips);
-  cfg.blockDim = dim3(kThreads);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, small_stats_kernel, a);
+bool small_path_fits(int M, int K) {
+  if (M > kSmallMP) return false;
+  const SmallPlan p = plan_small(1, K);
+  return p.kb_per_split <= kSmallMaxKbPerSplit;
 }
 
-cudaError_t launch_small_gemm(const CUtensorMap& map_wq, const SmallArgs& a, const SmallPlan& p,
-                              cudaStream_t stream, bool pdl) {
-  const size_t smem = small_gemm_smem_bytes(p.kb_per_split);
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(small_gemm_kernel,
+cudaError_t launch_small(const CUtensorMap& map_wq, const SmallArgs& a, const SmallPlan& p,
+                         cudaStream_t stream, bool pdl) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(small_fused_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(small_gemm_smem_bytes(kSmallMaxKbPerSplit)));
+                                         static_cast<int>(small_smem_bytes(kSmallMaxKbPerSplit)));
     if (e != cudaSuccess) return e;
-    configured = small_gemm_smem_bytes(kSmallMaxKbPerSplit);
+    configured = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.tiles * p.splits);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = small_smem_bytes(p.kb_per_split);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, small_gemm_kernel, map_wq, a);
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, small_fused_kernel, map_wq, a);
 }
 
 }  // namespace i8mm

@@ -262,3 +262,27 @@ def test_few_token_path_many_calls_one_workspace():
     for Y in Ys:
         np.testing.assert_array_equal(f16_bits(to_np(Y)), f16_bits(first))
     assert i8.int8_read_device_status(ws[:4].view(torch.int32)) == 0
+
+
+@pytest.mark.parametrize("M", [4, 16, 40])
+def test_quantizer_ties_and_near_ties_exact(M):
+    """Values placed on and next to half-integer quotients; W = I makes acc = 127 * Xq."""
+    K = 256
+    rng = np.random.default_rng(100 + M)
+    X = rng.standard_normal((M, K)) * 0.05
+    for i in range(M):
+        a = float(np.float16(1.0029296875 + 0.0078125 * i))  # row absmax
+        X[i, 0] = a
+        ks = rng.integers(-126, 126, size=120)
+        X[i, 1:121] = (ks + 0.5) * a / 127.0           # lands on or near x/s = k + 1/2
+    X[0, 1] = 0.50146484375                            # the golden division-by-scale case
+    X[0, 0] = 1.0029296875
+    X = X.astype(np.float16)
+    W = np.eye(K, dtype=np.float16)
+    Y, acc = check_forward_acc(X, W, None, math.inf)
+    Wq, sw = oracle.quant_weight(W)
+    assert (np.diag(Wq) == 127).all()
+    mask, _ = oracle.outlier_columns(X, math.inf)
+    Xq, _ = oracle.quantize_rows(X, mask)
+    np.testing.assert_array_equal(acc, 127 * Xq.astype(np.int32))
+    assert Xq[0, 1] == 63
