@@ -238,25 +238,30 @@ __global__ void __launch_bounds__(kThreads, 2)
     cluster_arrive();
     cluster_wait();
   } else {
-    // ---- warps 2..7: statistics and quantization of this K-slice of X
+    // ---- warps 2..7: statistics and quantization of this K-slice of X.  Thread tq owns
+    // 8-column chunks c = tq, tq + 192, ...; when it owns one chunk, that chunk's values
+    // for all rows stay in registers from the statistics pass to the quantization pass.
     const int tq = threadIdx.x - 64;  // 0..191
     const int col_begin = kb_begin * kBKBytes;
-    const int chunks = nkb * (kBKBytes / 8);  // 8 columns per chunk
+    const int chunks = nkb * (kBKBytes / 8);
     float rmax[kSmallMP];
 #pragma unroll
     for (int i = 0; i < kSmallMP; ++i) rmax[i] = 0.0f;
-    for (int c = tq; c < chunks; c += kQuantThreads) {
+    uint4 v[kSmallMP];
+    auto load_chunk = [&](int c) {
       const int k = col_begin + c * 8;
-      uint4 v[kSmallMP];
-      __half2 cm[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) cm[e] = __float2half2_rn(0.0f);
 #pragma unroll
       for (int i = 0; i < kSmallMP; ++i) {
         v[i] = make_uint4(0u, 0u, 0u, 0u);
         if (i < a.M && k < a.K)
           v[i] = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * a.K + k));
       }
+    };
+    for (int c = tq; c < chunks; c += kQuantThreads) {
+      load_chunk(c);
+      __half2 cm[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cm[e] = __float2half2_rn(0.0f);
 #pragma unroll
       for (int i = 0; i < kSmallMP; ++i) {
         const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
@@ -302,9 +307,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     cluster_arrive();  // phase 1: every CTA's rowmax_local is written
     cluster_wait();
     if (tq < kSmallMP) {
-      float m = 0.0f;
       const uint32_t local = smem_addr(&sh.rowmax_local[tq]);
-      for (int r = 0; r < S; ++r) m = fmaxf(m, ld_cluster_f32(map_rank(local, r)));
+      float peer[kSmallMaxSplits];
+#pragma unroll
+      for (int r = 0; r < kSmallMaxSplits; ++r)  // all remote loads in flight at once
+        peer[r] = r < S ? ld_cluster_f32(map_rank(local, r)) : 0.0f;
+      float m = 0.0f;
+#pragma unroll
+      for (int r = 0; r < kSmallMaxSplits; ++r) m = fmaxf(m, peer[r]);
       const float s = __fdiv_rn(m, 127.0f);
       sh.sx[tq] = (tq < a.M) ? s : 0.0f;
       sh.rcp[tq] = (tq < a.M && m > 0.0f) ? __frcp_rn(s) : 0.0f;
@@ -313,29 +323,29 @@ __global__ void __launch_bounds__(kThreads, 2)
     named_barrier(1, kQuantThreads);
     // quantize into the B operand: row i, k-block kbl, byte kk at
     //   kbl*2048 + (i/8)*1024 + (i%8)*128 + ((kk/16) ^ (i%8))*16 + kk%16
-    for (int u = tq; u < kSmallMP * chunks; u += kQuantThreads) {
-      const int i = u / chunks, c = u % chunks;
-      const int k = col_begin + c * 8;
-      uint2 q = make_uint2(0u, 0u);
-      if (!sh.zero_row[i] && k < a.K) {
-        const uint4 v =
-            __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * a.K + k));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        const uint32_t bits = sh.flags[c];
-        const float s = sh.sx[i], r = sh.rcp[i];
-        uint32_t p[2] = {0u, 0u};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if ((bits >> e) & 1u) continue;
-          const int qv = quantize_exact(half_bits_to_float(w[e / 2], e & 1), s, r);
-          p[e / 4] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
-        }
-        q = make_uint2(p[0], p[1]);
-      }
+    for (int c = tq; c < chunks; c += kQuantThreads) {
+      if (chunks > kQuantThreads) load_chunk(c);  // wide slices reload (L1/L2 hits)
+      const uint32_t bits = sh.flags[c];
       const int kbl = c / 16, kk = (c % 16) * 8;
-      uint8_t* dst = xq_tiles + kbl * kBBytesPerKb + (i / 8) * 1024 + (i % 8) * 128 +
-                     (((kk / 16) ^ (i % 8)) * 16) + (kk % 16);
-      *reinterpret_cast<uint2*>(dst) = q;
+#pragma unroll
+      for (int i = 0; i < kSmallMP; ++i) {
+        uint2 q = make_uint2(0u, 0u);
+        if (!sh.zero_row[i]) {
+          const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+          const float s = sh.sx[i], r = sh.rcp[i];
+          uint32_t p[2] = {0u, 0u};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if ((bits >> e) & 1u) continue;
+            const int qv = quantize_exact(half_bits_to_float(w[e / 2], e & 1), s, r);
+            p[e / 4] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
+          }
+          q = make_uint2(p[0], p[1]);
+        }
+        uint8_t* dst = xq_tiles + kbl * kBBytesPerKb + (i / 8) * 1024 + (i % 8) * 128 +
+                       (((kk / 16) ^ (i % 8)) * 16) + (kk % 16);
+        *reinterpret_cast<uint2*>(dst) = q;
+      }
     }
     fence_async_shared();
     mbar_arrive(&sh.xq_ready);
@@ -391,11 +401,19 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (gn >= a.N) continue;
       const uint32_t acc_l = smem_addr(&sh.acc[n][i]);
       const uint32_t p_l = smem_addr(&sh.psum[n][i]);
+      int32_t pa[kSmallMaxSplits];
+      float pp[kSmallMaxSplits];
+#pragma unroll
+      for (int r = 0; r < kSmallMaxSplits; ++r) {  // all remote loads in flight at once
+        pa[r] = r < S ? ld_cluster_s32(map_rank(acc_l, r)) : 0;
+        pp[r] = r < S ? ld_cluster_f32(map_rank(p_l, r)) : 0.0f;
+      }
       int32_t acc = 0;
       float P = 0.0f;
-      for (int r = 0; r < S; ++r) {
-        acc += ld_cluster_s32(map_rank(acc_l, r));
-        P += ld_cluster_f32(map_rank(p_l, r));
+#pragma unroll
+      for (int r = 0; r < kSmallMaxSplits; ++r) {  // rank order: the same bits every call
+        acc += pa[r];
+        P += pp[r];
       }
       const float b = a.bias ? __half2float(a.bias[gn]) : 0.0f;
       const float y = static_cast<float>(acc) * sh.sx[i] * a.w_scale[gn] + P + b;
