@@ -5,7 +5,7 @@
 // once at HBM speed and everything else hidden behind that stream.  Each output tile of
 // 128 channels is computed by a thread-block cluster of S CTAs that split K (split-K).
 // Each CTA of a cluster:
-//   1. starts the TMA stream of its Wq slice [128 channels x K/S] into a 4-stage ring;
+//   1. starts the TMA stream of its Wq slice [128 channels x K/S] into a 6-stage ring;
 //   2. reads its K-slice of X for all M rows and finds, per column, whether any |x|
 //      exceeds the threshold (the outlier columns of [P2] "8位量化实战：离群值处理与显存
 //      优化避坑指南" section 2.3 -- complete per slice, since every row is present) and,
@@ -38,7 +38,7 @@ namespace i8mm {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kABytes = kSmallBN * kBKBytes;       // 16 KB of Wq per stage
 constexpr int kBBytesPerKb = kSmallMP * kBKBytes;  // 2 KB of Xq per k-block
 constexpr uint32_t kTmemCols = 32;
@@ -135,7 +135,7 @@ size_t small_smem_bytes(int kb_per_split) {
          static_cast<size_t>(kb_per_split) * kBBytesPerKb + sizeof(SmallShared) + 16;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     small_fused_kernel(const __grid_constant__ CUtensorMap map_wq, const SmallArgs a) {
   extern __shared__ uint8_t small_smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
@@ -435,31 +435,89 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 // ------------------------------------------------------------------ host side
 
+namespace {
+
+int kb_per_split(int kb_total, int S) { return (kb_total + S - 1) / S; }
+
+cudaError_t configure_small() {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev == configured_device) return cudaSuccess;
+  e = cudaFuncSetAttribute(small_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(small_smem_bytes(kSmallMaxKbPerSplit)));
+  if (e == cudaSuccess) configured_device = dev;
+  return e;
+}
+
+// Clusters of S CTAs that can be resident at once with this shared-memory footprint.
+int max_active_clusters(int S, size_t smem) {
+  struct Entry { int dev, S; size_t smem; int n; };
+  static Entry cache[32];
+  static int used = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].dev == dev && cache[i].S == S && cache[i].smem == smem) return cache[i].n;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, small_fused_kernel, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  if (used < 32) cache[used++] = {dev, S, smem, n};
+  return n;
+}
+
+}  // namespace
+
+// Cluster size S (CTAs splitting K per 128-channel tile): the one that minimises
+// (waves of resident clusters) x (k-blocks per CTA), preferring larger S on ties.
 SmallPlan plan_small(int N, int K) {
   SmallPlan p;
   p.tiles = (N + kSmallBN - 1) / kSmallBN;
   const int kb_total = (K + kBKBytes - 1) / kBKBytes;
-  p.splits = kb_total < kSmallMaxSplits ? kb_total : kSmallMaxSplits;
-  p.kb_per_split = (kb_total + p.splits - 1) / p.splits;
+  p.splits = 0;
+  long long best = 0;
+  if (configure_small() != cudaSuccess) cudaGetLastError();
+  for (int S = kSmallMaxSplits; S >= 1; S /= 2) {
+    if (S > kb_total) continue;
+    const int kbps = kb_per_split(kb_total, S);
+    if (kbps > kSmallMaxKbPerSplit) continue;
+    const int act = max_active_clusters(S, small_smem_bytes(kbps));
+    const long long cost = static_cast<long long>((p.tiles + act - 1) / act) * kbps;
+    if (p.splits == 0 || cost < best) {
+      best = cost;
+      p.splits = S;
+    }
+  }
+  if (p.splits == 0) p.splits = 1;
+  p.kb_per_split = kb_per_split(kb_total, p.splits);
   return p;
 }
 
 bool small_path_fits(int M, int K) {
   if (M > kSmallMP) return false;
-  const SmallPlan p = plan_small(1, K);
-  return p.kb_per_split <= kSmallMaxKbPerSplit;
+  const int kb_total = (K + kBKBytes - 1) / kBKBytes;
+  const int S = kb_total < kSmallMaxSplits ? kb_total : kSmallMaxSplits;
+  return kb_per_split(kb_total, S) <= kSmallMaxKbPerSplit;
 }
 
 cudaError_t launch_small(const CUtensorMap& map_wq, const SmallArgs& a, const SmallPlan& p,
                          cudaStream_t stream, bool pdl) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(small_fused_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(small_smem_bytes(kSmallMaxKbPerSplit)));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t e = configure_small();
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.tiles * p.splits);
   cfg.blockDim = dim3(kThreads);
