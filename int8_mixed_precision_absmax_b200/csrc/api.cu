@@ -161,7 +161,7 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
                const void* bias, int N, float threshold, void* Y, int32_t* acc,
                void* workspace, const ForwardPlan& p, cudaStream_t stream, bool pdl) {
   if (small_path_fits(M, K)) {
-    const SmallPlan sp = plan_small(N, K);
+    const SmallPlan sp = plan_small(M, N, K);
     const SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p, sp);
     CUtensorMap map;
     if (!encode_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kSmallBN))

@@ -27,7 +27,7 @@ namespace i8mm {
 constexpr int kSmallMP = 16;             // tokens per MMA (N of the swapped product)
 constexpr int kSmallBN = 128;            // output channels per tile (M of the MMA)
 constexpr int kSmallMaxSplits = 8;       // CTAs per cluster (portable cluster size)
-constexpr int kSmallMaxKbPerSplit = 32;  // 128-byte k-blocks of Xq one CTA keeps in smem
+constexpr int kSmallMaxKbPerSplit = 16;  // 128-byte k-blocks of X / Xq one CTA keeps in smem
 
 struct WorkspaceLayout {
   size_t header, mask, cols, xscale, xq, xo, wo, total;
@@ -100,7 +100,7 @@ struct SmallArgs {
 struct SmallPlan {
   int tiles, splits, kb_per_split;
 };
-SmallPlan plan_small(int N, int K);
+SmallPlan plan_small(int M, int N, int K);
 bool small_path_fits(int M, int K);
 cudaError_t launch_small(const CUtensorMap& map_wq, const SmallArgs& a, const SmallPlan& p,
                          cudaStream_t stream, bool pdl);

@@ -43,7 +43,9 @@ constexpr int kABytes = kSmallBN * kBKBytes;       // 16 KB of Wq per stage
 constexpr int kBBytesPerKb = kSmallMP * kBKBytes;  // 2 KB of Xq per k-block
 constexpr uint32_t kTmemCols = 32;
 constexpr uint32_t kIdesc = idesc_i8_s32(kSmallBN, kSmallMP);
-constexpr int kQuantThreads = 192;  // warps 2..7
+constexpr int kStatThreads = 192;   // warps 2..7: statistics of the slice
+constexpr int kQuantThreads = 128;  // warps 4..7: quantization and the accumulator drain
+constexpr int kOutlierThreads = 64; // warps 2..3: the fp16 outlier term
 
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -101,11 +103,10 @@ __device__ __forceinline__ float half_bits_to_float(uint32_t word, int hi) {
 
 // rne(fl(x / s)) clamped to [-127, 127]; rcp = 1/s rounded to nearest (see file comment)
 __device__ __forceinline__ int quantize_exact(float x, float s, float rcp) {
-  float v = x * rcp;
-  const float av = fabsf(v);
-  const float frac = av - floorf(av);
-  if (fabsf(frac - 0.5f) <= 0x1p-15f) v = __fdiv_rn(x, s);
-  const int q = __float2int_rn(v);
+  const float v = x * rcp;
+  const float d = fabsf(v - rintf(v));  // distance to the nearest integer, exact
+  int q = __float2int_rn(v);
+  if (fabsf(d - 0.5f) <= 0x1p-15f) q = __float2int_rn(__fdiv_rn(x, s));  // near a tie
   return max(-127, min(127, q));
 }
 
@@ -121,7 +122,7 @@ struct SmallShared {
   int abort;
   int epi_ok;
   float rowmax_local[kSmallMP];  // read by the other CTAs of the cluster
-  float red[kQuantThreads / 32][kSmallMP];
+  float red[kStatThreads / 32][kSmallMP];
   float sx[kSmallMP];
   float rcp[kSmallMP];
   int zero_row[kSmallMP];
@@ -130,9 +131,11 @@ struct SmallShared {
   float psum[kSmallBN][kSmallMP];           // this CTA's outlier term, read cluster-wide
 };
 
-size_t small_smem_bytes(int kb_per_split) {
+// [Wq ring | Xq tiles | X slice (M rows) | SmallShared]
+size_t small_smem_bytes(int kb_per_split, int M) {
   return 1024 + static_cast<size_t>(kStages) * kABytes +
-         static_cast<size_t>(kb_per_split) * kBBytesPerKb + sizeof(SmallShared) + 16;
+         static_cast<size_t>(kb_per_split) * kBBytesPerKb +
+         static_cast<size_t>(M) * kb_per_split * kBKBytes * sizeof(__half) + sizeof(SmallShared) + 16;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -151,7 +154,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kb_end = static_cast<int>(static_cast<long long>(split + 1) * kb_total / S);
   const int nkb = kb_end - kb_begin;
   const int kb_max = (kb_total + S - 1) / S;  // the same in every CTA: a common smem layout
-  SmallShared& sh = *reinterpret_cast<SmallShared*>(xq_tiles + kb_max * kBBytesPerKb);
+  __half* x_slice = reinterpret_cast<__half*>(xq_tiles + kb_max * kBBytesPerKb);  // [M][kb_max*128]
+  const int xs_ld = kb_max * kBKBytes;
+  SmallShared& sh = *reinterpret_cast<SmallShared*>(x_slice + static_cast<size_t>(a.M) * xs_ld);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort = &sh.abort;
 
@@ -160,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], 1);
     }
-    mbar_init(&sh.xq_ready, kQuantThreads);
+    mbar_init(&sh.xq_ready, kQuantThreads);  // warps 4..7
     mbar_init(&sh.tmem_full, 1);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -238,32 +243,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_arrive();
     cluster_wait();
   } else {
-    // ---- warps 2..7: statistics and quantization of this K-slice of X.  Thread tq owns
-    // 8-column chunks c = tq, tq + 192, ...; when it owns one chunk, that chunk's values
-    // for all rows stay in registers from the statistics pass to the quantization pass.
+    // ---- warps 2..7: statistics of this K-slice of X.  Thread tq owns 8-column chunks
+    // c = tq, tq + 192, ... for all rows; the slice is also staged in shared memory.
     const int tq = threadIdx.x - 64;  // 0..191
     const int col_begin = kb_begin * kBKBytes;
     const int chunks = nkb * (kBKBytes / 8);
     float rmax[kSmallMP];
 #pragma unroll
     for (int i = 0; i < kSmallMP; ++i) rmax[i] = 0.0f;
-    uint4 v[kSmallMP];
-    auto load_chunk = [&](int c) {
+    for (int c = tq; c < chunks; c += kStatThreads) {
       const int k = col_begin + c * 8;
+      uint4 v[kSmallMP];
 #pragma unroll
       for (int i = 0; i < kSmallMP; ++i) {
         v[i] = make_uint4(0u, 0u, 0u, 0u);
         if (i < a.M && k < a.K)
           v[i] = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * a.K + k));
       }
-    };
-    for (int c = tq; c < chunks; c += kQuantThreads) {
-      load_chunk(c);
       __half2 cm[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) cm[e] = __float2half2_rn(0.0f);
 #pragma unroll
       for (int i = 0; i < kSmallMP; ++i) {
+        if (i < a.M) *reinterpret_cast<uint4*>(x_slice + static_cast<size_t>(i) * xs_ld + c * 8) = v[i];
         const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -297,89 +299,104 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < kSmallMP; ++i) sh.red[warp - 2][i] = rmax[i];
     }
-    named_barrier(1, kQuantThreads);
+    named_barrier(1, kStatThreads);  // flags, x_slice and red are complete
     if (tq < kSmallMP) {
       float m = 0.0f;
 #pragma unroll
-      for (int w = 0; w < kQuantThreads / 32; ++w) m = fmaxf(m, sh.red[w][tq]);
+      for (int w = 0; w < kStatThreads / 32; ++w) m = fmaxf(m, sh.red[w][tq]);
       sh.rowmax_local[tq] = m;
     }
     cluster_arrive();  // phase 1: every CTA's rowmax_local is written
-    cluster_wait();
-    if (tq < kSmallMP) {
-      const uint32_t local = smem_addr(&sh.rowmax_local[tq]);
-      float peer[kSmallMaxSplits];
+
+    if (warp < 4) {
+      // ---- warps 2..3: the fp16 outlier term of the outlier columns in this slice,
+      // P[n][i] = sum_j X[i,j] * fp16(Wq[n0+n, j] * w_scale[n0+n]), channels tq and tq + 64.
+      // It needs no row scale, so it runs while the cluster agrees on the scales.
+      float P0[kSmallMP], P1[kSmallMP];
 #pragma unroll
-      for (int r = 0; r < kSmallMaxSplits; ++r)  // all remote loads in flight at once
-        peer[r] = r < S ? ld_cluster_f32(map_rank(local, r)) : 0.0f;
-      float m = 0.0f;
+      for (int i = 0; i < kSmallMP; ++i) P0[i] = P1[i] = 0.0f;
+      const int g0 = n0 + tq, g1 = n0 + tq + 64;
+      const float s0 = g0 < a.N ? a.w_scale[g0] : 0.0f;
+      const float s1 = g1 < a.N ? a.w_scale[g1] : 0.0f;
+      const int8_t* w0row = a.Wq + static_cast<size_t>(g0 < a.N ? g0 : 0) * a.K;
+      const int8_t* w1row = a.Wq + static_cast<size_t>(g1 < a.N ? g1 : 0) * a.K;
+      for (int c = 0; c < chunks; ++c) {
+        uint32_t bits = sh.flags[c];
+        while (bits) {
+          const int j = col_begin + c * 8 + __ffs(bits) - 1;
+          bits &= bits - 1u;
+          const float w0 = __half2float(__float2half_rn(static_cast<float>(w0row[j]) * s0));
+          const float w1 = __half2float(__float2half_rn(static_cast<float>(w1row[j]) * s1));
+          const __half* xc = x_slice + (j - col_begin);
 #pragma unroll
-      for (int r = 0; r < kSmallMaxSplits; ++r) m = fmaxf(m, peer[r]);
-      const float s = __fdiv_rn(m, 127.0f);
-      sh.sx[tq] = (tq < a.M) ? s : 0.0f;
-      sh.rcp[tq] = (tq < a.M && m > 0.0f) ? __frcp_rn(s) : 0.0f;
-      sh.zero_row[tq] = (tq >= a.M) || m == 0.0f;
-    }
-    named_barrier(1, kQuantThreads);
-    // quantize into the B operand: row i, k-block kbl, byte kk at
-    //   kbl*2048 + (i/8)*1024 + (i%8)*128 + ((kk/16) ^ (i%8))*16 + kk%16
-    for (int c = tq; c < chunks; c += kQuantThreads) {
-      if (chunks > kQuantThreads) load_chunk(c);  // wide slices reload (L1/L2 hits)
-      const uint32_t bits = sh.flags[c];
-      const int kbl = c / 16, kk = (c % 16) * 8;
+          for (int i = 0; i < kSmallMP; ++i)
+            if (i < a.M) {
+              const float xv = __half2float(xc[static_cast<size_t>(i) * xs_ld]);
+              P0[i] += w0 * xv;
+              P1[i] += w1 * xv;
+            }
+        }
+      }
 #pragma unroll
       for (int i = 0; i < kSmallMP; ++i) {
+        sh.psum[tq][i] = P0[i];
+        sh.psum[tq + 64][i] = P1[i];
+      }
+      cluster_wait();
+    } else {
+      // ---- warps 4..7: the row scales, then quantize the slice into the B operand
+      const int tz = threadIdx.x - 128;  // 0..127
+      cluster_wait();
+      if (tz < kSmallMP) {
+        const uint32_t local = smem_addr(&sh.rowmax_local[tz]);
+        float peer[kSmallMaxSplits];
+#pragma unroll
+        for (int r = 0; r < kSmallMaxSplits; ++r)  // all remote loads in flight at once
+          peer[r] = r < S ? ld_cluster_f32(map_rank(local, r)) : 0.0f;
+        float m = 0.0f;
+#pragma unroll
+        for (int r = 0; r < kSmallMaxSplits; ++r) m = fmaxf(m, peer[r]);
+        const float sc = __fdiv_rn(m, 127.0f);
+        sh.sx[tz] = (tz < a.M) ? sc : 0.0f;
+        sh.rcp[tz] = (tz < a.M && m > 0.0f) ? __frcp_rn(sc) : 0.0f;
+        sh.zero_row[tz] = (tz >= a.M) || m == 0.0f;
+      }
+      named_barrier(2, kQuantThreads);
+      // unit (row i, chunk c): 8 codes for row i, k-block kbl, byte kk at
+      //   kbl*2048 + (i/8)*1024 + (i%8)*128 + ((kk/16) ^ (i%8))*16 + kk%16
+      for (int u = tz; u < kSmallMP * chunks; u += kQuantThreads) {
+        const int i = u / chunks, c = u % chunks;
         uint2 q = make_uint2(0u, 0u);
         if (!sh.zero_row[i]) {
-          const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-          const float s = sh.sx[i], r = sh.rcp[i];
+          const uint4 v = *reinterpret_cast<const uint4*>(x_slice + static_cast<size_t>(i) * xs_ld + c * 8);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          const uint32_t bits = sh.flags[c];
+          const float sc = sh.sx[i], r = sh.rcp[i];
           uint32_t p[2] = {0u, 0u};
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            if ((bits >> e) & 1u) continue;
-            const int qv = quantize_exact(half_bits_to_float(w[e / 2], e & 1), s, r);
-            p[e / 4] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
+            const int qv = quantize_exact(half_bits_to_float(w[e / 2], e & 1), sc, r);
+            const uint32_t code = ((bits >> e) & 1u) ? 0u : (static_cast<uint32_t>(qv) & 0xFFu);
+            p[e / 4] |= code << (8 * (e & 3));
           }
           q = make_uint2(p[0], p[1]);
         }
+        const int kbl = c / 16, kk = (c % 16) * 8;
         uint8_t* dst = xq_tiles + kbl * kBBytesPerKb + (i / 8) * 1024 + (i % 8) * 128 +
                        (((kk / 16) ^ (i % 8)) * 16) + (kk % 16);
         *reinterpret_cast<uint2*>(dst) = q;
       }
-    }
-    fence_async_shared();
-    mbar_arrive(&sh.xq_ready);
+      fence_async_shared();
+      mbar_arrive(&sh.xq_ready);
 
-    if (warp >= 4) {
-      // ---- warps 4..7: TMEM lane quadrant q <-> channels 32q .. 32q+31
+      // ---- drain the accumulator: TMEM lane quadrant q <-> channels 32q .. 32q+31
       const int quad = warp & 3;
-      const int n = quad * 32 + lane, gn = n0 + n;
-      // fp16 outlier term of the outlier columns in this slice, while the MMAs run
-      float P[kSmallMP];
-#pragma unroll
-      for (int i = 0; i < kSmallMP; ++i) P[i] = 0.0f;
-      if (gn < a.N) {
-        const float sw_n = a.w_scale[gn];
-        const int8_t* wrow = a.Wq + static_cast<size_t>(gn) * a.K;
-        for (int c = 0; c < chunks; ++c) {
-          uint32_t bits = sh.flags[c];
-          while (bits) {
-            const int j = col_begin + c * 8 + __ffs(bits) - 1;
-            bits &= bits - 1u;
-            const float wv = __half2float(__float2half_rn(static_cast<float>(wrow[j]) * sw_n));
-#pragma unroll
-            for (int i = 0; i < kSmallMP; ++i)
-              if (i < a.M) P[i] += wv * __half2float(a.X[static_cast<size_t>(i) * a.K + j]);
-          }
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < kSmallMP; ++i) sh.psum[n][i] = P[i];
+      const int n = quad * 32 + lane;
       mbar_wait_bounded(&sh.tmem_full, 0, abort);
-      // one decision for the 128 epilogue threads
-      named_barrier(2, 128);
+      // one decision for the 128 threads
+      named_barrier(2, kQuantThreads);
       if (threadIdx.x == 128) sh.epi_ok = (*abort == 0);
-      named_barrier(2, 128);
+      named_barrier(2, kQuantThreads);
       tc_fence_after();
       uint32_t r[16];
       __syncwarp();
@@ -396,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int outs = kSmallBN * a.M;
     const int per = (outs + S - 1) / S;
     const int o_begin = split * per, o_end = min(outs, o_begin + per);
-    for (int o = o_begin + tq; o < o_end; o += kQuantThreads) {
+    for (int o = o_begin + tq; o < o_end; o += kStatThreads) {
       const int n = o / a.M, i = o % a.M, gn = n0 + n;
       if (gn >= a.N) continue;
       const uint32_t acc_l = smem_addr(&sh.acc[n][i]);
@@ -446,7 +463,7 @@ cudaError_t configure_small() {
   if (e != cudaSuccess) return e;
   if (dev == configured_device) return cudaSuccess;
   e = cudaFuncSetAttribute(small_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(small_smem_bytes(kSmallMaxKbPerSplit)));
+                           static_cast<int>(small_smem_bytes(kSmallMaxKbPerSplit, kSmallMP)));
   if (e == cudaSuccess) configured_device = dev;
   return e;
 }
@@ -484,7 +501,7 @@ int max_active_clusters(int S, size_t smem) {
 
 // Cluster size S (CTAs splitting K per 128-channel tile): the one that minimises
 // (waves of resident clusters) x (k-blocks per CTA), preferring larger S on ties.
-SmallPlan plan_small(int N, int K) {
+SmallPlan plan_small(int M, int N, int K) {
   SmallPlan p;
   p.tiles = (N + kSmallBN - 1) / kSmallBN;
   const int kb_total = (K + kBKBytes - 1) / kBKBytes;
@@ -495,7 +512,7 @@ SmallPlan plan_small(int N, int K) {
     if (S > kb_total) continue;
     const int kbps = kb_per_split(kb_total, S);
     if (kbps > kSmallMaxKbPerSplit) continue;
-    const int act = max_active_clusters(S, small_smem_bytes(kbps));
+    const int act = max_active_clusters(S, small_smem_bytes(kbps, M));
     const long long cost = static_cast<long long>((p.tiles + act - 1) / act) * kbps;
     if (p.splits == 0 || cost < best) {
       best = cost;
@@ -521,7 +538,7 @@ cudaError_t launch_small(const CUtensorMap& map_wq, const SmallArgs& a, const Sm
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.tiles * p.splits);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = small_smem_bytes(p.kb_per_split);
+  cfg.dynamicSmemBytes = small_smem_bytes(p.kb_per_split, a.M);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
