@@ -126,6 +126,7 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
   a.Y = static_cast<__half*>(Y);
   a.acc = acc;
   a.splits = sp.splits;
+  a.stages = sp.stages;
   a.status = p.header;
   return a;
 }

@@ -95,10 +95,11 @@ struct SmallArgs {
   __half* Y;
   int32_t* acc;          // nullable: also write the int32 accumulators
   int splits;            // CTAs per cluster, each owning a K-slice
+  int stages;            // depth of the Wq ring
   int32_t* status;
 };
 struct SmallPlan {
-  int tiles, splits, kb_per_split;
+  int tiles, splits, kb_per_split, stages;
 };
 SmallPlan plan_small(int M, int N, int K);
 bool small_path_fits(int M, int K);

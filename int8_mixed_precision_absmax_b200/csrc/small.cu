@@ -5,7 +5,8 @@
 // once at HBM speed and everything else hidden behind that stream.  Each output tile of
 // 128 channels is computed by a thread-block cluster of S CTAs that split K (split-K).
 // Each CTA of a cluster:
-//   1. starts the TMA stream of its Wq slice [128 channels x K/S] into a 6-stage ring;
+//   1. starts the TMA stream of its Wq slice [128 channels x K/S] into a ring of up to 8
+//      stages (all of it, when the slice is that short);
 //   2. reads its K-slice of X for all M rows and finds, per column, whether any |x|
 //      exceeds the threshold (the outlier columns of [P2] "8位量化实战：离群值处理与显存
 //      优化避坑指南" section 2.3 -- complete per slice, since every row is present) and,
@@ -38,7 +39,7 @@ namespace i8mm {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kStages = 6;
+constexpr int kMaxStages = 8;
 constexpr int kABytes = kSmallBN * kBKBytes;       // 16 KB of Wq per stage
 constexpr int kBBytesPerKb = kSmallMP * kBKBytes;  // 2 KB of Xq per k-block
 constexpr uint32_t kTmemCols = 32;
@@ -101,20 +102,11 @@ __device__ __forceinline__ float half_bits_to_float(uint32_t word, int hi) {
       __ushort_as_half(static_cast<unsigned short>(hi ? (word >> 16) : (word & 0xFFFFu))));
 }
 
-// rne(fl(x / s)) clamped to [-127, 127]; rcp = 1/s rounded to nearest (see file comment)
-__device__ __forceinline__ int quantize_exact(float x, float s, float rcp) {
-  const float v = x * rcp;
-  const float d = fabsf(v - rintf(v));  // distance to the nearest integer, exact
-  int q = __float2int_rn(v);
-  if (fabsf(d - 0.5f) <= 0x1p-15f) q = __float2int_rn(__fdiv_rn(x, s));  // near a tie
-  return max(-127, min(127, q));
-}
-
 }  // namespace
 
 struct SmallShared {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t xq_ready;
   uint64_t tmem_full;
   uint64_t drain;
@@ -129,13 +121,24 @@ struct SmallShared {
   uint8_t flags[kSmallMaxKbPerSplit * 16];  // outlier bits, 8 columns per byte
   int32_t acc[kSmallBN][kSmallMP];          // this CTA's partial sums, read cluster-wide
   float psum[kSmallBN][kSmallMP];           // this CTA's outlier term, read cluster-wide
+  float wscale[kSmallBN];                   // the tile's w_scale and bias
+  float bias[kSmallBN];
 };
 
+constexpr size_t kSmemLimit = 227 * 1024;
+
 // [Wq ring | Xq tiles | X slice (M rows) | SmallShared]
-size_t small_smem_bytes(int kb_per_split, int M) {
-  return 1024 + static_cast<size_t>(kStages) * kABytes +
+size_t small_smem_bytes(int stages, int kb_per_split, int M) {
+  return 1024 + static_cast<size_t>(stages) * kABytes +
          static_cast<size_t>(kb_per_split) * kBBytesPerKb +
          static_cast<size_t>(M) * kb_per_split * kBKBytes * sizeof(__half) + sizeof(SmallShared) + 16;
+}
+
+// The deepest ring (all of the slice when it fits) within the shared-memory limit.
+int small_stages(int kb_per_split, int M) {
+  int st = kb_per_split < kMaxStages ? kb_per_split : kMaxStages;
+  while (st > 2 && small_smem_bytes(st, kb_per_split, M) > kSmemLimit) --st;
+  return st;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -143,17 +146,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t small_smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(small_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int S = a.splits;
+  const int kb_total = (a.K + kBKBytes - 1) / kBKBytes;
+  const int kb_max = (kb_total + S - 1) / S;  // the same in every CTA: a common smem layout
+  const int kStages = a.stages;
   uint8_t* a_stage = base;                       // kStages x 16 KB
   uint8_t* xq_tiles = base + kStages * kABytes;  // kb_max x 2 KB
-  const int S = a.splits;
   const int split = static_cast<int>(cluster_rank());
   const int tile = blockIdx.x / S;
   const int n0 = tile * kSmallBN;
-  const int kb_total = (a.K + kBKBytes - 1) / kBKBytes;
   const int kb_begin = static_cast<int>(static_cast<long long>(split) * kb_total / S);
   const int kb_end = static_cast<int>(static_cast<long long>(split + 1) * kb_total / S);
   const int nkb = kb_end - kb_begin;
-  const int kb_max = (kb_total + S - 1) / S;  // the same in every CTA: a common smem layout
   __half* x_slice = reinterpret_cast<__half*>(xq_tiles + kb_max * kBBytesPerKb);  // [M][kb_max*128]
   const int xs_ld = kb_max * kBKBytes;
   SmallShared& sh = *reinterpret_cast<SmallShared*>(x_slice + static_cast<size_t>(a.M) * xs_ld);
@@ -299,7 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < kSmallMP; ++i) sh.red[warp - 2][i] = rmax[i];
     }
-    named_barrier(1, kStatThreads);  // flags, x_slice and red are complete
+    if (tq < kSmallBN) {
+      const int gn = n0 + tq;
+      sh.wscale[tq] = gn < a.N ? a.w_scale[gn] : 0.0f;
+      sh.bias[tq] = (a.bias && gn < a.N) ? __half2float(a.bias[gn]) : 0.0f;
+    }
+    named_barrier(1, kStatThreads);  // flags, x_slice, red, wscale and bias are complete
     if (tq < kSmallMP) {
       float m = 0.0f;
 #pragma unroll
@@ -316,8 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < kSmallMP; ++i) P0[i] = P1[i] = 0.0f;
       const int g0 = n0 + tq, g1 = n0 + tq + 64;
-      const float s0 = g0 < a.N ? a.w_scale[g0] : 0.0f;
-      const float s1 = g1 < a.N ? a.w_scale[g1] : 0.0f;
+      const float s0 = sh.wscale[tq], s1 = sh.wscale[tq + 64];
       const int8_t* w0row = a.Wq + static_cast<size_t>(g0 < a.N ? g0 : 0) * a.K;
       const int8_t* w1row = a.Wq + static_cast<size_t>(g1 < a.N ? g1 : 0) * a.K;
       for (int c = 0; c < chunks; ++c) {
@@ -372,11 +380,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
           const uint32_t bits = sh.flags[c];
           const float sc = sh.sx[i], r = sh.rcp[i];
+          float x[8];
+          int qv[8];
+          uint32_t near_tie = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {  // 8 independent elements: no branch inside
+            x[e] = half_bits_to_float(w[e / 2], e & 1);
+            const float t = x[e] * r;
+            qv[e] = __float2int_rn(t);
+            const float d = fabsf(t - rintf(t));
+            near_tie |= (fabsf(d - 0.5f) <= 0x1p-15f ? 1u : 0u) << e;
+          }
+          if (near_tie) {  // rare: round the IEEE quotient itself
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if ((near_tie >> e) & 1u) qv[e] = __float2int_rn(__fdiv_rn(x[e], sc));
+          }
           uint32_t p[2] = {0u, 0u};
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int qv = quantize_exact(half_bits_to_float(w[e / 2], e & 1), sc, r);
-            const uint32_t code = ((bits >> e) & 1u) ? 0u : (static_cast<uint32_t>(qv) & 0xFFu);
+            const int qc = max(-127, min(127, qv[e]));
+            const uint32_t code = ((bits >> e) & 1u) ? 0u : (static_cast<uint32_t>(qc) & 0xFFu);
             p[e / 4] |= code << (8 * (e & 3));
           }
           q = make_uint2(p[0], p[1]);
@@ -432,8 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc += pa[r];
         P += pp[r];
       }
-      const float b = a.bias ? __half2float(a.bias[gn]) : 0.0f;
-      const float y = static_cast<float>(acc) * sh.sx[i] * a.w_scale[gn] + P + b;
+      const float y = static_cast<float>(acc) * sh.sx[i] * sh.wscale[n] + P + sh.bias[n];
       a.Y[static_cast<size_t>(i) * a.N + gn] = __float2half_rn(y);
       if (a.acc) a.acc[static_cast<size_t>(i) * a.N + gn] = acc;
     }
@@ -463,7 +486,7 @@ cudaError_t configure_small() {
   if (e != cudaSuccess) return e;
   if (dev == configured_device) return cudaSuccess;
   e = cudaFuncSetAttribute(small_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(small_smem_bytes(kSmallMaxKbPerSplit, kSmallMP)));
+                           static_cast<int>(kSmemLimit));
   if (e == cudaSuccess) configured_device = dev;
   return e;
 }
@@ -512,7 +535,7 @@ SmallPlan plan_small(int M, int N, int K) {
     if (S > kb_total) continue;
     const int kbps = kb_per_split(kb_total, S);
     if (kbps > kSmallMaxKbPerSplit) continue;
-    const int act = max_active_clusters(S, small_smem_bytes(kbps, M));
+    const int act = max_active_clusters(S, small_smem_bytes(small_stages(kbps, M), kbps, M));
     const long long cost = static_cast<long long>((p.tiles + act - 1) / act) * kbps;
     if (p.splits == 0 || cost < best) {
       best = cost;
@@ -521,6 +544,7 @@ SmallPlan plan_small(int M, int N, int K) {
   }
   if (p.splits == 0) p.splits = 1;
   p.kb_per_split = kb_per_split(kb_total, p.splits);
+  p.stages = small_stages(p.kb_per_split, M);
   return p;
 }
 
@@ -528,7 +552,9 @@ bool small_path_fits(int M, int K) {
   if (M > kSmallMP) return false;
   const int kb_total = (K + kBKBytes - 1) / kBKBytes;
   const int S = kb_total < kSmallMaxSplits ? kb_total : kSmallMaxSplits;
-  return kb_per_split(kb_total, S) <= kSmallMaxKbPerSplit;
+  const int kbps = kb_per_split(kb_total, S);
+  return kbps <= kSmallMaxKbPerSplit &&
+         small_smem_bytes(small_stages(kbps, M), kbps, M) <= kSmemLimit;
 }
 
 cudaError_t launch_small(const CUtensorMap& map_wq, const SmallArgs& a, const SmallPlan& p,
@@ -538,7 +564,7 @@ cudaError_t launch_small(const CUtensorMap& map_wq, const SmallArgs& a, const Sm
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.tiles * p.splits);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = small_smem_bytes(p.kb_per_split, a.M);
+  cfg.dynamicSmemBytes = small_smem_bytes(p.stages, p.kb_per_split, a.M);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
