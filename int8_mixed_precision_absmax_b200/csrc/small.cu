@@ -42,11 +42,11 @@ constexpr int kThreads = 256;
 constexpr int kMaxStages = 8;
 constexpr int kABytes = kSmallBN * kBKBytes;       // 16 KB of Wq per stage
 constexpr int kBBytesPerKb = kSmallMP * kBKBytes;  // 2 KB of Xq per k-block
-constexpr uint32_t kTmemCols = 32;
+constexpr int kAccs = 4;               // independent accumulators, summed in the drain
+constexpr uint32_t kTmemCols = 64;      // kAccs x 16 columns
 constexpr uint32_t kIdesc = idesc_i8_s32(kSmallBN, kSmallMP);
 constexpr int kStatThreads = 192;   // warps 2..7: statistics of the slice
 constexpr int kQuantThreads = 128;  // warps 4..7: quantization and the accumulator drain
-constexpr int kOutlierThreads = 64; // warps 2..3: the fp16 outlier term
 
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -113,6 +113,7 @@ struct SmallShared {
   uint32_t tmem_base;
   int abort;
   int epi_ok;
+  int issued;
   float rowmax_local[kSmallMP];  // read by the other CTAs of the cluster
   float red[kStatThreads / 32][kSmallMP];
   float sx[kSmallMP];
@@ -173,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sh.tmem_full, 1);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
+    sh.issued = 0;
     fence_mbarrier_init();
   }
   if (threadIdx.x == 32) prefetch_tmap(&map_wq);
@@ -206,9 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(&map_wq, a_stage + s * kABytes, &sh.full[s], (kb_begin + j) * kBKBytes, n0);
         ++issued;
       }
-      int dummy = 0;  // every issued copy lands before the block may exit
-      for (int d = issued > kStages ? issued - kStages : 0; d < issued; ++d)
-        mbar_wait_bounded(&sh.full[d % kStages], static_cast<uint32_t>(d / kStages) & 1u, &dummy);
+      sh.issued = issued;  // the teardown drains these if any role gave up
       if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
     }
     cluster_wait();
@@ -231,9 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a0 = smem_addr(a_stage + s * kABytes);
           const uint32_t b0 = smem_addr(xq_tiles + j * kBBytesPerKb);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_i8(tmem, sw128_kmajor_desc(a0 + 32u * k), sw128_kmajor_desc(b0 + 32u * k),
-                   kIdesc, (j > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k)  // accumulator k: four independent chains
+            mma_i8(tmem + static_cast<uint32_t>(k * kSmallMP), sw128_kmajor_desc(a0 + 32u * k),
+                   sw128_kmajor_desc(b0 + 32u * k), kIdesc, j > 0 ? 1u : 0u);
           mma_commit(&sh.empty[s]);
         }
         if (ok) mma_commit(&sh.tmem_full);
@@ -328,13 +328,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float s0 = sh.wscale[tq], s1 = sh.wscale[tq + 64];
       const int8_t* w0row = a.Wq + static_cast<size_t>(g0 < a.N ? g0 : 0) * a.K;
       const int8_t* w1row = a.Wq + static_cast<size_t>(g1 < a.N ? g1 : 0) * a.K;
+      // With the whole slice resident in the ring (no stage is reused), the weights of an
+      // outlier column are read from the landed TMA tile instead of from HBM.
+      const bool resident = nkb <= kStages;
       for (int c = 0; c < chunks; ++c) {
         uint32_t bits = sh.flags[c];
         while (bits) {
-          const int j = col_begin + c * 8 + __ffs(bits) - 1;
+          const int jl = c * 8 + __ffs(bits) - 1;  // column within the slice
+          const int j = col_begin + jl;
           bits &= bits - 1u;
-          const float w0 = __half2float(__float2half_rn(static_cast<float>(w0row[j]) * s0));
-          const float w1 = __half2float(__float2half_rn(static_cast<float>(w1row[j]) * s1));
+          int8_t q0, q1;
+          if (resident) {
+            const int kbl = jl / kBKBytes, kk = jl % kBKBytes;
+            mbar_wait_bounded(&sh.full[kbl], 0, abort);
+            const uint8_t* tile = a_stage + kbl * kABytes;
+            q0 = static_cast<int8_t>(tile[(tq / 8) * 1024 + (tq % 8) * 128 +
+                                          (((kk / 16) ^ (tq % 8)) * 16) + kk % 16]);
+            const int t1 = tq + 64;
+            q1 = static_cast<int8_t>(tile[(t1 / 8) * 1024 + (t1 % 8) * 128 +
+                                          (((kk / 16) ^ (t1 % 8)) * 16) + kk % 16]);
+          } else {
+            q0 = w0row[j];
+            q1 = w1row[j];
+          }
+          const float w0 = __half2float(__float2half_rn(static_cast<float>(q0) * s0));
+          const float w1 = __half2float(__float2half_rn(static_cast<float>(q1) * s1));
           const __half* xc = x_slice + (j - col_begin);
 #pragma unroll
           for (int i = 0; i < kSmallMP; ++i)
@@ -370,45 +388,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         sh.zero_row[tz] = (tz >= a.M) || m == 0.0f;
       }
       named_barrier(2, kQuantThreads);
-      // unit (row i, chunk c): 8 codes for row i, k-block kbl, byte kk at
+      // thread tz quantizes chunk c (8 columns) for all 16 rows, independently per row;
+      // codes for row i, k-block kbl, byte kk go to
       //   kbl*2048 + (i/8)*1024 + (i%8)*128 + ((kk/16) ^ (i%8))*16 + kk%16
-      for (int u = tz; u < kSmallMP * chunks; u += kQuantThreads) {
-        const int i = u / chunks, c = u % chunks;
-        uint2 q = make_uint2(0u, 0u);
-        if (!sh.zero_row[i]) {
-          const uint4 v = *reinterpret_cast<const uint4*>(x_slice + static_cast<size_t>(i) * xs_ld + c * 8);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          const uint32_t bits = sh.flags[c];
-          const float sc = sh.sx[i], r = sh.rcp[i];
-          float x[8];
-          int qv[8];
-          uint32_t near_tie = 0;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {  // 8 independent elements: no branch inside
-            x[e] = half_bits_to_float(w[e / 2], e & 1);
-            const float t = x[e] * r;
-            qv[e] = __float2int_rn(t);
-            const float d = fabsf(t - rintf(t));
-            near_tie |= (fabsf(d - 0.5f) <= 0x1p-15f ? 1u : 0u) << e;
-          }
-          if (near_tie) {  // rare: round the IEEE quotient itself
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              if ((near_tie >> e) & 1u) qv[e] = __float2int_rn(__fdiv_rn(x[e], sc));
-          }
-          uint32_t p[2] = {0u, 0u};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int qc = max(-127, min(127, qv[e]));
-            const uint32_t code = ((bits >> e) & 1u) ? 0u : (static_cast<uint32_t>(qc) & 0xFFu);
-            p[e / 4] |= code << (8 * (e & 3));
-          }
-          q = make_uint2(p[0], p[1]);
-        }
+      for (int c = tz; c < chunks; c += kQuantThreads) {
+        const uint32_t bits = sh.flags[c];
         const int kbl = c / 16, kk = (c % 16) * 8;
-        uint8_t* dst = xq_tiles + kbl * kBBytesPerKb + (i / 8) * 1024 + (i % 8) * 128 +
-                       (((kk / 16) ^ (i % 8)) * 16) + (kk % 16);
-        *reinterpret_cast<uint2*>(dst) = q;
+        uint8_t* tile = xq_tiles + kbl * kBBytesPerKb + (kk % 16);
+#pragma unroll
+        for (int i = 0; i < kSmallMP; ++i) {
+          uint2 q = make_uint2(0u, 0u);
+          if (!sh.zero_row[i]) {
+            const uint4 v =
+                *reinterpret_cast<const uint4*>(x_slice + static_cast<size_t>(i) * xs_ld + c * 8);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            const float sc = sh.sx[i], r = sh.rcp[i];
+            float x[8];
+            int qv[8];
+            uint32_t near_tie = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {  // 8 independent elements: no branch inside
+              x[e] = half_bits_to_float(w[e / 2], e & 1);
+              const float t = x[e] * r;
+              qv[e] = __float2int_rn(t);
+              const float d = fabsf(t - rintf(t));
+              near_tie |= (fabsf(d - 0.5f) <= 0x1p-15f ? 1u : 0u) << e;
+            }
+            if (near_tie) {  // rare: round the IEEE quotient itself
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                if ((near_tie >> e) & 1u) qv[e] = __float2int_rn(__fdiv_rn(x[e], sc));
+            }
+            uint32_t p[2] = {0u, 0u};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int qc = max(-127, min(127, qv[e]));
+              const uint32_t code = ((bits >> e) & 1u) ? 0u : (static_cast<uint32_t>(qc) & 0xFFu);
+              p[e / 4] |= code << (8 * (e & 3));
+            }
+            q = make_uint2(p[0], p[1]);
+          }
+          *reinterpret_cast<uint2*>(tile + (i / 8) * 1024 + (i % 8) * 128 +
+                                    (((kk / 16) ^ (i % 8)) * 16)) = q;
+        }
       }
       fence_async_shared();
       mbar_arrive(&sh.xq_ready);
@@ -422,13 +444,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (threadIdx.x == 128) sh.epi_ok = (*abort == 0);
       named_barrier(2, kQuantThreads);
       tc_fence_after();
-      uint32_t r[16];
+      int32_t accs[kSmallMP];
+#pragma unroll
+      for (int i = 0; i < kSmallMP; ++i) accs[i] = 0;
       __syncwarp();
-      tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16), r);
-      tmem_ld_wait();
+#pragma unroll
+      for (int k = 0; k < kAccs; ++k) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(k * kSmallMP), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < kSmallMP; ++i) accs[i] += static_cast<int32_t>(r[i]);
+      }
       const bool ok = sh.epi_ok != 0;
 #pragma unroll
-      for (int i = 0; i < kSmallMP; ++i) sh.acc[n][i] = ok ? static_cast<int32_t>(r[i]) : 0;
+      for (int i = 0; i < kSmallMP; ++i) sh.acc[n][i] = ok ? accs[i] : 0;
       if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
     }
     cluster_arrive();  // phase 2: every CTA's partial sums are in its shared memory
@@ -467,6 +498,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_wait();
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0 && sh.abort) {
+    // A wait gave up: the MMA thread may not have seen every stage land, so let the copies
+    // still in flight finish before the shared memory is released.
+    int dummy = 0;
+    for (int d = sh.issued > kStages ? sh.issued - kStages : 0; d < sh.issued; ++d)
+      mbar_wait_bounded(&sh.full[d % kStages], static_cast<uint32_t>(d / kStages) & 1u, &dummy);
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
