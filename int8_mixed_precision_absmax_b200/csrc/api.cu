@@ -36,6 +36,25 @@ int check_device() {
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? INT8MM_OK : INT8MM_ERR_CUDA; }
 
+}  // namespace
+
+int i8mm::device_sm_count() {
+  static int cached_device = -1, cached_sms = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev != cached_device) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
+      sms = 148;
+    cached_sms = sms;
+    cached_device = dev;
+  }
+  return cached_sms;
+}
+
+namespace {
+
 float effective_threshold(float t) { return t < 0.0f ? 0.0f : t; }
 
 template <typename T>
@@ -134,7 +153,8 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
 int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale, int N,
                  float threshold, void* workspace, const ForwardPlan& p, cudaStream_t stream,
                  bool pdl_first) {
-  if (small_path_fits(M, K)) return INT8MM_OK;  // one kernel does everything: see run_matmul
+  if (M <= kSmallMP && (plan_gemv(M, N, K, device_sm_count()).fits || small_path_fits(M, K)))
+    return INT8MM_OK;  // one kernel does everything: see run_matmul
   int rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
                                         effective_threshold(threshold), p.mask, stream,
                                         pdl_first));
@@ -161,6 +181,31 @@ int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_s
 int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                const void* bias, int N, float threshold, void* Y, int32_t* acc,
                void* workspace, const ForwardPlan& p, cudaStream_t stream, bool pdl) {
+  if (M <= kSmallMP) {
+    const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
+    if (gp.fits) {
+      GemvArgs g;
+      g.X = static_cast<const __half*>(X);
+      g.M = M;
+      g.K = K;
+      g.N = N;
+      g.threshold = effective_threshold(threshold);
+      g.Wq = Wq;
+      g.w_scale = w_scale;
+      g.bias = static_cast<const __half*>(bias);
+      g.Y = static_cast<__half*>(Y);
+      g.acc = acc;
+      g.channels = gp.channels;
+      g.stages = gp.stages;
+      g.kpad = gp.kpad;
+      g.status = p.header;
+      CUtensorMap map;
+      if (!encode_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, 256,
+                          static_cast<uint32_t>(gp.channels), CU_TENSOR_MAP_SWIZZLE_NONE))
+        return INT8MM_ERR_CUDA;
+      return launch_status(launch_gemv(map, g, gp, stream, pdl));
+    }
+  }
   if (small_path_fits(M, K)) {
     const SmallPlan sp = plan_small(M, N, K);
     const SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p, sp);

@@ -106,6 +106,29 @@ bool small_path_fits(int M, int K);
 cudaError_t launch_small(const CUtensorMap& map_wq, const SmallArgs& a, const SmallPlan& p,
                          cudaStream_t stream, bool pdl);
 
+struct GemvArgs {
+  const __half* X;
+  int M, K, N;
+  float threshold;       // already clamped to >= 0
+  const int8_t* Wq;
+  const float* w_scale;
+  const __half* bias;
+  __half* Y;
+  int32_t* acc;          // nullable: also write the int32 accumulators
+  int channels;          // output channels per CTA
+  int stages;            // depth of the Wq ring (256-byte slabs of K)
+  int kpad;              // K rounded up to 256
+  int32_t* status;
+};
+struct GemvPlan {
+  int mt, channels, ctas, kpad, stages;
+  bool fits;
+};
+GemvPlan plan_gemv(int M, int N, int K, int num_sms);
+cudaError_t launch_gemv(const CUtensorMap& map_wq, const GemvArgs& a, const GemvPlan& p,
+                        cudaStream_t stream, bool pdl);
+int device_sm_count();
+
 struct GemmArgs {
   int M, N, K;
   const float* xscale;   // [M]
@@ -122,7 +145,8 @@ struct GemmMaps {
 // Host-side tensor-map encoding (driver entry point fetched through the runtime).
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                     uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
-                    uint32_t box_inner, uint32_t box_outer);
+                    uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream, bool pdl);
 
 // GEMM tile shape (shared with the host for map boxes)

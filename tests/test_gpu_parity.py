@@ -231,7 +231,10 @@ def check_forward_acc(X, W, b, t, rows=None):
     (16, 2048, 640, 5, 6.0),    # the largest few-token batch
     (16, 256, 128, 0, math.inf),
     (7, 512, 384, 0, 0.0),      # every column an outlier: int8 product is zero
-    (5, 20000, 200, 4, 6.0),    # long rows: many splits
+    (5, 20000, 200, 4, 6.0),    # long rows: a weight ring that is refilled
+    (16, 16384, 300, 4, 6.0),   # activations too long for shared memory: cluster path
+    (12, 14336, 256, 3, 6.0),   # cluster path, ragged rows
+    (9, 4096, 4100, 5, 6.0),    # channels not a multiple of the per-CTA share
     (17, 512, 300, 3, 6.0),     # one row past the few-token path
     (200, 1040, 600, 5, 6.0),   # the tiled path
 ])
