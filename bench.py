@@ -424,8 +424,8 @@ def run_ours(args):
     n_out = int(i8.int8_quantize_rows(Xs[0], w.threshold)[3].item())
     pad = (n_out + 63) // 64 * 64 if n_out else 0
     few_tokens = w.M <= 16
-    kernel = ("small_fused_kernel (one launch: X statistics and quantization in smem, "
-              "tcgen05 int8 swap-AB, split-K reduced through cluster shared memory)"
+    kernel = ("gemv_kernel (one launch per step: weight slice streamed by TMA into shared "
+              "memory while X is quantized, exact dp4a int8 products, fused epilogue)"
               if few_tokens else "gemm_kernel (int8 + fp16 tcgen05, fused epilogue)")
     if few_tokens:  # reads X (fp16) and Wq, writes Y
         gemm_bytes = (2 * w.M * w.K + w.N * w.K + 4 * w.N + 2 * w.M * w.N

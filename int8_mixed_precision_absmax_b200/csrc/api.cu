@@ -130,6 +130,33 @@ int plan_forward(int M, int N, int K, const int8_t* Wq, const float* w_scale, vo
   return INT8MM_OK;
 }
 
+GemvArgs gemv_args(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+                   const void* bias, int N, float threshold, void* Y, int32_t* acc,
+                   void* workspace, const ForwardPlan& p, const GemvPlan& gp) {
+  GemvArgs g;
+  g.X = static_cast<const __half*>(X);
+  g.M = M;
+  g.K = K;
+  g.N = N;
+  g.threshold = effective_threshold(threshold);
+  g.Wq = Wq;
+  g.w_scale = w_scale;
+  g.bias = static_cast<const __half*>(bias);
+  g.Y = static_cast<__half*>(Y);
+  g.acc = acc;
+  g.channels = gp.channels;
+  g.stages = gp.stages;
+  g.kpad = gp.kpad;
+  g.quant_ctas = gp.quant_ctas;
+  g.xq = at<int8_t>(workspace, p.L.few_xq);
+  g.xo = at<__half>(workspace, p.L.few_xo);
+  g.sx = at<float>(workspace, p.L.few_sx);
+  g.cols = at<int32_t>(workspace, p.L.cols);
+  g.n_out = p.header + 1;
+  g.status = p.header;
+  return g;
+}
+
 SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                      const void* bias, int N, float threshold, void* Y, int32_t* acc,
                      const ForwardPlan& p, const SmallPlan& sp) {
@@ -153,8 +180,15 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
 int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale, int N,
                  float threshold, void* workspace, const ForwardPlan& p, cudaStream_t stream,
                  bool pdl_first) {
-  if (M <= kSmallMP && (plan_gemv(M, N, K, device_sm_count()).fits || small_path_fits(M, K)))
-    return INT8MM_OK;  // one kernel does everything: see run_matmul
+  if (M <= kSmallMP) {
+    const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
+    if (gp.fits) {
+      const GemvArgs g = gemv_args(X, M, K, Wq, w_scale, nullptr, N, threshold, nullptr, nullptr,
+                                   workspace, p, gp);
+      return launch_status(launch_few_quant(g, gp, stream, pdl_first));
+    }
+    if (small_path_fits(M, K)) return INT8MM_OK;  // one kernel does everything: see run_matmul
+  }
   int rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
                                         effective_threshold(threshold), p.mask, stream,
                                         pdl_first));
@@ -184,21 +218,8 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   if (M <= kSmallMP) {
     const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
     if (gp.fits) {
-      GemvArgs g;
-      g.X = static_cast<const __half*>(X);
-      g.M = M;
-      g.K = K;
-      g.N = N;
-      g.threshold = effective_threshold(threshold);
-      g.Wq = Wq;
-      g.w_scale = w_scale;
-      g.bias = static_cast<const __half*>(bias);
-      g.Y = static_cast<__half*>(Y);
-      g.acc = acc;
-      g.channels = gp.channels;
-      g.stages = gp.stages;
-      g.kpad = gp.kpad;
-      g.status = p.header;
+      const GemvArgs g = gemv_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace,
+                                   p, gp);
       CUtensorMap map;
       if (!encode_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, 256,
                           static_cast<uint32_t>(gp.channels), CU_TENSOR_MAP_SWIZZLE_NONE))

@@ -3,22 +3,26 @@
 // With M <= 16 the layer reads every byte of Wq once and does M multiply-adds per byte:
 // it is bound by HBM, not by the tensor cores (a tcgen05 MMA with M = 128 channels costs
 // the same time at N = 16 tokens as at N = 256, so it would run at 1/16 of its rate).
-// This kernel therefore streams Wq at full bandwidth and multiplies on the CUDA cores:
+// Two launches:
 //
-//   * one CTA per SM owns C <= 32 output channels over all of K (no split-K, no reduction
-//     across CTAs); its first instruction starts the TMA stream of its Wq rows into a
-//     shared-memory ring (all of it when it fits);
-//   * meanwhile its 512 threads read X (M x K, from L2 after the first CTA) and find the
-//     outlier columns, max_i |x| > threshold ([P2] "8位量化实战：离群值处理与显存优化避坑
-//     指南" section 2.3), the row scales sx = max over the regular columns / 127 and the
-//     int8 codes q = rne(x / sx) clamped to [-127, 127], 0 in outlier columns ([P5]
-//     "PyTorch 2.9 支持 LLM.int8()" item 2); every CTA does this redundantly, which costs
-//     less than any exchange between CTAs;
-//   * acc[i,n] = sum_k q[i,k] * Wq[n,k] exactly in int32 with dp4a, lanes splitting each
-//     256-byte slab of K and a warp reduction at the end;
-//   * the fp16 outlier term sum_{j in O} X[i,j] * fp16(Wq[n,j] * w_scale[n]) ([P5] "如何在
-//     PyTorch 2.9 中启用 LLM.int8 推理": no fp16 weights are kept) and the epilogue
-//     Y = fp16(acc * sx * w_scale + P + bias) follow in the same warps.
+//   few_quant_kernel  one thread-block cluster (<= 8 CTAs, each a strip of columns) reads X
+//                     once and finds the outlier columns, max_i |x| > threshold ([P2]
+//                     "8位量化实战：离群值处理与显存优化避坑指南" section 2.3), the row scales
+//                     sx = max over the regular columns / 127 -- the strips exchange their
+//                     row maxima and outlier counts through distributed shared memory --
+//                     and writes q = rne(x / sx) clamped to [-127, 127], 0 in outlier
+//                     columns ([P5] "PyTorch 2.9 支持 LLM.int8()" item 2), as int8 rows
+//                     padded to 16, plus the compact outlier list with its fp16 values.
+//   gemv_kernel       one CTA per SM owns C <= 32 output channels over all of K (no split-K,
+//                     no reduction across CTAs).  It starts the TMA stream of its Wq rows
+//                     into a shared-memory ring before it waits for the quantization (the
+//                     quantization kernel lets it start only after its own inputs were
+//                     complete, and the weights are not written by it); then
+//                     acc[i,n] = sum_k q[i,k] * Wq[n,k] exactly in int32 with dp4a, lanes
+//                     splitting each 256-byte slab of K; the fp16 outlier term
+//                     sum_{j in O} X[i,j] * fp16(Wq[n,j] * w_scale[n]) ([P5] "如何在
+//                     PyTorch 2.9 中启用 LLM.int8 推理": no fp16 weights are kept) from the
+//                     compact list; and Y = fp16(acc * sx * w_scale + P + bias).
 //
 // Quantization arithmetic, exact to the IEEE quotient: v = x * r with r = 1/sx rounded to
 // nearest is within 2^-16 of x/sx (|x/sx| <= 127) and the rounded quotient fl(x/sx) is
@@ -31,13 +35,15 @@ namespace i8mm {
 
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
 constexpr int kSlab = 256;              // bytes of K per ring stage (and per TMA box row)
 constexpr int kMaxChannels = 32;        // per CTA
-constexpr int kChPerWarp = kMaxChannels / kWarps;  // 2
 constexpr int kMaxStages = 64;
 constexpr size_t kSmemLimit = 227 * 1024;
+constexpr int kQThreads = 256;          // per CTA of the quantization cluster
+constexpr int kQMaxCtas = 8;            // portable cluster size
+constexpr int kGThreads = 512;          // per CTA of the product
+constexpr int kGWarps = kGThreads / 32;
+constexpr int kChPerWarp = kMaxChannels / kGWarps;  // 2
 
 __device__ __forceinline__ float h2f(uint32_t word, int hi) {
   return __half2float(
@@ -46,6 +52,31 @@ __device__ __forceinline__ float h2f(uint32_t word, int hi) {
 
 __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 // 8 codes of one row chunk, packed little-endian (see the file comment for exactness)
@@ -79,74 +110,57 @@ __device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, 
 
 }  // namespace
 
-struct GemvShared {
-  uint64_t full[kMaxStages];
-  uint64_t empty[kMaxStages];
-  float red[kWarps][kSmallMP];
+// ------------------------------------------------------------------ activation quantization
+
+struct FewQuantShared {
+  float red[kQThreads / 32][kSmallMP];
+  float rowmax_local[kSmallMP];  // read by the other CTAs of the cluster
+  int count_local;               // read by the other CTAs of the cluster
+  int warp_count[kQThreads / 32];
   float sx[kSmallMP];
   float rcp[kSmallMP];
   int zero_row[kSmallMP];
-  int abort;
+  int base;
 };
 
-// [Wq ring: stages x C x 256 B | Xq: MT x kpad | flags: kpad/8 | GemvShared]
-size_t gemv_smem_bytes(int stages, int C, int MT, int kpad) {
-  return 1024 + static_cast<size_t>(stages) * C * kSlab + static_cast<size_t>(MT) * kpad +
-         kpad / 8 + sizeof(GemvShared) + 16;
-}
-
 template <int MT>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemv_kernel(const __grid_constant__ CUtensorMap map_wq, const GemvArgs a) {
-  extern __shared__ uint8_t gemv_smem_raw[];
-  uint8_t* ring = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(gemv_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int C = a.channels, R = a.stages, kpad = a.kpad;
-  const int nst = kpad / kSlab;  // ring stages to consume
-  const int stage_bytes = C * kSlab;
-  int8_t* xq = reinterpret_cast<int8_t*>(ring + static_cast<size_t>(R) * stage_bytes);
-  uint8_t* flags = reinterpret_cast<uint8_t*>(xq + static_cast<size_t>(MT) * kpad);
-  GemvShared& sh = *reinterpret_cast<GemvShared*>(
-      (reinterpret_cast<uintptr_t>(flags + kpad / 8) + 15) & ~static_cast<uintptr_t>(15));
+__global__ void __launch_bounds__(kQThreads) few_quant_kernel(const GemvArgs a) {
+  __shared__ FewQuantShared sh;
+  // Everything this kernel reads may come from the previous launch; once that is complete,
+  // the product kernel may start its weight stream.
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int Q = static_cast<int>(gridDim.x);
+  const int r = static_cast<int>(cluster_rank());
+  const int chunks = a.kpad / 8;
+  const int c_begin = static_cast<int>(static_cast<long long>(r) * chunks / Q);
+  const int c_end = static_cast<int>(static_cast<long long>(r + 1) * chunks / Q);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int n0 = blockIdx.x * C;
   const int M = a.M, K = a.K;
-  volatile int* abort = &sh.abort;
+  // thread t owns the contiguous chunks [t_begin, t_end) of this strip, so the outlier list
+  // comes out in ascending column order
+  const int per = (c_end - c_begin + kQThreads - 1) / kQThreads;
+  const int t_begin = min(c_end, c_begin + static_cast<int>(threadIdx.x) * per);
+  const int t_end = min(c_end, t_begin + per);
+  const bool one_chunk = per <= 1;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < R; ++s) {
-      mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.empty[s], kWarps);
-    }
-    sh.abort = 0;
-    fence_mbarrier_init();
-    prefetch_tmap(&map_wq);
-  }
-  __syncthreads();
-  grid_dependency_wait();  // the inputs may come from the previous launch on the stream
-
-  if (threadIdx.x == 0) {  // start the weight stream before touching X
-    const int first = nst < R ? nst : R;
-    for (int j = 0; j < first; ++j) {
-      mbar_arrive_expect_tx(&sh.full[j], stage_bytes);
-      tma_load_2d(&map_wq, ring + static_cast<size_t>(j) * stage_bytes, &sh.full[j], j * kSlab, n0);
-    }
-  }
-
-  // ---- pass 1: outlier columns and row maxima over the regular columns
-  const int chunks = kpad / 8;  // 8-column chunks, K padded to the slab
+  // ---- phase 1: outlier flags and row maxima of this strip
   float rmax[MT];
 #pragma unroll
   for (int i = 0; i < MT; ++i) rmax[i] = 0.0f;
-  for (int c = threadIdx.x; c < chunks; c += kThreads) {
+  uint4 v[MT];
+  uint32_t my_bits = 0;
+  int my_count = 0;
+  auto load_chunk = [&](int c) {
     const int k = c * 8;
-    uint4 v[MT];
 #pragma unroll
     for (int i = 0; i < MT; ++i) {
       v[i] = make_uint4(0u, 0u, 0u, 0u);
       if (i < M && k < K)
         v[i] = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * K + k));
     }
+  };
+  auto chunk_flags = [&]() {
     __half2 cm[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) cm[e] = __float2half2_rn(0.0f);
@@ -163,7 +177,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (__low2float(cm[e]) > a.threshold) bits |= 1u << (2 * e);
       if (__high2float(cm[e]) > a.threshold) bits |= 1u << (2 * e + 1);
     }
-    flags[c] = static_cast<uint8_t>(bits);
+    return bits;
+  };
+  for (int c = t_begin; c < t_end; ++c) {
+    load_chunk(c);
+    const uint32_t bits = chunk_flags();
+    my_count += __popc(bits);
+    if (one_chunk) my_bits = bits;
 #pragma unroll
     for (int i = 0; i < MT; ++i) {
       const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
@@ -172,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!((bits >> e) & 1u)) rmax[i] = fmaxf(rmax[i], fabsf(h2f(w[e / 2], e & 1)));
     }
   }
+  // row maxima over the strip and the strip's outlier count (exclusive scan per thread)
 #pragma unroll
   for (int i = 0; i < MT; ++i) {
     float m = rmax[i];
@@ -179,37 +200,150 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) sh.red[warp][i] = m;
   }
+  int incl = my_count;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) sh.warp_count[warp] = incl;
   __syncthreads();
+  int my_off = incl - my_count;
+  for (int w = 0; w < warp; ++w) my_off += sh.warp_count[w];
   if (threadIdx.x < MT) {
-    const int i = threadIdx.x;
     float m = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, sh.red[w][i]);
+    for (int w = 0; w < kQThreads / 32; ++w) m = fmaxf(m, sh.red[w][threadIdx.x]);
+    sh.rowmax_local[threadIdx.x] = m;
+  }
+  if (threadIdx.x == 0) {
+    int total = 0;
+    for (int w = 0; w < kQThreads / 32; ++w) total += sh.warp_count[w];
+    sh.count_local = total;
+  }
+  cluster_sync_all();  // every strip's maxima and count are in its shared memory
+
+  // ---- the row scales over all strips, and this strip's place in the outlier list
+  if (threadIdx.x < MT) {
+    const int i = threadIdx.x;
+    const uint32_t local = smem_addr(&sh.rowmax_local[i]);
+    float m = 0.0f;
+    for (int q = 0; q < Q; ++q) m = fmaxf(m, ld_cluster_f32(map_rank(local, q)));
     const float sc = __fdiv_rn(m, 127.0f);
     sh.sx[i] = (i < M) ? sc : 0.0f;
     sh.rcp[i] = (i < M && m > 0.0f) ? __frcp_rn(sc) : 0.0f;
     sh.zero_row[i] = (i >= M) || m == 0.0f;
+    if (r == 0) a.sx[i] = sh.sx[i];
+  }
+  if (threadIdx.x == 32) {
+    const uint32_t local = smem_addr(&sh.count_local);
+    int base = 0, total = 0;
+    for (int q = 0; q < Q; ++q) {
+      const int cq = ld_cluster_s32(map_rank(local, q));
+      if (q < r) base += cq;
+      total += cq;
+    }
+    sh.base = base;
+    if (r == 0) *a.n_out = total;
   }
   __syncthreads();
 
-  // ---- pass 2: int8 activations into shared memory, xq[i * kpad + k] (X re-read from L1/L2)
-  for (int c = threadIdx.x; c < chunks; c += kThreads) {
+  // ---- phase 2: int8 rows xq[i * kpad + k] (16 rows) and the compact outlier list
+  int pos = sh.base + my_off;
+  for (int c = t_begin; c < t_end; ++c) {
+    if (!one_chunk) load_chunk(c);
+    const uint32_t bits = one_chunk ? my_bits : chunk_flags();
     const int k = c * 8;
-    const uint32_t bits = flags[c];
 #pragma unroll
     for (int i = 0; i < MT; ++i) {
       uint2 q = make_uint2(0u, 0u);
-      if (!sh.zero_row[i] && k < K) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * K + k));
-        q = quantize8(v, sh.sx[i], sh.rcp[i], bits);
+      if (!sh.zero_row[i] && k < K) q = quantize8(v[i], sh.sx[i], sh.rcp[i], bits);
+      *reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(i) * a.kpad + k) = q;
+    }
+    uint32_t b = bits;
+    while (b) {
+      const int e = __ffs(b) - 1;
+      b &= b - 1u;
+      a.cols[pos] = k + e;
+#pragma unroll
+      for (int i = 0; i < kSmallMP; ++i) {
+        unsigned short hb = 0;
+        if (i < MT && i < M) {
+          const uint32_t w[4] = {v[i % MT].x, v[i % MT].y, v[i % MT].z, v[i % MT].w};
+          hb = static_cast<unsigned short>((w[e / 2] >> (16 * (e & 1))) & 0xFFFFu);
+        }
+        a.xo[static_cast<size_t>(pos) * kSmallMP + i] = __ushort_as_half(hb);
       }
-      *reinterpret_cast<uint2*>(xq + static_cast<size_t>(i) * kpad + k) = q;
+      ++pos;
     }
   }
+  cluster_sync_all();  // no CTA leaves while the others may still read its shared memory
+}
+
+// ------------------------------------------------------------------ product
+
+struct GemvShared {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  float sx[kSmallMP];
+  int abort;
+  int issued;  // ring stages whose copy was started
+};
+
+// [Wq ring: stages x C x 256 B | Xq: MT x kpad | GemvShared]
+size_t gemv_smem_bytes(int stages, int C, int MT, int kpad) {
+  return 1024 + static_cast<size_t>(stages) * C * kSlab + static_cast<size_t>(MT) * kpad +
+         sizeof(GemvShared) + 16;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kGThreads, 1)
+    gemv_kernel(const __grid_constant__ CUtensorMap map_wq, const GemvArgs a) {
+  extern __shared__ uint8_t gemv_smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(gemv_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int C = a.channels, R = a.stages, kpad = a.kpad;
+  const int nst = kpad / kSlab;  // ring stages to consume
+  const int stage_bytes = C * kSlab;
+  int8_t* xq = reinterpret_cast<int8_t*>(ring + static_cast<size_t>(R) * stage_bytes);
+  GemvShared& sh = *reinterpret_cast<GemvShared*>(xq + static_cast<size_t>(MT) * kpad);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n0 = blockIdx.x * C;
+  const int M = a.M;
+  volatile int* abort = &sh.abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < R; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.empty[s], kGWarps);
+    }
+    sh.abort = 0;
+    fence_mbarrier_init();
+    prefetch_tmap(&map_wq);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // the weight stream starts before the activations are ready
+    const int first = nst < R ? nst : R;
+    for (int j = 0; j < first; ++j) {
+      mbar_arrive_expect_tx(&sh.full[j], stage_bytes);
+      tma_load_2d(&map_wq, ring + static_cast<size_t>(j) * stage_bytes, &sh.full[j], j * kSlab, n0);
+    }
+    sh.issued = first;
+  }
+  grid_dependency_wait();  // the quantization kernel is complete from here on
+
+  // ---- int8 activations (rows < MT) and row scales into shared memory
+  {
+    const int vec = MT * kpad / 16;
+    const uint4* src = reinterpret_cast<const uint4*>(a.xq);
+    uint4* dst = reinterpret_cast<uint4*>(xq);
+    for (int t = threadIdx.x; t < vec; t += kGThreads) dst[t] = __ldcg(src + t);
+    if (threadIdx.x < kSmallMP) sh.sx[threadIdx.x] = __ldcg(a.sx + threadIdx.x);
+  }
+  const int n_out = __ldcg(a.n_out);
   __syncthreads();
 
-  // ---- int32 products on the CUDA cores: warp w owns channels w and w + 16 of the CTA;
-  // lane l owns bytes [8l, 8l + 8) of every 256-byte slab of K.
+  // ---- int32 products: warp w owns channels w and w + 16; lane l bytes [8l, 8l+8) of a slab
   int ch_count = a.N - n0;
   if (ch_count > C) ch_count = C;
   int32_t acc[kChPerWarp][MT];
@@ -220,11 +354,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool ok = true;
   for (int j = 0; j < nst; ++j) {
     const int s = j % R;
-    const bool landed = mbar_wait_bounded(&sh.full[s], static_cast<uint32_t>(j / R) & 1u, abort);
-    if (!__all_sync(0xffffffffu, landed)) {  // a warp-uniform decision
+    const uint32_t parity = static_cast<uint32_t>(j / R) & 1u;
+    bool landed = true;
+    if (lane == 0) landed = mbar_wait_bounded(&sh.full[s], parity, abort);
+    if (!__shfl_sync(0xffffffffu, landed ? 1 : 0, 0)) {
       ok = false;
       break;
     }
+    mbar_try_wait(&sh.full[s], parity);  // each lane observes the completed phase
     const uint8_t* tile = ring + static_cast<size_t>(s) * stage_bytes;
     uint2 xw[MT];
 #pragma unroll
@@ -234,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       : make_uint2(0u, 0u);
 #pragma unroll
     for (int r = 0; r < kChPerWarp; ++r) {
-      const int ch = warp + kWarps * r;
+      const int ch = warp + kGWarps * r;
       if (ch < ch_count) {
         const uint2 ww = *reinterpret_cast<const uint2*>(tile + ch * kSlab + 8 * lane);
 #pragma unroll
@@ -248,51 +385,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.empty[s]);
       if (threadIdx.x == 0) {
-        if (!mbar_wait_bounded(&sh.empty[s], static_cast<uint32_t>(j / R) & 1u, abort)) {
+        if (!mbar_wait_bounded(&sh.empty[s], parity, abort)) {
           ok = false;
         } else {
           mbar_arrive_expect_tx(&sh.full[s], stage_bytes);
           tma_load_2d(&map_wq, ring + static_cast<size_t>(s) * stage_bytes, &sh.full[s],
                       (j + R) * kSlab, n0);
+          sh.issued = j + R + 1;
         }
       }
     }
   }
   if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
 
-  // ---- fp16 outlier term: lanes stride over the outlier flags; weight bytes come from the
-  // resident ring when the whole slice fits, from global memory otherwise
+  // ---- fp16 outlier term from the compact list; weight bytes from the resident ring when
+  // the whole slice fits, from global memory otherwise
   float P[kChPerWarp][MT];
 #pragma unroll
   for (int r = 0; r < kChPerWarp; ++r)
 #pragma unroll
     for (int i = 0; i < MT; ++i) P[r][i] = 0.0f;
   const bool resident = nst <= R;
-  for (int c = lane; c < chunks; c += 32) {
-    uint32_t bits = flags[c];
-    while (bits) {
-      const int j = c * 8 + __ffs(bits) - 1;
-      bits &= bits - 1u;
-      float xv[MT];
+  for (int o = lane; o < n_out; o += 32) {
+    const int j = __ldcg(a.cols + o);
+    float xv[MT];
 #pragma unroll
-      for (int i = 0; i < MT; ++i)
-        xv[i] = (i < M) ? __half2float(a.X[static_cast<size_t>(i) * K + j]) : 0.0f;
+    for (int i = 0; i < MT; ++i)
+      xv[i] = __half2float(a.xo[static_cast<size_t>(o) * kSmallMP + i]);
 #pragma unroll
-      for (int r = 0; r < kChPerWarp; ++r) {
-        const int ch = warp + kWarps * r;
-        if (ch < ch_count) {
-          const int8_t q = resident ? static_cast<int8_t>(ring[static_cast<size_t>(j / kSlab) * stage_bytes +
-                                                              ch * kSlab + j % kSlab])
-                                    : a.Wq[static_cast<size_t>(n0 + ch) * K + j];
-          const float wv = __half2float(__float2half_rn(static_cast<float>(q) * a.w_scale[n0 + ch]));
+    for (int r = 0; r < kChPerWarp; ++r) {
+      const int ch = warp + kGWarps * r;
+      if (ch < ch_count) {
+        const int8_t q = resident ? static_cast<int8_t>(ring[static_cast<size_t>(j / kSlab) * stage_bytes +
+                                                            ch * kSlab + j % kSlab])
+                                  : a.Wq[static_cast<size_t>(n0 + ch) * a.K + j];
+        const float wv = __half2float(__float2half_rn(static_cast<float>(q) * a.w_scale[n0 + ch]));
 #pragma unroll
-          for (int i = 0; i < MT; ++i) P[r][i] += wv * xv[i];
-        }
+        for (int i = 0; i < MT; ++i) P[r][i] += wv * xv[i];
       }
     }
   }
 
-  // ---- reduce over the 32 lanes and write Y (lane l writes pair (r, i) = (l / MT, l % MT))
+  // ---- reduce over the 32 lanes; lane l writes pair (r, i) = (l / MT, l % MT)
 #pragma unroll
   for (int r = 0; r < kChPerWarp; ++r) {
 #pragma unroll
@@ -306,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 #pragma unroll
   for (int r = 0; r < kChPerWarp; ++r) {
-    const int ch = warp + kWarps * r;
+    const int ch = warp + kGWarps * r;
     const int n = n0 + ch;
 #pragma unroll
     for (int i = 0; i < MT; ++i) {
@@ -319,6 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
+  if (threadIdx.x == 0 && sh.abort) {
+    // a wait gave up: let the copies still in flight land before the block exits
+    int dummy = 0;
+    for (int d = sh.issued > R ? sh.issued - R : 0; d < sh.issued; ++d)
+      mbar_wait_bounded(&sh.full[d % R], static_cast<uint32_t>(d / R) & 1u, &dummy);
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -336,8 +476,29 @@ GemvPlan plan_gemv(int M, int N, int K, int num_sms) {
   int R = nst < kMaxStages ? nst : kMaxStages;
   while (R > 2 && gemv_smem_bytes(R, C, p.mt, p.kpad) > kSmemLimit) --R;
   p.stages = R;
+  const int chunks = p.kpad / 8;
+  int Q = (chunks + kQThreads - 1) / kQThreads;
+  p.quant_ctas = Q < 1 ? 1 : (Q > kQMaxCtas ? kQMaxCtas : Q);
   p.fits = M <= kSmallMP && gemv_smem_bytes(R, C, p.mt, p.kpad) <= kSmemLimit;
   return p;
+}
+
+cudaError_t launch_few_quant(const GemvArgs& a, const GemvPlan& p, cudaStream_t stream, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.quant_ctas);
+  cfg.blockDim = dim3(kQThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.quant_ctas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return p.mt == 8 ? cudaLaunchKernelEx(&cfg, few_quant_kernel<8>, a)
+                   : cudaLaunchKernelEx(&cfg, few_quant_kernel<kSmallMP>, a);
 }
 
 cudaError_t launch_gemv(const CUtensorMap& map_wq, const GemvArgs& a, const GemvPlan& p,
@@ -357,7 +518,7 @@ cudaError_t launch_gemv(const CUtensorMap& map_wq, const GemvArgs& a, const Gemv
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.ctas);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kGThreads);
   cfg.dynamicSmemBytes = gemv_smem_bytes(p.stages, p.channels, p.mt, p.kpad);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -22,15 +22,17 @@ namespace i8mm {
 //   xo       half[M*ldo]    outlier activations, compacted, zero-padded to a multiple of 64
 //   wo       half[N*ldo]    outlier weights fp16(Wq*w_scale), compacted, zero-padded
 // ldo = K rounded up to 64 (the fp16 operand tiles are 64 elements deep).
-// The few-token path (M <= kSmallMP) runs in one cluster kernel (small.cu) and keeps its
-// intermediates in shared memory; it uses only the status word of the workspace.
+// The few-token path (M <= kSmallMP) adds: int8 activations padded to 16 rows and to a
+// multiple of 256 columns (few_xq, int8[16*kpad]), the fp16 values of the outlier columns
+// (few_xo, half[K*16], outlier r at [r*16 + i]) and the 16 row scales (few_sx); the outlier
+// count and list use header[1] and cols.
 constexpr int kSmallMP = 16;             // tokens per MMA (N of the swapped product)
 constexpr int kSmallBN = 128;            // output channels per tile (M of the MMA)
 constexpr int kSmallMaxSplits = 8;       // CTAs per cluster (portable cluster size)
 constexpr int kSmallMaxKbPerSplit = 16;  // 128-byte k-blocks of X / Xq one CTA keeps in smem
 
 struct WorkspaceLayout {
-  size_t header, mask, cols, xscale, xq, xo, wo, total;
+  size_t header, mask, cols, xscale, xq, xo, wo, few_xq, few_xo, few_sx, total;
   int ldo;
 };
 
@@ -47,6 +49,13 @@ inline WorkspaceLayout workspace_layout(int M, int N, int K) {
   L.xq = off;     off = align256(off + static_cast<size_t>(M) * K);
   L.xo = off;     off = align256(off + static_cast<size_t>(M) * L.ldo * sizeof(__half));
   L.wo = off;     off = align256(off + static_cast<size_t>(N) * L.ldo * sizeof(__half));
+  L.few_xq = L.few_xo = L.few_sx = off;
+  if (M <= kSmallMP) {
+    const size_t kpad = static_cast<size_t>((K + 255) / 256) * 256;
+    L.few_xq = off; off = align256(off + kSmallMP * kpad);
+    L.few_xo = off; off = align256(off + static_cast<size_t>(K) * kSmallMP * sizeof(__half));
+    L.few_sx = off; off = align256(off + kSmallMP * sizeof(float));
+  }
   L.total = off;
   return L;
 }
@@ -118,13 +127,20 @@ struct GemvArgs {
   int channels;          // output channels per CTA
   int stages;            // depth of the Wq ring (256-byte slabs of K)
   int kpad;              // K rounded up to 256
+  int quant_ctas;        // CTAs (one cluster) of the activation-quantization kernel
+  int8_t* xq;            // [16][kpad] int8 activations (written by the quantization kernel)
+  __half* xo;            // [n_out][16] fp16 activations of the outlier columns
+  float* sx;             // [16] row scales
+  int32_t* cols;         // [K] outlier columns, ascending
+  int32_t* n_out;        // outlier count
   int32_t* status;
 };
 struct GemvPlan {
-  int mt, channels, ctas, kpad, stages;
+  int mt, channels, ctas, kpad, stages, quant_ctas;
   bool fits;
 };
 GemvPlan plan_gemv(int M, int N, int K, int num_sms);
+cudaError_t launch_few_quant(const GemvArgs& a, const GemvPlan& p, cudaStream_t stream, bool pdl);
 cudaError_t launch_gemv(const CUtensorMap& map_wq, const GemvArgs& a, const GemvPlan& p,
                         cudaStream_t stream, bool pdl);
 int device_sm_count();

@@ -51,19 +51,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Every wait in this library is bounded: it gives up after kWaitIters polls or
 // kWaitNs nanoseconds, whichever comes first, or as soon as *abort is set by another
-// role of the same CTA.  On giving up it sets *abort and returns false.  After a few fast
-// polls the waiting thread sleeps between polls (up to kMaxSleepNs), so that waiters do
-// not flood the shared-memory pipe the working warps of the SM depend on.
+// role of the same CTA.  On giving up it sets *abort and returns false.  Short waits poll
+// (try_wait itself suspends the thread briefly); only waits longer than kFastPolls polls
+// sleep between polls (up to kMaxSleepNs), so that long waiters leave the issue slots and
+// the shared-memory pipe to the working warps.
 constexpr uint32_t kWaitIters = 1u << 26;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
-constexpr uint32_t kFastPolls = 8;
-constexpr uint32_t kMaxSleepNs = 64;
+constexpr uint32_t kFastPolls = 4096;
+constexpr uint32_t kMaxSleepNs = 256;
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t sleep_ns = 8;
+  uint32_t sleep_ns = 32;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if (it >= kFastPolls) {
