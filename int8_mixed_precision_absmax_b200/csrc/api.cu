@@ -220,9 +220,14 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
     if (gp.fits) {
       const GemvArgs g = gemv_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace,
                                    p, gp);
+      // Wq viewed as [K/128 k-blocks][N rows][128 bytes]: one box is 32 rows x 8 k-blocks,
+      // each k-block landing as a 128-byte-swizzled 32 x 128 tile
       CUtensorMap map;
-      if (!encode_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, 256,
-                          static_cast<uint32_t>(gp.channels), CU_TENSOR_MAP_SWIZZLE_NONE))
+      const uint64_t dims[3] = {128, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 128)};
+      const uint64_t strides[2] = {static_cast<uint64_t>(K), 128};
+      const uint32_t box[3] = {128, static_cast<uint32_t>(gp.channels), 8};
+      if (!encode_tmap_3d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, dims, strides, box,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
         return INT8MM_ERR_CUDA;
       return launch_status(launch_gemv(map, g, gp, stream, pdl));
     }

@@ -13,21 +13,25 @@
 //                     and writes q = rne(x / sx) clamped to [-127, 127], 0 in outlier
 //                     columns ([P5] "PyTorch 2.9 支持 LLM.int8()" item 2), as int8 rows
 //                     padded to 16, plus the compact outlier list with its fp16 values.
-//   gemv_kernel       one CTA per SM owns C <= 32 output channels over all of K (no split-K,
-//                     no reduction across CTAs).  It starts the TMA stream of its Wq rows
-//                     into a shared-memory ring before it waits for the quantization (the
-//                     quantization kernel lets it start only after its own inputs were
-//                     complete, and the weights are not written by it); then
-//                     acc[i,n] = sum_k q[i,k] * Wq[n,k] exactly in int32 with dp4a, lanes
-//                     splitting each 256-byte slab of K; the fp16 outlier term
-//                     sum_{j in O} X[i,j] * fp16(Wq[n,j] * w_scale[n]) ([P5] "如何在
-//                     PyTorch 2.9 中启用 LLM.int8 推理": no fp16 weights are kept) from the
-//                     compact list; and Y = fp16(acc * sx * w_scale + P + bias).
+//   gemv_kernel       each CTA owns 32 output channels over all of K (no split-K, no
+//                     reduction across CTAs).  It starts the TMA stream of its Wq rows into
+//                     shared memory (32 KB boxes: 32 rows x 8 swizzled 128-byte k-blocks)
+//                     before it waits for the quantization (that kernel lets it start only
+//                     after its own inputs were complete; the weights are not written by it).
+//                     Each warp owns a range of K and computes acc[i,n] = sum_k q[i,k]*Wq[n,k]
+//                     exactly with the int8 warp-level MMA m16n8k32 (16 channels x 8 tokens x
+//                     32 K per instruction; a tcgen05 MMA with M = 128 channels takes the same
+//                     time at N = 8 tokens as at N = 256, so at this shape it would idle);
+//                     the warps' partial sums meet in shared memory.  The fp16 outlier term
+//                     sum_{j in O} X[i,j] * fp16(Wq[n,j] * w_scale[n]) ([P5] "如何在 PyTorch
+//                     2.9 中启用 LLM.int8 推理": no fp16 weights are kept) comes from the
+//                     compact list, and Y = fp16(acc * sx * w_scale + P + bias).
 //
-// Quantization arithmetic, exact to the IEEE quotient: v = x * r with r = 1/sx rounded to
-// nearest is within 2^-16 of x/sx (|x/sx| <= 127) and the rounded quotient fl(x/sx) is
-// within 2^-18 of x/sx, so rne(v) = rne(fl(x/sx)) unless v lies within 2^-15 of a
-// half-integer; there the quotient itself (__fdiv_rn) is rounded.
+// Quantization arithmetic, exact to the IEEE quotient.  With r = 1/sx rounded to nearest,
+// the exact product x*r is within 2^-17 of x/sx (|x/sx| <= 128) and the rounded quotient
+// fl(x/sx) within 2^-18, so rne(x*r) = rne(fl(x/sx)) unless x*r lies within 2^-15 of a
+// half-integer, where the quotient itself (__fdiv_rn) is rounded.  rne(x*r) is formed by one
+// fused multiply-add with 1.5*2^23, whose bits hold the integer.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -35,15 +39,16 @@ namespace i8mm {
 
 namespace {
 
-constexpr int kSlab = 256;              // bytes of K per ring stage (and per TMA box row)
-constexpr int kMaxChannels = 32;        // per CTA
-constexpr int kMaxStages = 64;
+constexpr int kSlab = 256;              // activation rows are padded to this many bytes
 constexpr size_t kSmemLimit = 227 * 1024;
 constexpr int kQThreads = 256;          // per CTA of the quantization cluster
 constexpr int kQMaxCtas = 8;            // portable cluster size
 constexpr int kGThreads = 512;          // per CTA of the product
 constexpr int kGWarps = kGThreads / 32;
-constexpr int kChPerWarp = kMaxChannels / kGWarps;  // 2
+constexpr int kCh = 32;                 // output channels per CTA: two m16 tiles
+constexpr int kBoxKb = 8;               // 128-byte k-blocks per TMA box
+constexpr int kBoxBytes = kCh * kBoxKb * 128;  // 32 KB
+constexpr int kMaxBoxes = 6;            // ring depth (boxes)
 
 __device__ __forceinline__ float h2f(uint32_t word, int hi) {
   return __half2float(
@@ -81,6 +86,7 @@ __device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
 
 // 8 codes of one row chunk, packed little-endian (see the file comment for exactness)
 __device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, uint32_t bits) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   float x[8];
   int qv[8];
@@ -88,9 +94,9 @@ __device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, 
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     x[e] = h2f(w[e / 2], e & 1);
-    const float t = x[e] * rcp;
-    qv[e] = __float2int_rn(t);
-    const float d = fabsf(t - rintf(t));
+    const float tb = __fmaf_rn(x[e], rcp, kRound);      // rne(x*r) + 1.5*2^23, exactly
+    qv[e] = __float_as_int(tb) - 0x4B400000;              // the integer rne(x*r)
+    const float d = fabsf(__fmaf_rn(x[e], rcp, -(tb - kRound)));  // |x*r - rne(x*r)|
     near_tie |= (fabsf(d - 0.5f) <= 0x1p-15f ? 1u : 0u) << e;
   }
   if (near_tie) {
@@ -106,6 +112,16 @@ __device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, 
     p[e / 4] |= code << (8 * (e & 3));
   }
   return make_uint2(p[0], p[1]);
+}
+
+// D(16 x 8, int32) += A(16 x 32, int8, row-major) * B(32 x 8, int8, column-major)
+__device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 }  // namespace
@@ -283,17 +299,23 @@ __global__ void __launch_bounds__(kQThreads) few_quant_kernel(const GemvArgs a) 
 // ------------------------------------------------------------------ product
 
 struct GemvShared {
-  uint64_t full[kMaxStages];
-  uint64_t empty[kMaxStages];
+  uint64_t full[kMaxBoxes];
+  uint64_t empty[kMaxBoxes];
   float sx[kSmallMP];
   int abort;
-  int issued;  // ring stages whose copy was started
+  int issued;  // boxes whose copy was started
 };
 
-// [Wq ring: stages x C x 256 B | Xq: MT x kpad | GemvShared]
-size_t gemv_smem_bytes(int stages, int C, int MT, int kpad) {
-  return 1024 + static_cast<size_t>(stages) * C * kSlab + static_cast<size_t>(MT) * kpad +
-         sizeof(GemvShared) + 16;
+// [Wq ring: boxes x 32 KB | partial sums: 16 warps x 32 channels x MT | GemvShared]
+size_t gemv_smem_bytes(int boxes, int MT) {
+  return 1024 + static_cast<size_t>(boxes) * kBoxBytes +
+         static_cast<size_t>(kGWarps) * kCh * MT * sizeof(int32_t) + sizeof(GemvShared) + 16;
+}
+
+// byte (row, kk) of a 32-row tile of 128-byte rows written with the 128-byte swizzle
+__device__ __forceinline__ uint32_t sw128_offset(int row, int kk) {
+  return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 +
+                               ((((kk >> 4) ^ (row & 7))) << 4) + (kk & 15));
 }
 
 template <int MT>
@@ -302,13 +324,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
   extern __shared__ uint8_t gemv_smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(gemv_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int C = a.channels, R = a.stages, kpad = a.kpad;
-  const int nst = kpad / kSlab;  // ring stages to consume
-  const int stage_bytes = C * kSlab;
-  int8_t* xq = reinterpret_cast<int8_t*>(ring + static_cast<size_t>(R) * stage_bytes);
-  GemvShared& sh = *reinterpret_cast<GemvShared*>(xq + static_cast<size_t>(MT) * kpad);
+  const int R = a.stages;                       // ring depth in boxes
+  const int kb_total = a.K / 128;               // 128-byte k-blocks (K % 128 == 0 here)
+  const int nbox = (kb_total + kBoxKb - 1) / kBoxKb;
+  int32_t* red = reinterpret_cast<int32_t*>(ring + static_cast<size_t>(R) * kBoxBytes);
+  GemvShared& sh = *reinterpret_cast<GemvShared*>(red + kGWarps * kCh * MT);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int n0 = blockIdx.x * C;
+  const int n0 = blockIdx.x * kCh;
   const int M = a.M;
   volatile int* abort = &sh.abort;
 
@@ -323,163 +345,137 @@ __global__ void __launch_bounds__(kGThreads, 1)
   }
   __syncthreads();
   if (threadIdx.x == 0) {  // the weight stream starts before the activations are ready
-    const int first = nst < R ? nst : R;
-    for (int j = 0; j < first; ++j) {
-      mbar_arrive_expect_tx(&sh.full[j], stage_bytes);
-      tma_load_2d(&map_wq, ring + static_cast<size_t>(j) * stage_bytes, &sh.full[j], j * kSlab, n0);
+    const int first = nbox < R ? nbox : R;
+    for (int b = 0; b < first; ++b) {
+      mbar_arrive_expect_tx(&sh.full[b], kBoxBytes);
+      tma_load_3d(&map_wq, ring + static_cast<size_t>(b) * kBoxBytes, &sh.full[b], 0, n0,
+                  b * kBoxKb);
     }
     sh.issued = first;
   }
   grid_dependency_wait();  // the quantization kernel is complete from here on
 
-  // ---- int8 activations (rows < MT) and row scales into shared memory
-  {
-    const int vec = MT * kpad / 16;
-    const uint4* src = reinterpret_cast<const uint4*>(a.xq);
-    uint4* dst = reinterpret_cast<uint4*>(xq);
-    for (int t = threadIdx.x; t < vec; t += kGThreads) dst[t] = __ldcg(src + t);
-    if (threadIdx.x < kSmallMP) sh.sx[threadIdx.x] = __ldcg(a.sx + threadIdx.x);
-  }
-  const int n_out = __ldcg(a.n_out);
-  __syncthreads();
-
-  // ---- int32 products: warp w owns channels w and w + 16; lane l bytes [8l, 8l+8) of a slab
-  int ch_count = a.N - n0;
-  if (ch_count > C) ch_count = C;
-  int32_t acc[kChPerWarp][MT];
+  // ---- this warp's k32 steps: [s_begin, s_end) of K/32, inside one box each time
+  const int steps = a.K / 32;
+  const int per = (steps + kGWarps - 1) / kGWarps;
+  const int s_begin = min(steps, warp * per), s_end = min(steps, s_begin + per);
+  const int g = lane >> 2, tig = lane & 3;
+  constexpr int NT = MT / 8;  // n8 tiles of tokens
+  int d[2][NT][4];
 #pragma unroll
-  for (int r = 0; r < kChPerWarp; ++r)
+  for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int i = 0; i < MT; ++i) acc[r][i] = 0;
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d[m][t][e] = 0;
   bool ok = true;
-  for (int j = 0; j < nst; ++j) {
-    const int s = j % R;
-    const uint32_t parity = static_cast<uint32_t>(j / R) & 1u;
-    bool landed = true;
-    if (lane == 0) landed = mbar_wait_bounded(&sh.full[s], parity, abort);
-    if (!__shfl_sync(0xffffffffu, landed ? 1 : 0, 0)) {
-      ok = false;
-      break;
-    }
-    mbar_try_wait(&sh.full[s], parity);  // each lane observes the completed phase
-    const uint8_t* tile = ring + static_cast<size_t>(s) * stage_bytes;
-    uint2 xw[MT];
-#pragma unroll
-    for (int i = 0; i < MT; ++i)
-      xw[i] = (i < M) ? *reinterpret_cast<const uint2*>(xq + static_cast<size_t>(i) * kpad +
-                                                       j * kSlab + 8 * lane)
-                      : make_uint2(0u, 0u);
-#pragma unroll
-    for (int r = 0; r < kChPerWarp; ++r) {
-      const int ch = warp + kGWarps * r;
-      if (ch < ch_count) {
-        const uint2 ww = *reinterpret_cast<const uint2*>(tile + ch * kSlab + 8 * lane);
-#pragma unroll
-        for (int i = 0; i < MT; ++i) {
-          acc[r][i] = __dp4a(static_cast<int>(ww.x), static_cast<int>(xw[i].x), acc[r][i]);
-          acc[r][i] = __dp4a(static_cast<int>(ww.y), static_cast<int>(xw[i].y), acc[r][i]);
-        }
+  int waited_box = -1;
+  for (int st = s_begin; st < s_end; ++st) {
+    const int k0 = st * 32;
+    const int box = k0 / (kBoxKb * 128);
+    if (box != waited_box) {  // boxes are consumed in order; R >= boxes here (resident)
+      const int slot = box % R;
+      const uint32_t parity = static_cast<uint32_t>(box / R) & 1u;
+      bool landed = true;
+      if (lane == 0) landed = mbar_wait_bounded(&sh.full[slot], parity, abort);
+      if (!__shfl_sync(0xffffffffu, landed ? 1 : 0, 0)) {
+        ok = false;
+        break;
       }
+      mbar_try_wait(&sh.full[slot], parity);  // each lane observes the completed phase
+      waited_box = box;
     }
-    if (j + R < nst) {  // refill this stage once every warp is done with it
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.empty[s]);
-      if (threadIdx.x == 0) {
-        if (!mbar_wait_bounded(&sh.empty[s], parity, abort)) {
-          ok = false;
-        } else {
-          mbar_arrive_expect_tx(&sh.full[s], stage_bytes);
-          tma_load_2d(&map_wq, ring + static_cast<size_t>(s) * stage_bytes, &sh.full[s],
-                      (j + R) * kSlab, n0);
-          sh.issued = j + R + 1;
-        }
-      }
+    const uint8_t* tile = ring + static_cast<size_t>(box % R) * kBoxBytes +
+                          ((k0 / 128) % kBoxKb) * (kCh * 128);
+    const int kk = k0 % 128 + 4 * tig;
+    uint32_t b[NT][2];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int8_t* xrow = a.xq + static_cast<size_t>(t * 8 + g) * a.kpad + k0 + 4 * tig;
+      b[t][0] = __ldcg(reinterpret_cast<const unsigned int*>(xrow));
+      b[t][1] = __ldcg(reinterpret_cast<const unsigned int*>(xrow + 16));
+    }
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      uint32_t af[4];
+      af[0] = *reinterpret_cast<const uint32_t*>(tile + sw128_offset(m * 16 + g, kk));
+      af[1] = *reinterpret_cast<const uint32_t*>(tile + sw128_offset(m * 16 + g + 8, kk));
+      af[2] = *reinterpret_cast<const uint32_t*>(tile + sw128_offset(m * 16 + g, kk + 16));
+      af[3] = *reinterpret_cast<const uint32_t*>(tile + sw128_offset(m * 16 + g + 8, kk + 16));
+#pragma unroll
+      for (int t = 0; t < NT; ++t) mma_s8_16832(d[m][t], af, b[t][0], b[t][1]);
     }
   }
   if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
+  // partial sums to shared memory: red[warp][channel][token]
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      int32_t* rw = red + static_cast<size_t>(warp) * kCh * MT;
+      rw[(m * 16 + g) * MT + t * 8 + 2 * tig] = d[m][t][0];
+      rw[(m * 16 + g) * MT + t * 8 + 2 * tig + 1] = d[m][t][1];
+      rw[(m * 16 + g + 8) * MT + t * 8 + 2 * tig] = d[m][t][2];
+      rw[(m * 16 + g + 8) * MT + t * 8 + 2 * tig + 1] = d[m][t][3];
+    }
+  if (threadIdx.x < kSmallMP) sh.sx[threadIdx.x] = __ldcg(a.sx + threadIdx.x);
+  __syncthreads();
 
-  // ---- fp16 outlier term from the compact list; weight bytes from the resident ring when
-  // the whole slice fits, from global memory otherwise
-  float P[kChPerWarp][MT];
+  // ---- thread (c, i): sum the warps, add the outlier term and bias, write Y[i, n0 + c]
+  const int n_out = __ldcg(a.n_out);
+  const bool resident = nbox <= R;
+  for (int t = threadIdx.x; t < kCh * MT; t += kGThreads) {
+    const int c = t % kCh, i = t / kCh, n = n0 + c;
+    if (i >= M || n >= a.N) continue;
+    int32_t acc = 0;
 #pragma unroll
-  for (int r = 0; r < kChPerWarp; ++r)
-#pragma unroll
-    for (int i = 0; i < MT; ++i) P[r][i] = 0.0f;
-  const bool resident = nst <= R;
-  for (int o = lane; o < n_out; o += 32) {
-    const int j = __ldcg(a.cols + o);
-    float xv[MT];
-#pragma unroll
-    for (int i = 0; i < MT; ++i)
-      xv[i] = __half2float(a.xo[static_cast<size_t>(o) * kSmallMP + i]);
-#pragma unroll
-    for (int r = 0; r < kChPerWarp; ++r) {
-      const int ch = warp + kGWarps * r;
-      if (ch < ch_count) {
-        const int8_t q = resident ? static_cast<int8_t>(ring[static_cast<size_t>(j / kSlab) * stage_bytes +
-                                                            ch * kSlab + j % kSlab])
-                                  : a.Wq[static_cast<size_t>(n0 + ch) * a.K + j];
-        const float wv = __half2float(__float2half_rn(static_cast<float>(q) * a.w_scale[n0 + ch]));
-#pragma unroll
-        for (int i = 0; i < MT; ++i) P[r][i] += wv * xv[i];
+    for (int w = 0; w < kGWarps; ++w) acc += red[(static_cast<size_t>(w) * kCh + c) * MT + i];
+    const float swn = a.w_scale[n];
+    float P = 0.0f;
+    for (int o = 0; o < n_out; ++o) {
+      const int j = __ldcg(a.cols + o);
+      int8_t q;
+      if (resident) {
+        const int kb = j / 128;
+        const uint8_t* tile = ring + static_cast<size_t>(kb / kBoxKb) * kBoxBytes +
+                              (kb % kBoxKb) * (kCh * 128);
+        q = static_cast<int8_t>(tile[sw128_offset(c, j % 128)]);
+      } else {
+        q = a.Wq[static_cast<size_t>(n) * a.K + j];
       }
+      const float wv = __half2float(__float2half_rn(static_cast<float>(q) * swn));
+      P += wv * __half2float(a.xo[static_cast<size_t>(o) * kSmallMP + i]);
     }
-  }
-
-  // ---- reduce over the 32 lanes; lane l writes pair (r, i) = (l / MT, l % MT)
-#pragma unroll
-  for (int r = 0; r < kChPerWarp; ++r) {
-#pragma unroll
-    for (int i = 0; i < MT; ++i) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        acc[r][i] += __shfl_xor_sync(0xffffffffu, acc[r][i], o);
-        P[r][i] += __shfl_xor_sync(0xffffffffu, P[r][i], o);
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < kChPerWarp; ++r) {
-    const int ch = warp + kGWarps * r;
-    const int n = n0 + ch;
-#pragma unroll
-    for (int i = 0; i < MT; ++i) {
-      if (lane == (r * MT + i) % 32 && ch < ch_count && i < M) {
-        const float b = a.bias ? __half2float(a.bias[n]) : 0.0f;
-        const float y = static_cast<float>(acc[r][i]) * sh.sx[i] * a.w_scale[n] + P[r][i] + b;
-        a.Y[static_cast<size_t>(i) * a.N + n] = __float2half_rn(y);
-        if (a.acc) a.acc[static_cast<size_t>(i) * a.N + n] = ok ? acc[r][i] : 0;
-      }
-    }
+    const float bb = a.bias ? __half2float(a.bias[n]) : 0.0f;
+    const float y = static_cast<float>(acc) * sh.sx[i] * swn + P + bb;
+    a.Y[static_cast<size_t>(i) * a.N + n] = __float2half_rn(y);
+    if (a.acc) a.acc[static_cast<size_t>(i) * a.N + n] = ok ? acc : 0;
   }
   __syncthreads();
   if (threadIdx.x == 0 && sh.abort) {
     // a wait gave up: let the copies still in flight land before the block exits
     int dummy = 0;
-    for (int d = sh.issued > R ? sh.issued - R : 0; d < sh.issued; ++d)
-      mbar_wait_bounded(&sh.full[d % R], static_cast<uint32_t>(d / R) & 1u, &dummy);
+    for (int b2 = sh.issued > R ? sh.issued - R : 0; b2 < sh.issued; ++b2)
+      mbar_wait_bounded(&sh.full[b2 % R], static_cast<uint32_t>(b2 / R) & 1u, &dummy);
   }
 }
 
 // ------------------------------------------------------------------ host side
 
 GemvPlan plan_gemv(int M, int N, int K, int num_sms) {
+  (void)num_sms;
   GemvPlan p;
   p.mt = M <= 8 ? 8 : kSmallMP;
-  int C = (N + num_sms - 1) / num_sms;
-  if (C < 1) C = 1;
-  if (C > kMaxChannels) C = kMaxChannels;
-  p.channels = C;
-  p.ctas = (N + C - 1) / C;
+  p.channels = kCh;
+  p.ctas = (N + kCh - 1) / kCh;
   p.kpad = (K + kSlab - 1) / kSlab * kSlab;
-  const int nst = p.kpad / kSlab;
-  int R = nst < kMaxStages ? nst : kMaxStages;
-  while (R > 2 && gemv_smem_bytes(R, C, p.mt, p.kpad) > kSmemLimit) --R;
-  p.stages = R;
+  const int nbox = (K / 128 + kBoxKb - 1) / kBoxKb;
+  p.stages = nbox;  // the whole slice stays resident: the outlier term reads it back
   const int chunks = p.kpad / 8;
-  int Q = (chunks + kQThreads - 1) / kQThreads;
+  int Q = (chunks + 63) / 64;  // about 64 chunks (512 columns) per CTA of the cluster
   p.quant_ctas = Q < 1 ? 1 : (Q > kQMaxCtas ? kQMaxCtas : Q);
-  p.fits = M <= kSmallMP && gemv_smem_bytes(R, C, p.mt, p.kpad) <= kSmemLimit;
+  p.fits = M <= kSmallMP && K % 128 == 0 && nbox <= kMaxBoxes &&
+           gemv_smem_bytes(nbox, p.mt) <= kSmemLimit;
   return p;
 }
 
@@ -519,7 +515,7 @@ cudaError_t launch_gemv(const CUtensorMap& map_wq, const GemvArgs& a, const Gemv
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.ctas);
   cfg.blockDim = dim3(kGThreads);
-  cfg.dynamicSmemBytes = gemv_smem_bytes(p.stages, p.channels, p.mt, p.kpad);
+  cfg.dynamicSmemBytes = gemv_smem_bytes(p.stages, p.mt);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -163,6 +163,10 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
                     uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
                     uint32_t box_inner, uint32_t box_outer,
                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
+// 3-D map: dims[0] innermost; strides_bytes[i] is the byte stride of dims[i + 1].
+bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                    const uint64_t (&dims)[3], const uint64_t (&strides_bytes)[2],
+                    const uint32_t (&box)[3], CUtensorMapSwizzle swizzle);
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream, bool pdl);
 
 // GEMM tile shape (shared with the host for map boxes)
