@@ -128,7 +128,11 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4]
 
 // ------------------------------------------------------------------ activation quantization
 
+constexpr int kQMaxChunks = 256;  // chunks per CTA of the cluster: strip of 2048 columns
+
 struct FewQuantShared {
+  uint8_t flags[kQMaxChunks];    // outlier bits of this strip's chunks
+  int chunk_pos[kQMaxChunks];    // position of a chunk's first outlier in the list
   float red[kQThreads / 32][kSmallMP];
   float rowmax_local[kSmallMP];  // read by the other CTAs of the cluster
   int count_local;               // read by the other CTAs of the cluster
@@ -264,33 +268,61 @@ __global__ void __launch_bounds__(kQThreads) few_quant_kernel(const GemvArgs a) 
   }
   __syncthreads();
 
-  // ---- phase 2: int8 rows xq[i * kpad + k] (16 rows) and the compact outlier list
-  int pos = sh.base + my_off;
-  for (int c = t_begin; c < t_end; ++c) {
-    if (!one_chunk) load_chunk(c);
-    const uint32_t bits = one_chunk ? my_bits : chunk_flags();
-    const int k = c * 8;
-#pragma unroll
-    for (int i = 0; i < MT; ++i) {
+  // ---- phase 2: int8 rows xq[i * kpad + k] over (row, chunk) units, and the compact
+  // outlier list (chunk c's outliers start at chunk_pos[c])
+  if (one_chunk && t_begin < t_end) {
+    sh.flags[t_begin - c_begin] = static_cast<uint8_t>(my_bits);
+    sh.chunk_pos[t_begin - c_begin] = sh.base + my_off;
+  }
+  __syncthreads();
+  const int nch = c_end - c_begin;
+  if (one_chunk) {
+    for (int u = threadIdx.x; u < MT * nch; u += kQThreads) {
+      const int i = u / nch, cl = u % nch;
+      const int k = (c_begin + cl) * 8;
       uint2 q = make_uint2(0u, 0u);
-      if (!sh.zero_row[i] && k < K) q = quantize8(v[i], sh.sx[i], sh.rcp[i], bits);
+      if (!sh.zero_row[i] && k < K) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * K + k));
+        q = quantize8(x, sh.sx[i], sh.rcp[i], sh.flags[cl]);
+      }
       *reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(i) * a.kpad + k) = q;
     }
-    uint32_t b = bits;
-    while (b) {
-      const int e = __ffs(b) - 1;
-      b &= b - 1u;
-      a.cols[pos] = k + e;
-#pragma unroll
-      for (int i = 0; i < kSmallMP; ++i) {
-        unsigned short hb = 0;
-        if (i < MT && i < M) {
-          const uint32_t w[4] = {v[i % MT].x, v[i % MT].y, v[i % MT].z, v[i % MT].w};
-          hb = static_cast<unsigned short>((w[e / 2] >> (16 * (e & 1))) & 0xFFFFu);
-        }
-        a.xo[static_cast<size_t>(pos) * kSmallMP + i] = __ushort_as_half(hb);
+    for (int cl = threadIdx.x; cl < nch; cl += kQThreads) {
+      uint32_t b = sh.flags[cl];
+      int pos = sh.chunk_pos[cl];
+      const int k = (c_begin + cl) * 8;
+      while (b) {
+        const int e = __ffs(b) - 1;
+        b &= b - 1u;
+        a.cols[pos] = k + e;
+        for (int i = 0; i < kSmallMP; ++i)
+          a.xo[static_cast<size_t>(pos) * kSmallMP + i] =
+              (i < M) ? a.X[static_cast<size_t>(i) * K + k + e] : __float2half_rn(0.0f);
+        ++pos;
       }
-      ++pos;
+    }
+  } else {
+    int pos = sh.base + my_off;
+    for (int c = t_begin; c < t_end; ++c) {
+      load_chunk(c);
+      const uint32_t bits = chunk_flags();
+      const int k = c * 8;
+#pragma unroll
+      for (int i = 0; i < MT; ++i) {
+        uint2 q = make_uint2(0u, 0u);
+        if (!sh.zero_row[i] && k < K) q = quantize8(v[i], sh.sx[i], sh.rcp[i], bits);
+        *reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(i) * a.kpad + k) = q;
+      }
+      uint32_t b = bits;
+      while (b) {
+        const int e = __ffs(b) - 1;
+        b &= b - 1u;
+        a.cols[pos] = k + e;
+        for (int i = 0; i < kSmallMP; ++i)
+          a.xo[static_cast<size_t>(pos) * kSmallMP + i] =
+              (i < M) ? a.X[static_cast<size_t>(i) * K + k + e] : __float2half_rn(0.0f);
+        ++pos;
+      }
     }
   }
   cluster_sync_all();  // no CTA leaves while the others may still read its shared memory
@@ -298,10 +330,17 @@ __global__ void __launch_bounds__(kQThreads) few_quant_kernel(const GemvArgs a) 
 
 // ------------------------------------------------------------------ product
 
+constexpr int kMaxStagedOutliers = 256;  // outlier columns staged in shared memory
+
 struct GemvShared {
   uint64_t full[kMaxBoxes];
   uint64_t empty[kMaxBoxes];
   float sx[kSmallMP];
+  float wscale[kCh];
+  float bias[kCh];
+  int cols[kMaxStagedOutliers];
+  __half xo[kMaxStagedOutliers][kSmallMP];
+  int n_out;
   int abort;
   int issued;  // boxes whose copy was started
 };
@@ -368,9 +407,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
     for (int t = 0; t < NT; ++t)
 #pragma unroll
       for (int e = 0; e < 4; ++e) d[m][t][e] = 0;
+  // all of this warp's int8-X fragments in one batch of loads (L2), before any wait
+  constexpr int kMaxSteps = 16;  // k32 steps per warp: K <= 16 warps x 16 x 32 = 8192
+  uint32_t bfr[kMaxSteps][NT][2];
+#pragma unroll
+  for (int u = 0; u < kMaxSteps; ++u)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      bfr[u][t][0] = bfr[u][t][1] = 0u;
+      if (s_begin + u < s_end) {
+        const int8_t* xrow = a.xq + static_cast<size_t>(t * 8 + g) * a.kpad + (s_begin + u) * 32 + 4 * tig;
+        bfr[u][t][0] = __ldcg(reinterpret_cast<const unsigned int*>(xrow));
+        bfr[u][t][1] = __ldcg(reinterpret_cast<const unsigned int*>(xrow + 16));
+      }
+    }
   bool ok = true;
   int waited_box = -1;
-  for (int st = s_begin; st < s_end; ++st) {
+#pragma unroll
+  for (int u = 0; u < kMaxSteps; ++u) {
+    const int st = s_begin + u;
+    if (st >= s_end) break;
     const int k0 = st * 32;
     const int box = k0 / (kBoxKb * 128);
     if (box != waited_box) {  // boxes are consumed in order; R >= boxes here (resident)
@@ -388,13 +444,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const uint8_t* tile = ring + static_cast<size_t>(box % R) * kBoxBytes +
                           ((k0 / 128) % kBoxKb) * (kCh * 128);
     const int kk = k0 % 128 + 4 * tig;
-    uint32_t b[NT][2];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const int8_t* xrow = a.xq + static_cast<size_t>(t * 8 + g) * a.kpad + k0 + 4 * tig;
-      b[t][0] = __ldcg(reinterpret_cast<const unsigned int*>(xrow));
-      b[t][1] = __ldcg(reinterpret_cast<const unsigned int*>(xrow + 16));
-    }
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       uint32_t af[4];
@@ -403,7 +452,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       af[2] = *reinterpret_cast<const uint32_t*>(tile + sw128_offset(m * 16 + g, kk + 16));
       af[3] = *reinterpret_cast<const uint32_t*>(tile + sw128_offset(m * 16 + g + 8, kk + 16));
 #pragma unroll
-      for (int t = 0; t < NT; ++t) mma_s8_16832(d[m][t], af, b[t][0], b[t][1]);
+      for (int t = 0; t < NT; ++t) mma_s8_16832(d[m][t], af, bfr[u][t][0], bfr[u][t][1]);
     }
   }
   if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
@@ -419,10 +468,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
       rw[(m * 16 + g + 8) * MT + t * 8 + 2 * tig + 1] = d[m][t][3];
     }
   if (threadIdx.x < kSmallMP) sh.sx[threadIdx.x] = __ldcg(a.sx + threadIdx.x);
+  if (threadIdx.x < kCh) {
+    const int n = n0 + threadIdx.x;
+    sh.wscale[threadIdx.x] = n < a.N ? a.w_scale[n] : 0.0f;
+    sh.bias[threadIdx.x] = (a.bias && n < a.N) ? __half2float(a.bias[n]) : 0.0f;
+  }
+  const int n_out = __ldcg(a.n_out);
+  const int staged = n_out < kMaxStagedOutliers ? n_out : kMaxStagedOutliers;
+  for (int t = threadIdx.x; t < staged * (kSmallMP + 1); t += kGThreads) {
+    const int o = t / (kSmallMP + 1), i = t % (kSmallMP + 1);
+    if (i == kSmallMP) sh.cols[o] = __ldcg(a.cols + o);
+    else sh.xo[o][i] = a.xo[static_cast<size_t>(o) * kSmallMP + i];
+  }
   __syncthreads();
 
   // ---- thread (c, i): sum the warps, add the outlier term and bias, write Y[i, n0 + c]
-  const int n_out = __ldcg(a.n_out);
   const bool resident = nbox <= R;
   for (int t = threadIdx.x; t < kCh * MT; t += kGThreads) {
     const int c = t % kCh, i = t / kCh, n = n0 + c;
@@ -430,10 +490,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     int32_t acc = 0;
 #pragma unroll
     for (int w = 0; w < kGWarps; ++w) acc += red[(static_cast<size_t>(w) * kCh + c) * MT + i];
-    const float swn = a.w_scale[n];
+    const float swn = sh.wscale[c];
     float P = 0.0f;
     for (int o = 0; o < n_out; ++o) {
-      const int j = __ldcg(a.cols + o);
+      const int j = o < staged ? sh.cols[o] : __ldcg(a.cols + o);
       int8_t q;
       if (resident) {
         const int kb = j / 128;
@@ -444,9 +504,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
         q = a.Wq[static_cast<size_t>(n) * a.K + j];
       }
       const float wv = __half2float(__float2half_rn(static_cast<float>(q) * swn));
-      P += wv * __half2float(a.xo[static_cast<size_t>(o) * kSmallMP + i]);
+      P += wv * __half2float(o < staged ? sh.xo[o][i] : a.xo[static_cast<size_t>(o) * kSmallMP + i]);
     }
-    const float bb = a.bias ? __half2float(a.bias[n]) : 0.0f;
+    const float bb = sh.bias[c];
     const float y = static_cast<float>(acc) * sh.sx[i] * swn + P + bb;
     a.Y[static_cast<size_t>(i) * a.N + n] = __float2half_rn(y);
     if (a.acc) a.acc[static_cast<size_t>(i) * a.N + n] = ok ? acc : 0;
@@ -474,8 +534,9 @@ GemvPlan plan_gemv(int M, int N, int K, int num_sms) {
   const int chunks = p.kpad / 8;
   int Q = (chunks + 63) / 64;  // about 64 chunks (512 columns) per CTA of the cluster
   p.quant_ctas = Q < 1 ? 1 : (Q > kQMaxCtas ? kQMaxCtas : Q);
-  p.fits = M <= kSmallMP && K % 128 == 0 && nbox <= kMaxBoxes &&
-           gemv_smem_bytes(nbox, p.mt) <= kSmemLimit;
+  const int chunks_per_cta = (chunks + p.quant_ctas - 1) / p.quant_ctas;
+  p.fits = M <= kSmallMP && K % 128 == 0 && K <= kGWarps * 16 * 32 && nbox <= kMaxBoxes &&
+           chunks_per_cta <= 256 && gemv_smem_bytes(nbox, p.mt) <= kSmemLimit;
   return p;
 }
 
