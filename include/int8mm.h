@@ -10,7 +10,8 @@
  *   - Matrices are row-major with K (the input-feature axis) contiguous.
  *   - Half-precision data is IEEE binary16 (passed as void*; the ABI has no half type).
  *   - Every pointer is a caller-owned DEVICE pointer on the current CUDA device, unless
- *     stated otherwise; the library allocates nothing and keeps no state between calls.
+ *     stated otherwise; the library allocates nothing and keeps no state between calls
+ *     (except the static scratch of int8_linear_forward_noalloc, described there).
  *     Matrix and vector pointers must be 16-byte aligned.
  *   - K must be a multiple of 16 (each row must start on a 16-byte boundary for the
  *     tensor-memory-access unit); 1 <= M, N and K <= INT8MM_MAX_K.
@@ -45,6 +46,10 @@ typedef struct CUstream_st *int8mm_stream_t; /* the same type as cudaStream_t */
 #define INT8MM_ERR_DEVICE (-7)       /* the current device is not sm_100 */
 #define INT8MM_ERR_TIMEOUT (-8)      /* device side: a bounded wait gave up */
 #define INT8MM_ERR_OVERFLOW (-9)     /* device side: an outlier count beyond K */
+#define INT8MM_ERR_SCRATCH (-10)     /* shape beyond int8_linear_forward_noalloc's scratch */
+
+/* Bytes of the static device scratch behind int8_linear_forward_noalloc (per device). */
+#define INT8MM_NOALLOC_SCRATCH_BYTES (512 * 1024)
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *int8_status_string(int status);
@@ -163,6 +168,30 @@ int int8_gemm_i32(const int8_t *Xq, const int8_t *Wq, int M, int N, int K, int32
 int int8_outlier_weights(const int8_t *Wq, const float *w_scale, int N, int K,
                          const int32_t *outlier_cols, const int32_t *n_outliers, void *W_hat,
                          int8mm_stream_t stream);
+
+/*
+ * int8_linear_forward without a workspace argument, for few-token (decode) shapes.
+ * The pages have no counterpart: this is a calling convention, not part of the method.
+ * It serves callers that cannot allocate device memory where they call the layer -- a
+ * stream being captured into a graph, an allocator that must not grow mid-step, or a C
+ * host that has no way to hand over a workspace -- so it allocates nothing and calls no
+ * allocating routine.  Its scratch (outlier list, int8 and outlier activations, row
+ * scales) is a static device array of INT8MM_NOALLOC_SCRATCH_BYTES that every GPU which
+ * loads the library holds until the process exits.
+ *   X, Wq, w_scale, bias, threshold, Y   as for int8_linear_forward (same kernels, same bits)
+ *   dev_status [in/out] one int32 of device memory that receives a negative code if a
+ *              bounded device-side wait gives up (zero it first), or NULL to not be told
+ * Limits: M <= 16, and a shape the few-token kernels take (K <= 8192 with K % 128 == 0, or
+ * the single-kernel cluster path); anything else returns INT8MM_ERR_SCRATCH at once.
+ * The first call on each device looks up that device's copy of the array (with the device
+ * current); make that first call before any stream capture begins.
+ * Every call on a device shares the one array and leaves its contents behind (nothing in
+ * it needs to start at zero), so calls that overlap on the GPU -- on two streams, or from
+ * two threads -- race and give wrong results; order them on one stream.
+ */
+int int8_linear_forward_noalloc(const void *X, int M, int K, const int8_t *Wq,
+                                const float *w_scale, const void *bias, int N, float threshold,
+                                void *Y, int32_t *dev_status, int8mm_stream_t stream);
 
 /*
  * Waits for `stream`, then returns the device status word at dev_status (for the forward

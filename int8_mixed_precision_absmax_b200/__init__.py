@@ -8,7 +8,7 @@ built, importing the binding's functions raises.
 Functions keep the C names:
     int8_quant_weight, int8_linear_workspace_size, int8_linear_forward,
     int8_quantize_rows, int8_gemm_i32, int8_outlier_weights, int8_read_device_status,
-    int8_status_string
+    int8_status_string, int8_linear_forward_noalloc
 and ``Int8Linear`` bundles them the way the pages use the layer
 (``Linear8bitLt(in, out, bias, has_fp16_weights=False, threshold=6.0)``).
 """
@@ -26,7 +26,8 @@ __all__ = [
     "int8_quant_weight", "int8_linear_workspace_size", "int8_linear_forward",
     "int8_linear_quantize", "int8_linear_matmul", "int8_linear_forward_acc",
     "int8_quantize_rows", "int8_gemm_i32", "int8_outlier_weights",
-    "int8_read_device_status", "int8_status_string", "Int8Linear", "DEFAULT_THRESHOLD",
+    "int8_read_device_status", "int8_status_string", "int8_linear_forward_noalloc",
+    "Int8Linear", "DEFAULT_THRESHOLD",
 ]
 
 DEFAULT_THRESHOLD = 6.0
@@ -70,9 +71,11 @@ def load_library():
         lib.int8_gemm_i32.argtypes = [p, p, i, i, i, p, p, p]
         lib.int8_outlier_weights.argtypes = [p, p, i, i, p, p, p, p]
         lib.int8_read_device_status.argtypes = [p, p]
+        lib.int8_linear_forward_noalloc.argtypes = [p, i, i, p, p, p, i, f, p, p, p]
         for name in ("int8_quant_weight", "int8_linear_forward", "int8_linear_quantize",
                      "int8_linear_matmul", "int8_linear_forward_acc", "int8_quantize_rows",
-                     "int8_gemm_i32", "int8_outlier_weights", "int8_read_device_status"):
+                     "int8_gemm_i32", "int8_outlier_weights", "int8_read_device_status",
+                     "int8_linear_forward_noalloc"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -161,6 +164,33 @@ def int8_linear_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor
         _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(bias), N, float(threshold), _ptr(Y),
         _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream, X.device))),
         "int8_linear_forward")
+    return Y
+
+
+def int8_linear_forward_noalloc(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                                bias: torch.Tensor | None, threshold: float, Y: torch.Tensor,
+                                dev_status: torch.Tensor | None = None,
+                                stream=None) -> torch.Tensor:
+    """int8_linear_forward for M <= 16 with no workspace argument.
+
+    For callers that cannot allocate device memory where they run the layer (a stream being
+    captured, an allocator that must not grow): the library keeps the scratch in a static
+    device array, so nothing here allocates -- Y (and dev_status, an optional int32 that
+    receives a device-side failure code) come from the caller.  Calls that overlap on the
+    GPU share that array and race; keep them on one stream."""
+    _need(X, torch.float16, "X", 2)
+    _need(Wq, torch.int8, "Wq", 2)
+    _need(w_scale, torch.float32, "w_scale", 1)
+    _need(Y, torch.float16, "Y", 2)
+    if bias is not None:
+        _need(bias, torch.float16, "bias", 1)
+    if dev_status is not None:
+        _need(dev_status, torch.int32, "dev_status", 1)
+    M, K = X.shape
+    _check(load_library().int8_linear_forward_noalloc(
+        _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(bias), Wq.shape[0], float(threshold),
+        _ptr(Y), _ptr(dev_status), ctypes.c_void_p(_stream(stream, X.device))),
+        "int8_linear_forward_noalloc")
     return Y
 
 

@@ -3,6 +3,7 @@
 // point allocates memory or synchronizes, except int8_read_device_status (documented).
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "kernels.cuh"
 
@@ -78,6 +79,8 @@ const char* int8_status_string(int status) {
     case INT8MM_ERR_DEVICE: return "the current device is not sm_100";
     case INT8MM_ERR_TIMEOUT: return "a bounded device-side wait gave up";
     case INT8MM_ERR_OVERFLOW: return "outlier count out of range";
+    case INT8MM_ERR_SCRATCH:
+      return "the shape needs more scratch than the library's static buffer holds";
     default: return "unknown status";
   }
 }
@@ -399,6 +402,114 @@ int int8_read_device_status(const int32_t* dev_status, int8mm_stream_t stream) {
   if (cudaMemcpy(&v, dev_status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
     return INT8MM_ERR_CUDA;
   return v;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- no-alloc forward
+//
+// int8_linear_forward_noalloc serves callers that cannot allocate device memory at the
+// point of the call -- code running while a stream is being captured, under an allocator
+// that must not grow, or behind a C interface with no workspace argument.  Its scratch (the
+// few-token kernels' outlier list, int8 activations, outlier activations and row scales)
+// lives in one file-scope device array that every GPU loading the library holds until exit.
+// Every call on a device shares it and it keeps the last call's contents.
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[INT8MM_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoallocMaxDevices];
+
+// Device address of this device's copy of g_noalloc_scratch, looked up once per device with
+// that device current (the host-side name is only a handle for the runtime).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return INT8MM_ERR_CUDA;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return INT8MM_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();
+      return INT8MM_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return INT8MM_OK;
+}
+
+// The few-token kernels' regions, carved from the scratch: status header, outlier list,
+// 16-row int8 activations, outlier activations, row scales (the same regions and sizes as
+// the few-token part of workspace_layout; the other regions are not used on this path).
+WorkspaceLayout noalloc_layout(int K) {
+  WorkspaceLayout L = {};
+  L.ldo = (K + 63) / 64 * 64;
+  const size_t kpad = static_cast<size_t>((K + 255) / 256) * 256;
+  size_t off = 0;
+  L.header = off;  off = align256(off + 64 * sizeof(int32_t));
+  L.cols = off;    off = align256(off + static_cast<size_t>(K) * sizeof(int32_t));
+  L.few_xq = off;  off = align256(off + kSmallMP * kpad);
+  L.few_xo = off;  off = align256(off + static_cast<size_t>(K) * kSmallMP * sizeof(__half));
+  L.few_sx = off;  off = align256(off + kSmallMP * sizeof(float));
+  L.mask = L.xscale = L.xq = L.xo = L.wo = L.header;
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+int int8_linear_forward_noalloc(const void* X, int M, int K, const int8_t* Wq,
+                                const float* w_scale, const void* bias, int N, float threshold,
+                                void* Y, int32_t* dev_status, int8mm_stream_t stream_) {
+  if (!X || !Y || !Wq || !w_scale) return INT8MM_ERR_NULL;
+  int rc = check_shape(M, N, K);
+  if (rc) return rc;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(Wq) || !aligned16(w_scale) ||
+      (bias && !aligned16(bias)) || (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)))
+    return INT8MM_ERR_ALIGN;
+  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
+  if (M > kSmallMP) return INT8MM_ERR_SCRATCH;
+  if ((rc = check_device())) return rc;
+  const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
+  const bool small = !gp.fits && small_path_fits(M, K);
+  if (!gp.fits && !small) return INT8MM_ERR_SCRATCH;
+  const WorkspaceLayout L = noalloc_layout(K);
+  if (L.total > INT8MM_NOALLOC_SCRATCH_BYTES) return INT8MM_ERR_SCRATCH;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  ForwardPlan p = {};
+  p.L = L;
+  p.header = at<int32_t>(scratch, L.header);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  // Nothing in the scratch has to start at zero: the quantization kernel writes the outlier
+  // count, list and activations before the product kernel reads them, and the status goes to
+  // the caller's word (or nowhere).
+  if (small) {
+    const SmallPlan sp = plan_small(M, N, K);
+    SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, p, sp);
+    a.status = dev_status;
+    CUtensorMap map;
+    if (!encode_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kSmallBN))
+      return INT8MM_ERR_CUDA;
+    return launch_status(launch_small(map, a, sp, stream, true));
+  }
+  GemvArgs g = gemv_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, scratch, p, gp);
+  g.status = dev_status;
+  CUtensorMap map;
+  const uint64_t dims[3] = {128, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 128)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(K), 128};
+  const uint32_t box[3] = {128, static_cast<uint32_t>(gp.channels), 8};
+  if (!encode_tmap_3d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return INT8MM_ERR_CUDA;
+  if ((rc = launch_status(launch_few_quant(g, gp, stream, true)))) return rc;
+  return launch_status(launch_gemv(map, g, gp, stream, true));
 }
 
 }  // extern "C"
