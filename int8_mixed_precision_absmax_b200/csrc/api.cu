@@ -180,10 +180,41 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
   return a;
 }
 
+// The one-launch few-token layer: Wq viewed as [K/128 k-blocks][N rows][128 bytes], one box
+// is 16 rows x (a slice of) k-blocks, each k-block landing as a 128-byte-swizzled 16 x 128
+// tile.
+int run_decode(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+               const void* bias, int N, float threshold, void* Y, int32_t* acc, int32_t* status,
+               const DecodePlan& dp, cudaStream_t stream, bool pdl) {
+  CUtensorMap map;
+  const uint64_t dims[3] = {128, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 128)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(K), 128};
+  const uint32_t box[3] = {128, static_cast<uint32_t>(dp.tile_rows),
+                           static_cast<uint32_t>(dp.nqmax)};
+  if (!encode_tmap_3d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return INT8MM_ERR_CUDA;
+  DecodeArgs a;
+  a.X = static_cast<const __half*>(X);
+  a.M = M;
+  a.K = K;
+  a.N = N;
+  a.threshold = effective_threshold(threshold);
+  a.Wq = Wq;
+  a.w_scale = w_scale;
+  a.bias = static_cast<const __half*>(bias);
+  a.Y = static_cast<__half*>(Y);
+  a.acc = acc;
+  a.nqmax = dp.nqmax;
+  a.status = status;
+  return launch_status(launch_decode(map, a, dp, stream, pdl));
+}
+
 int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale, int N,
                  float threshold, void* workspace, const ForwardPlan& p, cudaStream_t stream,
                  bool pdl_first) {
   if (M <= kSmallMP) {
+    if (plan_decode(M, N, K).fits) return INT8MM_OK;  // one kernel does everything
     const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
     if (gp.fits) {
       const GemvArgs g = gemv_args(X, M, K, Wq, w_scale, nullptr, N, threshold, nullptr, nullptr,
@@ -219,6 +250,10 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
                const void* bias, int N, float threshold, void* Y, int32_t* acc,
                void* workspace, const ForwardPlan& p, cudaStream_t stream, bool pdl) {
   if (M <= kSmallMP) {
+    const DecodePlan dp = plan_decode(M, N, K);
+    if (dp.fits)
+      return run_decode(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p.header, dp, stream,
+                        pdl);
     const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
     if (gp.fits) {
       const GemvArgs g = gemv_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace,
@@ -476,17 +511,21 @@ int int8_linear_forward_noalloc(const void* X, int M, int K, const int8_t* Wq,
   if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
   if (M > kSmallMP) return INT8MM_ERR_SCRATCH;
   if ((rc = check_device())) return rc;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const DecodePlan dp = plan_decode(M, N, K);
+  if (dp.fits)  // the one-launch kernel needs no scratch
+    return run_decode(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, dev_status, dp,
+                      stream, true);
   const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
   const bool small = !gp.fits && small_path_fits(M, K);
   if (!gp.fits && !small) return INT8MM_ERR_SCRATCH;
   const WorkspaceLayout L = noalloc_layout(K);
   if (L.total > INT8MM_NOALLOC_SCRATCH_BYTES) return INT8MM_ERR_SCRATCH;
-  void* scratch = nullptr;
-  if ((rc = noalloc_scratch(&scratch))) return rc;
   ForwardPlan p = {};
   p.L = L;
   p.header = at<int32_t>(scratch, L.header);
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   // Nothing in the scratch has to start at zero: the quantization kernel writes the outlier
   // count, list and activations before the product kernel reads them, and the status goes to
   // the caller's word (or nowhere).

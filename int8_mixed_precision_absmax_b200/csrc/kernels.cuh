@@ -145,6 +145,31 @@ cudaError_t launch_gemv(const CUtensorMap& map_wq, const GemvArgs& a, const Gemv
                         cudaStream_t stream, bool pdl);
 int device_sm_count();
 
+// One-launch layer for M <= 8 tokens (decode.cu): no workspace.
+struct DecodeArgs {
+  const __half* X;
+  int M, K, N;
+  float threshold;       // already clamped to >= 0
+  const int8_t* Wq;
+  const float* w_scale;
+  const __half* bias;
+  __half* Y;
+  int32_t* acc;          // nullable: also write the int32 accumulators
+  int nqmax;             // k-blocks of the largest slice of K (one slice per CTA of a cluster)
+  int32_t* status;
+};
+struct DecodePlan {
+  int cluster;           // CTAs per cluster = slices of K
+  int wpm;               // pairs of 16-channel tiles per CTA (the kernel's P)
+  int tile_rows;         // rows of Wq per TMA box
+  int ctas, nqmax;
+  size_t smem;
+  bool fits;
+};
+DecodePlan plan_decode(int M, int N, int K);
+cudaError_t launch_decode(const CUtensorMap& map_wq, const DecodeArgs& a, const DecodePlan& p,
+                          cudaStream_t stream, bool pdl);
+
 struct GemmArgs {
   int M, N, K;
   const float* xscale;   // [M]

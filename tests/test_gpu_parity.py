@@ -237,6 +237,15 @@ def check_forward_acc(X, W, b, t, rows=None):
     (9, 4096, 4100, 5, 6.0),    # channels not a multiple of the per-CTA share
     (17, 512, 300, 3, 6.0),     # one row past the few-token path
     (200, 1040, 600, 5, 6.0),   # the tiled path
+    # the one-launch decode kernel (M <= 8, K % 128 == 0, K <= 8192)
+    (8, 128, 64, 1, 6.0),       # one k-block: a single slice of the cluster holds X
+    (2, 8192, 512, 4, 6.0),     # longest rows: two-box ring, refilled six times
+    (6, 3072, 1000, 3, 6.0),    # three boxes, channels not a multiple of 32
+    (8, 2176, 96, 2, 6.0),      # 17 k-blocks over 8 slices; most CTAs past N
+    (5, 4096, 256, 40, 6.0),    # many outlier columns
+    (8, 1024, 1024, 0, 0.0),    # every column an outlier: the fp16 term everywhere
+    (4, 512, 96, 0, math.inf),  # no outlier term at all
+    (8, 6144, 300, 2, 6.0),     # six boxes through a two-box ring
 ])
 def test_forward_accumulators_and_y(M, K, N, n_out, t):
     X, W, b = random_case(M, K, N, n_out, seed=M + 3 * K + 7 * N)
