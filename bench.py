@@ -214,21 +214,27 @@ def oracle_sample_rate(w, X, W_q, sw, bias, budget_s: float):
             n_cols = min(w.N, int(n_cols * grow))
         else:
             n_rows = min(w.M, int(n_rows * grow))
-    # one final evaluation sized to the budget
+    # one final evaluation sized to the budget; a problem the oracle finishes well inside it
+    # is evaluated repeatedly
     scale = max(1.0, budget_s / max(t, 1e-6))
     if n_cols < w.N:
         n_cols = min(w.N, int(n_cols * scale))
     elif n_rows < w.M:
         n_rows = min(w.M, int(n_rows * scale))
     rows = rows_all[np.linspace(0, w.M - 1, n_rows).astype(np.int64)] if n_rows < w.M else rows_all
+    passes = 0
     t0 = time.perf_counter()
-    oracle.linear_forward_rows(X, W_q[:n_cols], sw[:n_cols], None if bias is None else bias[:n_cols],
-                               w.threshold, rows)
-    t = time.perf_counter() - t0
-    ops = 2.0 * len(rows) * n_cols * w.K
+    while True:
+        oracle.linear_forward_rows(X, W_q[:n_cols], sw[:n_cols],
+                                   None if bias is None else bias[:n_cols], w.threshold, rows)
+        passes += 1
+        t = time.perf_counter() - t0
+        if t >= budget_s * 0.8 or n_rows < w.M or n_cols < w.N:
+            break
+    ops = 2.0 * len(rows) * n_cols * w.K * passes
     threads = min(os.cpu_count() or 1, len(rows))
     desc = (f"{len(rows)} of {w.M} rows x {n_cols} of {w.N} output channels "
-            f"(K={w.K}, outlier set over all rows), one pass")
+            f"(K={w.K}, outlier set over all rows), {passes} pass(es)")
     return ops / t / 1e12, t, desc, threads, (len(rows), n_cols)
 
 
@@ -277,6 +283,52 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- our arm
+
+def forward_path(M: int, N: int, K: int):
+    """Which kernels one int8_linear_forward launches for this shape (the library's dispatch:
+    api.cu with the plan functions of decode.cu, gemv.cu and small.cu)."""
+    if M <= 8 and K % 128 == 0 and K <= 8192:
+        return {"name": "decode", "launches": 1, "quantize": [],
+                "matmul": "decode_kernel (one launch: 8-CTA cluster per 128 channels, split-K, "
+                          "mma.sync int8 + fp16 outlier term, partial sums through DSMEM)"}
+    if M <= 16:
+        if K % 128 == 0 and K <= 8192:
+            return {"name": "few_tokens", "launches": 2, "quantize": ["few_quant_kernel"],
+                    "matmul": "gemv_kernel (mma.sync int8 + fp16 outlier term)"}
+        return {"name": "cluster", "launches": 1, "quantize": [],
+                "matmul": "small_fused_kernel (tcgen05, one cluster per channel tile)"}
+    return {"name": "tiled", "launches": 3, "quantize": ["colmask_kernel", "rowquant_kernel"],
+            "matmul": "gemm_kernel (int8 + fp16 tcgen05, fused epilogue)"}
+
+
+def graph_time_ms(fn, n: int, device) -> float:
+    """Average device time of fn() replayed back to back from one CUDA graph of n calls."""
+    import torch
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(side):
+        for i in range(n):
+            fn(i)
+    torch.cuda.current_stream(device).wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            fn(i)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (reps * n)
+    del g
+    return ms
+
 
 def run_ours(args):
     import numpy as np
@@ -402,21 +454,23 @@ def run_ours(args):
     value = whole_job_rate(w.ops, steps, world, max_s) / 1e12
     gbs = whole_job_rate(step_bytes, steps, world, max_s) / 1e9
 
-    # ---- per-kernel durations, live, with events on the launching stream
-    n_k = max(20, min(steps, 200))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-            torch.cuda.Event(enable_timing=True)) for _ in range(n_k)]
-    for i in range(n_k):
-        c = i % copies
-        a, m, z = evs[i]
-        a.record()
-        i8.int8_linear_quantize(Xs[c], Wqs[c], sws[c], w.threshold, wss[c])
-        m.record()
-        i8.int8_linear_matmul(Xs[c], Wqs[c], sws[c], bs[c], w.threshold, Ys[c], wss[c])
-        z.record()
+    # ---- per-kernel durations, live: the activation side and the product, each replayed
+    # back to back from its own CUDA graph over the rotating copies (CUDA events around the
+    # replays, on the launching stream); the product reads what earlier steps left in each
+    # copy's workspace
+    path = forward_path(w.M, w.N, w.K)
+    if path["quantize"]:
+        q_ms = graph_time_ms(lambda i: i8.int8_linear_quantize(
+            Xs[i % copies], Wqs[i % copies], sws[i % copies], w.threshold, wss[i % copies]),
+            max(copies, 32), device)
+    else:
+        q_ms = 0.0
+    g_ms = graph_time_ms(lambda i: i8.int8_linear_matmul(
+        Xs[i % copies], Wqs[i % copies], sws[i % copies], bs[i % copies], w.threshold,
+        Ys[i % copies], wss[i % copies]), max(copies, 32), device)
+    for c in range(copies):  # leave every copy's Y from a complete forward
+        step(c)
     torch.cuda.synchronize()
-    q_ms = statistics.mean(a.elapsed_time(m) for a, m, _ in evs)
-    g_ms = statistics.mean(m.elapsed_time(z) for _, m, z in evs)
 
     peaks = load_peaks()
     tensor_bound = w.ops / step_bytes > (peaks["bf16_tflops"] * INT8_OVER_BF16 * 1e12) / (peaks["hbm_gbs"] * 1e9)
@@ -424,9 +478,7 @@ def run_ours(args):
     n_out = int(i8.int8_quantize_rows(Xs[0], w.threshold)[3].item())
     pad = (n_out + 63) // 64 * 64 if n_out else 0
     few_tokens = w.M <= 16
-    kernel = ("gemv_kernel (one launch per step: weight slice streamed by TMA into shared "
-              "memory while X is quantized, exact dp4a int8 products, fused epilogue)"
-              if few_tokens else "gemm_kernel (int8 + fp16 tcgen05, fused epilogue)")
+    kernel = path["matmul"]
     if few_tokens:  # reads X (fp16) and Wq, writes Y
         gemm_bytes = (2 * w.M * w.K + w.N * w.K + 4 * w.N + 2 * w.M * w.N
                       + (2 * w.N if b_h is not None else 0))
@@ -494,9 +546,10 @@ def run_ours(args):
                        "l2": f"{copies} rotating copies of X, Wq, w_scale, Y and workspace "
                              f"({copies * step_bytes / 2**20:.0f} MiB of operands > 2 x L2)",
                        "launch": "CUDA graph replay" if use_graph else "direct launches",
+                       "path": path["name"],
                        "parallelism": f"{world} independent replica(s), one per GPU"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": (1 if few_tokens else 3) * steps,
+            "gpu_launches": path["launches"] * steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

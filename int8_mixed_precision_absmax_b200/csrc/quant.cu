@@ -48,6 +48,46 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return v;
 }
 
+// 8 halves -> 8 int8 codes q = rne(x / s) of a row whose regular columns satisfy
+// |x| <= absmax = 127 s, packed little-endian, outlier columns (bits) set to 0.
+// With r = 1/s rounded to nearest, the exact x * r is within 2^-17 of x / s (|x / s| <= 128)
+// and the rounded quotient within 2^-18, so rne(x * r) = rne(fl(x / s)) unless x * r lies
+// within 2^-15 of a half-integer; there the quotient itself (__fdiv_rn) is rounded.  rne(x * r)
+// comes from one fused multiply-add with 1.5 * 2^23, whose low bits then hold the integer;
+// |x / s| <= 127 (1 + 2^-22) on regular columns, so the code needs no clamp.
+__device__ __forceinline__ uint32_t keep_mask(uint32_t bits4) {  // bit e set -> byte e = 0
+  return ~(((bits4 * 0x204081u) & 0x01010101u) * 0xFFu);
+}
+__device__ __forceinline__ uint2 quantize_chunk_fast(const uint4& v, float s, float rcp,
+                                                     uint32_t bits) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float x[8];
+  int qv[8];
+  uint32_t near_tie = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    if ((e & 1) == 0) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e / 2]));
+      x[e] = f.x;
+      x[e + 1] = f.y;
+    }
+    const float tb = __fmaf_rn(x[e], rcp, kRound);
+    qv[e] = __float_as_int(tb) - 0x4B400000;
+    const float d = fabsf(__fmaf_rn(x[e], rcp, -(tb - kRound)));
+    near_tie |= (fabsf(d - 0.5f) <= 0x1p-15f ? 1u : 0u) << e;
+  }
+  near_tie &= ~bits;
+  if (near_tie) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if ((near_tie >> e) & 1u) qv[e] = __float2int_rn(__fdiv_rn(x[e], s));
+  }
+  const uint32_t lo = __byte_perm(__byte_perm(qv[0], qv[1], 0x0040), __byte_perm(qv[2], qv[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(qv[4], qv[5], 0x0040), __byte_perm(qv[6], qv[7], 0x0040), 0x5410);
+  return make_uint2(lo & keep_mask(bits & 0xFu), hi & keep_mask(bits >> 4));
+}
+
 // 8 halves (one 16-byte chunk) -> 8 int8 codes packed little-endian into 8 bytes.
 __device__ __forceinline__ uint2 quantize_chunk(uint4 v, float s, bool zero_all,
                                                 uint32_t outlier_bits) {
@@ -102,83 +142,98 @@ cudaError_t launch_quant_weight(const __half* W, int N, int K, int8_t* Wq, float
 
 // ------------------------------------------------------------------ outlier columns
 //
-// One block owns 32 consecutive columns (one mask word) for all M rows, so no two blocks
-// write the same word and the mask needs no atomics and no prior clearing.  Thread
-// (r, g) = (tid / 4, tid % 4) reads the 16-byte chunk of columns [32b + 8g, +8) of rows
-// r, r + 64, ...; the per-column maxima are then reduced across the 64 row lanes.
+// Block (strip, rb) takes columns [64 strip, +64) of rows [256 rb, +256): thread (r, c) =
+// (tid / 8, tid % 8) reads the 16-byte chunk c of the strip in rows 256 rb + r + 32 u,
+// u = 0..7, all eight loads in flight.  The block's column maxima (fp16, exact) go to
+// pmax[rb][column]; the last block of the strip to arrive (counted in strip[s], which it
+// sets back to zero) takes the maximum over the row blocks and writes the strip's two mask
+// words.  No two blocks write the same word, so the mask needs no clearing.
 
 constexpr int kCMThreads = 256;
-constexpr int kCMRowLanes = kCMThreads / 4;
-constexpr int kCMUnroll = 8;
+constexpr int kCMRowLanes = kCMThreads / 8;           // 32
+constexpr int kCMUnroll = kColRowBlock / kCMRowLanes;  // 8
 
 __global__ void __launch_bounds__(kCMThreads) colmask_kernel(const __half* __restrict__ X, int M,
                                                              int K, float threshold,
-                                                             uint32_t* __restrict__ mask) {
-  __shared__ __half2 red[kCMThreads / 32][4][4];
+                                                             uint32_t* __restrict__ mask,
+                                                             __half* __restrict__ pmax,
+                                                             int32_t* __restrict__ strip_cnt) {
+  __shared__ __half2 red[kCMThreads / 32][8][4];
+  __shared__ int last;
   grid_dependency_wait();
-  const int g = threadIdx.x & 3, r = threadIdx.x >> 2;
-  const int col0 = blockIdx.x * 32 + g * 8;
+  const int strip = blockIdx.x, rb = blockIdx.y, nrb = gridDim.y;
+  const int c = threadIdx.x & 7, r = threadIdx.x >> 3;
+  const int col0 = strip * kColStrip + c * 8;
   __half2 m[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) m[e] = __float2half2_rn(0.0f);
   if (col0 < K) {  // K % 8 == 0: a chunk is entirely inside or outside the matrix
-    const __half* base = X + col0;
-    int i = r;
-    for (; i + (kCMUnroll - 1) * kCMRowLanes < M; i += kCMUnroll * kCMRowLanes) {
-      uint4 v[kCMUnroll];
+    uint4 v[kCMUnroll];
 #pragma unroll
-      for (int u = 0; u < kCMUnroll; ++u)
-        v[u] = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(i + u * kCMRowLanes) * K));
-#pragma unroll
-      for (int u = 0; u < kCMUnroll; ++u) {
-        m[0] = habs2_max(m[0], v[u].x);
-        m[1] = habs2_max(m[1], v[u].y);
-        m[2] = habs2_max(m[2], v[u].z);
-        m[3] = habs2_max(m[3], v[u].w);
-      }
+    for (int u = 0; u < kCMUnroll; ++u) {
+      const int i = rb * kColRowBlock + r + u * kCMRowLanes;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < M) v[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(i) * K + col0));
     }
-    for (; i < M; i += kCMRowLanes) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(i) * K));
-      m[0] = habs2_max(m[0], v.x);
-      m[1] = habs2_max(m[1], v.y);
-      m[2] = habs2_max(m[2], v.z);
-      m[3] = habs2_max(m[3], v.w);
+#pragma unroll
+    for (int u = 0; u < kCMUnroll; ++u) {
+      m[0] = habs2_max(m[0], v[u].x);
+      m[1] = habs2_max(m[1], v[u].y);
+      m[2] = habs2_max(m[2], v[u].z);
+      m[3] = habs2_max(m[3], v[u].w);
     }
   }
   grid_launch_dependents();
-  // reduce over the 8 row lanes inside the warp (lanes with equal g), then across warps
+  // reduce over the 4 row lanes of the warp (lanes with equal c), then across warps
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      const __half2 other = __shfl_xor_sync(0xffffffffu, m[e], o);
-      m[e] = __hmax2(m[e], other);
-    }
+    for (int o = 8; o < 32; o <<= 1) m[e] = __hmax2(m[e], __shfl_xor_sync(0xffffffffu, m[e], o));
   }
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (lane < 4) {
+  if (lane < 8) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) red[warp][lane][e] = m[e];
   }
   __syncthreads();
-  if (warp == 0) {
-    // lane c owns column 32b + c: chunk g = c / 8, half2 e = (c % 8) / 2, half (c % 2)
-    const int cg = lane / 8, ce = (lane % 8) / 2, hi = lane % 2;
-    float cmax = 0.0f;
+  if (threadIdx.x < kColStrip) {  // thread j: column 64 strip + j
+    const int j = threadIdx.x, cg = j / 8, ce = (j % 8) / 2, hi = j % 2;
+    __half h = __float2half_rn(0.0f);
 #pragma unroll
     for (int w = 0; w < kCMThreads / 32; ++w) {
       const __half2 v = red[w][cg][ce];
-      cmax = fmaxf(cmax, hi ? __high2float(v) : __low2float(v));
+      h = __hmax(h, hi ? __high2half(v) : __low2half(v));
     }
-    const uint32_t bits = __ballot_sync(0xffffffffu, cmax > threshold);
-    if (lane == 0) mask[blockIdx.x] = bits;
+    const int col = strip * kColStrip + j;
+    if (col < K) pmax[static_cast<size_t>(rb) * K + col] = h;
+    __threadfence();
   }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int done = atomicAdd(&strip_cnt[strip], 1);
+    last = done == nrb - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  // the strip's last block: every row block's maxima are in pmax
+  __threadfence();
+  if (threadIdx.x < kColStrip) {
+    const int col = strip * kColStrip + threadIdx.x;
+    float cmax = 0.0f;
+    if (col < K)
+      for (int b = 0; b < nrb; ++b)
+        cmax = fmaxf(cmax, __half2float(__ldcg(pmax + static_cast<size_t>(b) * K + col)));
+    const uint32_t bits = __ballot_sync(0xffffffffu, cmax > threshold);
+    const int word = strip * 2 + threadIdx.x / 32;
+    if ((threadIdx.x & 31) == 0 && word * 32 < K) mask[word] = bits;
+  }
+  if (threadIdx.x == 0) strip_cnt[strip] = 0;
 }
 
 cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint32_t* mask,
-                           cudaStream_t stream, bool pdl) {
+                           __half* pmax, int32_t* strip, cudaStream_t stream, bool pdl) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((K + 31) / 32);
+  cfg.gridDim = dim3((K + kColStrip - 1) / kColStrip, (M + kColRowBlock - 1) / kColRowBlock);
   cfg.blockDim = dim3(kCMThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -186,7 +241,7 @@ cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint3
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, colmask_kernel, X, M, K, threshold, mask);
+  return cudaLaunchKernelEx(&cfg, colmask_kernel, X, M, K, threshold, mask, pmax, strip);
 }
 
 // ------------------------------------------------------------------ rows + outlier operands
@@ -196,9 +251,12 @@ constexpr int kRQRegChunks = 8;                         // chunks of 8 halves ke
 constexpr int kRQRegK = kRQThreads * 8 * kRQRegChunks;  // rows up to this length stay in registers
 constexpr int kRQMaxWords = INT8MM_MAX_K / 32;
 
+constexpr int kGatherSmemCols = 2048;  // outlier columns the weight gather lists in smem
+
 struct RowQuantShared {
   uint32_t mask[kRQMaxWords];
   int32_t prefix[kRQMaxWords];  // outliers in the words before this one
+  int32_t cols[kGatherSmemCols];  // the outlier columns (weight gather, n_out <= 2048)
   int32_t warp_sum[kRQThreads / 32];
   float red[kRQThreads / 32];
   int32_t n_out;
@@ -240,141 +298,189 @@ __device__ void load_mask_prefix(RowQuantShared& S, const uint32_t* __restrict__
   __syncthreads();
 }
 
-// Column of the r-th outlier (0-based, r < n_out): binary search over the prefix table.
-__device__ __forceinline__ int outlier_column(const RowQuantShared& S, int words, int r) {
-  int lo = 0, hi = words - 1;  // find the last word with prefix <= r
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (S.prefix[mid] <= r) lo = mid; else hi = mid - 1;
-  }
-  uint32_t m = S.mask[lo];
-  for (int k = r - S.prefix[lo]; k > 0; --k) m &= m - 1u;  // drop the lower outliers
-  return lo * 32 + __ffs(m) - 1;
+// The row pass.  A block takes rpb = 256 / tpr rows (tpr = threads per row, 32..256): thread
+// (row t / tpr, lane t % tpr) holds chunks lane + u * tpr (u < 8) of its row in registers
+// (rows of up to kRQRegK columns), so the block keeps up to 32 KB of X in flight and shares
+// one mask prologue.  Longer rows (one per block) are read twice from global memory.
+
+// outlier bits (one per column) of chunk c: byte c % 4 of mask word c / 4
+__device__ __forceinline__ uint32_t chunk_bits(const RowQuantShared& S, int c) {
+  return (S.mask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
 }
 
-// Block for one row: absmax over the regular columns, scale, codes, outlier activations.
-__device__ void quantize_row(const RowQuantArgs& a, RowQuantShared& S, int i) {
+__device__ __forceinline__ void absmax_chunk(const uint4& x, uint32_t bits, __half2& m2, float& mf) {
+  if (bits == 0) {
+    m2 = habs2_max(m2, x.x);
+    m2 = habs2_max(m2, x.y);
+    m2 = habs2_max(m2, x.z);
+    m2 = habs2_max(m2, x.w);
+  } else {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (!((bits >> e) & 1u)) {
+        const uint32_t hb = (w[e / 2] >> (16 * (e & 1))) & 0xFFFFu;
+        mf = fmaxf(mf, fabsf(__half2float(__ushort_as_half(static_cast<unsigned short>(hb)))));
+      }
+  }
+}
+
+// the fp16 values of chunk c's outlier columns, at their places in the compacted row
+__device__ __forceinline__ void emit_outliers(const RowQuantShared& S, const uint4& x, int c,
+                                              uint32_t bits, __half* xo) {
+  const int word = c >> 2;
+  const uint32_t wm = S.mask[word];
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if ((bits >> e) & 1u) {
+      const int bit = (c & 3) * 8 + e;
+      const int r = S.prefix[word] + __popc(wm & ((1u << bit) - 1u));
+      const uint32_t hb = (w[e / 2] >> (16 * (e & 1))) & 0xFFFFu;
+      xo[r] = __ushort_as_half(static_cast<unsigned short>(hb));
+    }
+}
+
+// Row i of the block (tpr threads): absmax over the regular columns, scale, codes, outlier
+// activations.  In-register rows arrive in v.
+__device__ void quantize_rows_block(const RowQuantArgs& a, RowQuantShared& S, int tpr,
+                                    const uint4 (&v)[kRQRegChunks]) {
   const int K = a.K;
   const int chunks = K / 8;
-  const uint4* row = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * K);
+  const int rl = threadIdx.x / tpr, lr = threadIdx.x % tpr;
+  const int i = blockIdx.x * (kRQThreads / tpr) + rl;
+  const bool live = i < a.M;
   const bool in_regs = K <= kRQRegK;
-  uint4 v[kRQRegChunks];
+  const uint4* row = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(live ? i : 0) * K);
   __half2 m2 = __float2half2_rn(0.0f);
   float mf = 0.0f;
-  // pass 1: absmax over regular columns
-  auto absmax_chunk = [&](const uint4& x, int c) {
-    const uint32_t bits = (S.mask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-    if (bits == 0) {
-      m2 = habs2_max(m2, x.x);
-      m2 = habs2_max(m2, x.y);
-      m2 = habs2_max(m2, x.z);
-      m2 = habs2_max(m2, x.w);
-    } else {
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (!((bits >> e) & 1u)) {
-          const uint32_t hb = (w[e / 2] >> (16 * (e & 1))) & 0xFFFFu;
-          mf = fmaxf(mf, fabsf(__half2float(__ushort_as_half(static_cast<unsigned short>(hb)))));
-        }
-    }
-  };
+  uint32_t bits_r[kRQRegChunks];
   if (in_regs) {
 #pragma unroll
     for (int u = 0; u < kRQRegChunks; ++u) {
-      const int c = threadIdx.x + u * kRQThreads;
-      if (c < chunks) v[u] = __ldg(row + c);
+      const int c = lr + u * tpr;
+      bits_r[u] = 0u;
+      if (live && c < chunks) {
+        bits_r[u] = chunk_bits(S, c);
+        absmax_chunk(v[u], bits_r[u], m2, mf);
+      }
     }
-#pragma unroll
-    for (int u = 0; u < kRQRegChunks; ++u) {
-      const int c = threadIdx.x + u * kRQThreads;
-      if (c < chunks) absmax_chunk(v[u], c);
-    }
-  } else {
-    for (int c = threadIdx.x; c < chunks; c += kRQThreads) absmax_chunk(__ldg(row + c), c);
+  } else if (live) {
+    for (int c = lr; c < chunks; c += tpr) absmax_chunk(__ldg(row + c), chunk_bits(S, c), m2, mf);
   }
-  const float amax = block_max<kRQThreads>(fmaxf(mf, half2_max_f(m2)), S.red);
+  // maximum over the row's tpr threads: the warp, then the row's warps
+  float m = fmaxf(mf, half2_max_f(m2));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const int warp = threadIdx.x / 32;
+  if ((threadIdx.x & 31) == 0) S.red[warp] = m;
+  __syncthreads();
+  float amax = 0.0f;
+  for (int w = rl * (tpr / 32); w < (rl + 1) * (tpr / 32); ++w) amax = fmaxf(amax, S.red[w]);
+  if (!live) return;
   const float s = __fdiv_rn(amax, 127.0f);
-  if (threadIdx.x == 0) a.xscale[i] = s;
+  if (lr == 0) a.xscale[i] = s;
   const bool zero_row = amax == 0.0f;
+  const float rcp = zero_row ? 0.0f : __frcp_rn(s);
 
-  // pass 2: codes and the outlier activations
   uint2* out = reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(i) * K);
   __half* xo = a.xo ? a.xo + static_cast<size_t>(i) * a.ldo : nullptr;
-  auto emit_chunk = [&](const uint4& x, int c) {
-    const uint32_t bits = (S.mask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-    out[c] = quantize_chunk(x, s, zero_row, bits);
-    if (bits != 0 && xo != nullptr) {
-      const int word = c >> 2;
-      const uint32_t wm = S.mask[word];
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if ((bits >> e) & 1u) {
-          const int bit = (c & 3) * 8 + e;
-          const int r = S.prefix[word] + __popc(wm & ((1u << bit) - 1u));
-          const uint32_t hb = (w[e / 2] >> (16 * (e & 1))) & 0xFFFFu;
-          xo[r] = __ushort_as_half(static_cast<unsigned short>(hb));
-        }
-    }
-  };
   if (in_regs) {
 #pragma unroll
     for (int u = 0; u < kRQRegChunks; ++u) {
-      const int c = threadIdx.x + u * kRQThreads;
-      if (c < chunks) emit_chunk(v[u], c);
+      const int c = lr + u * tpr;
+      if (c < chunks) {
+        out[c] = zero_row ? make_uint2(0u, 0u) : quantize_chunk_fast(v[u], s, rcp, bits_r[u]);
+        if (bits_r[u] != 0 && xo != nullptr) emit_outliers(S, v[u], c, bits_r[u], xo);
+      }
     }
   } else {
-    for (int c = threadIdx.x; c < chunks; c += kRQThreads) emit_chunk(__ldg(row + c), c);
+    for (int c = lr; c < chunks; c += tpr) {
+      const uint4 x = __ldg(row + c);
+      const uint32_t bits = chunk_bits(S, c);
+      out[c] = zero_row ? make_uint2(0u, 0u) : quantize_chunk_fast(x, s, rcp, bits);
+      if (bits != 0 && xo != nullptr) emit_outliers(S, x, c, bits, xo);
+    }
   }
   if (xo != nullptr) {
     const int n_out = S.n_out;
     const int padded = (n_out + 63) / 64 * 64;
-    for (int r = n_out + threadIdx.x; r < padded; r += kRQThreads) xo[r] = __float2half_rn(0.0f);
+    for (int r = n_out + lr; r < padded; r += tpr) xo[r] = __float2half_rn(0.0f);
   }
 }
 
 // Extra blocks: W_hat[n, r] = fp16(float(Wq[n, col(r)]) * w_scale[n]), zero-padded to 64.
+// The outliers are taken in windows of kGatherSmemCols: the block lists the window's columns
+// in shared memory, then thread u writes the 8 consecutive entries (one 16-byte store) of
+// channel u / groups, group u % groups of the window.
 __device__ void gather_weights(const RowQuantArgs& a, RowQuantShared& S, int words, int gb,
                                int G) {
   const int n_out = S.n_out;
   const int width = (n_out + 63) / 64 * 64;
-  const int groups = width / 8;  // 8 consecutive outliers per thread step (one 16-byte store)
-  const long long units = static_cast<long long>(a.N) * groups;
-  for (long long u = static_cast<long long>(gb) * kRQThreads + threadIdx.x; u < units;
-       u += static_cast<long long>(G) * kRQThreads) {
-    const int n = static_cast<int>(u / groups);
-    const int r0 = static_cast<int>(u % groups) * 8;
-    const float sc = a.w_scale[n];
-    const int8_t* wrow = a.Wq + static_cast<size_t>(n) * a.K;
-    uint32_t h[4] = {0u, 0u, 0u, 0u};
-    if (r0 < n_out) {
-      int col = outlier_column(S, words, r0);
+  for (int R0 = 0; R0 < width; R0 += kGatherSmemCols) {  // block-uniform
+    const int R1 = min(n_out, R0 + kGatherSmemCols);     // outliers of this window
+    for (int w = threadIdx.x; w < words; w += kRQThreads) {
+      const int p0 = S.prefix[w];
+      uint32_t m = S.mask[w];
+      if (p0 >= R1 || p0 + __popc(m) <= R0) continue;
+      for (int r = p0; m; ++r, m &= m - 1)
+        if (r >= R0 && r < R1) S.cols[r - R0] = w * 32 + __ffs(m) - 1;
+    }
+    __syncthreads();
+    const int groups = (min(width, R0 + kGatherSmemCols) - R0) / 8;
+    const long long units = static_cast<long long>(a.N) * groups;
+    for (long long u = static_cast<long long>(gb) * kRQThreads + threadIdx.x; u < units;
+         u += static_cast<long long>(G) * kRQThreads) {
+      const int n = static_cast<int>(u / groups);
+      const int r0 = R0 + static_cast<int>(u % groups) * 8;
+      uint32_t h[4] = {0u, 0u, 0u, 0u};
+      if (r0 < n_out) {
+        const float sc = a.w_scale[n];
+        const int8_t* wrow = a.Wq + static_cast<size_t>(n) * a.K;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int r = r0 + e;
-        if (r < n_out) {
-          if (e > 0) {  // next set bit after col
-            int w = (col + 1) >> 5;
-            uint32_t rest = ((col + 1) & 31) ? (S.mask[w] & (~0u << ((col + 1) & 31))) : S.mask[w];
-            while (rest == 0) rest = S.mask[++w];
-            col = w * 32 + __ffs(rest) - 1;
+        for (int e = 0; e < 8; ++e) {
+          const int r = r0 + e;
+          if (r < n_out) {
+            const __half hv = __float2half_rn(static_cast<float>(wrow[S.cols[r - R0]]) * sc);
+            h[e / 2] |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * (e & 1));
           }
-          const __half hv = __float2half_rn(static_cast<float>(wrow[col]) * sc);
-          h[e / 2] |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * (e & 1));
         }
       }
+      *reinterpret_cast<uint4*>(a.wo + static_cast<size_t>(n) * a.ldo + r0) =
+          make_uint4(h[0], h[1], h[2], h[3]);
     }
-    *reinterpret_cast<uint4*>(a.wo + static_cast<size_t>(n) * a.ldo + r0) =
-        make_uint4(h[0], h[1], h[2], h[3]);
+    __syncthreads();  // the list is rewritten for the next window
   }
 }
 
-__global__ void __launch_bounds__(kRQThreads) rowquant_kernel(const RowQuantArgs a) {
+// threads per row of the row pass: rows of up to 2048 / rpb chunks share a block
+__host__ __device__ inline int rowquant_tpr(int K) {
+  const int chunks = K / 8;
+  int rpb = 1;
+  while (rpb < 8 && chunks * rpb * 2 <= kRQThreads * kRQRegChunks) rpb *= 2;
+  return kRQThreads / rpb;
+}
+
+__global__ void __launch_bounds__(kRQThreads) rowquant_kernel(const RowQuantArgs a, int row_blocks) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
   RowQuantShared& S = *reinterpret_cast<RowQuantShared*>(rq_smem);
   grid_dependency_wait();
   const int words = (a.K + 31) / 32;
+  const int tpr = rowquant_tpr(a.K);
+  // the rows' loads go out before the mask prologue, which waits on its own loads
+  const bool row_block = static_cast<int>(blockIdx.x) < row_blocks;
+  const int chunks = a.K / 8;
+  uint4 v[kRQRegChunks];
+  if (row_block && a.K <= kRQRegK) {
+    const int i = blockIdx.x * (kRQThreads / tpr) + threadIdx.x / tpr, lr = threadIdx.x % tpr;
+    const uint4* row = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * a.K);
+#pragma unroll
+    for (int u = 0; u < kRQRegChunks; ++u) {
+      const int c = lr + u * tpr;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < a.M && c < chunks) v[u] = __ldg(row + c);
+    }
+  }
   load_mask_prefix(S, a.mask, words);
   grid_launch_dependents();
   if (blockIdx.x == 0) {
@@ -389,10 +495,10 @@ __global__ void __launch_bounds__(kRQThreads) rowquant_kernel(const RowQuantArgs
     }
     if (threadIdx.x == 0) *a.n_out = S.n_out;
   }
-  if (static_cast<int>(blockIdx.x) < a.M) {
-    quantize_row(a, S, blockIdx.x);
+  if (row_block) {
+    quantize_rows_block(a, S, tpr, v);
   } else if (a.wo != nullptr) {
-    gather_weights(a, S, words, blockIdx.x - a.M, gridDim.x - a.M);
+    gather_weights(a, S, words, blockIdx.x - row_blocks, gridDim.x - row_blocks);
   }
 }
 
@@ -409,11 +515,14 @@ cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl
   if (a.wo != nullptr) {
     const long long worst_units = static_cast<long long>(a.N) * (a.ldo / 8);
     const long long want = (worst_units + kRQThreads - 1) / kRQThreads;
-    gather_blocks = static_cast<int>(want < 1184 ? want : 1184);
+    const long long cap = 2LL * device_sm_count();
+    gather_blocks = static_cast<int>(want < cap ? want : cap);
     if (gather_blocks < 1) gather_blocks = 1;
   }
+  const int rpb = kRQThreads / rowquant_tpr(a.K);
+  const int row_blocks = (a.M + rpb - 1) / rpb;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.M + gather_blocks);
+  cfg.gridDim = dim3(row_blocks + gather_blocks);
   cfg.blockDim = dim3(kRQThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -422,7 +531,7 @@ cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, rowquant_kernel, a);
+  return cudaLaunchKernelEx(&cfg, rowquant_kernel, a, row_blocks);
 }
 
 // ------------------------------------------------------------------ diagnostic: W_hat alone
