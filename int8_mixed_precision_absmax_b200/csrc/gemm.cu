@@ -9,9 +9,10 @@
 // results are merged at the end).  The dequantization by the outer product of the row
 // and column scales undoes x ~ q * sx and w ~ q * w_scale of [P5] items 1 and 2.
 //
-// Roles (192 threads): warp 0 issues TMA loads into a 4-stage shared-memory ring, warp 1
-// allocates tensor memory and issues the MMAs (one thread), warps 2-5 drain the
-// accumulators (each warp owns the 32 TMEM lanes of its quadrant).  With both products
+// Roles (320 threads): warp 0 issues TMA loads into a 4-stage shared-memory ring, warp 1
+// allocates tensor memory and issues the MMAs (one thread), warps 2-9 drain the
+// accumulators (two warps per 32-lane TMEM quadrant, each taking half of the tile's columns;
+// the tile's column scales and bias are staged in shared memory once).  With both products
 // present the 512 TMEM columns hold one int32 and one fp32 accumulator; with only one of
 // them, two accumulator slots alternate so the epilogue of a tile overlaps the next
 // tile's main loop.  Every wait is bounded (ptx.cuh); a wait that gives up writes
@@ -27,7 +28,8 @@ namespace {
 constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBKBytes;  // 16 KB
 constexpr int kBBytes = kBN * kBKBytes;  // 32 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = kThreads - 64;  // warps 2..9
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdescI8 = idesc_i8_s32(kBM, kBN);
 constexpr uint32_t kIdescF16 = idesc_f16_f32(kBM, kBN);
@@ -42,6 +44,8 @@ struct GemmShared {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  float wscale[2][kBN];  // the tile's column scales and bias, by accumulator slot parity
+  float bias[2][kBN];
 };
 constexpr size_t kSmemBytes = sizeof(GemmShared) + 1024;  // + alignment slack
 
@@ -52,6 +56,24 @@ struct TileSchedule {
     n0 = (tile / m_tiles) * kBN;
   }
 };
+
+// Named barrier 1 of the epilogue warps; the second form returns whether any of them
+// passed `v` true (one decision for all, so they leave the tile loop together).
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+}
+__device__ __forceinline__ bool epi_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "r"(kEpiThreads)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
@@ -95,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&S.tmem_full[b], 1);
-      mbar_init(&S.tmem_empty[b], 128);
+      mbar_init(&S.tmem_empty[b], kEpiThreads);
     }
     mbar_init(&S.drain, 1);
     S.abort = 0;
@@ -201,27 +223,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) report(args.status, INT8MM_ERR_TIMEOUT);
     }
   } else {
-    // -------------------------------------------------- epilogue (warps 2..5)
-    const int quad = warp & 3;
+    // -------------------------------------------------- epilogue (warps 2..9)
+    const int quad = warp & 3;                // TMEM lanes 32 quad .. 32 quad + 31
+    const int half = (warp - 2) / 4;          // columns 128 half .. 128 half + 127
+    const int et = threadIdx.x - 64;          // 0 .. kEpiThreads - 1
     const bool vec_ok = (N % 8) == 0;
     int it = 0;
     for (int tile = blockIdx.x; tile < sched.tiles; tile += gridDim.x, ++it) {
       const int slot = (nslots == 1) ? 0 : (it & 1);
       const uint32_t use = (nslots == 1) ? it : (it >> 1);
-      if (!mbar_wait_bounded(&S.tmem_full[slot], use & 1u, abort)) {
+      int m0, n0;
+      sched.coords(tile, m0, n0);
+      // the tile's column scales and bias (buffer it & 1: the previous tile's may still be
+      // in use by a slower epilogue warp)
+      {
+        const int n = n0 + et;
+        // (the raw int32 product has neither: w_scale and bias are null there)
+        S.wscale[it & 1][et] = (et < kBN && n < N && args.w_scale) ? args.w_scale[n] : 0.0f;
+        S.bias[it & 1][et] = (et < kBN && n < N && args.bias) ? __half2float(args.bias[n]) : 0.0f;
+        epi_sync();
+      }
+      const bool landed = mbar_wait_bounded(&S.tmem_full[slot], use & 1u, abort);
+      if (epi_any(!landed)) {  // every epilogue thread takes the same branch
         report(args.status, INT8MM_ERR_TIMEOUT);
         break;
       }
       tc_fence_after();
-      int m0, n0;
-      sched.coords(tile, m0, n0);
       const int row = m0 + quad * 32 + lane;
       const bool row_ok = row < M;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
       const uint32_t t_i8 = lane_base + (both ? 0u : slot * 256u);
       const uint32_t t_f32 = lane_base + (both ? 256u : slot * 256u);
       const float sx = (args.Y && row_ok) ? args.xscale[row] : 0.0f;
-      for (int c = 0; c < kBN; c += 32) {
+      const float* wsc = S.wscale[it & 1];
+      const float* bsc = S.bias[it & 1];
+      for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 32) {
         uint32_t ra[32], rp[32];
         __syncwarp();  // the tensor-memory loads are warp-collective
         if (kb_i8 > 0) tmem_ld_32x32b_x32(t_i8 + c, ra);
@@ -246,13 +282,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row_ok && valid > 0 && args.Y) {
           float y[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int nn = min(n + j, N - 1);
-            float acc = 0.0f;
-            if (kb_i8 > 0) acc = static_cast<float>(static_cast<int32_t>(ra[j])) * sx * args.w_scale[nn];
-            if (kb_f16 > 0) acc += __uint_as_float(rp[j]);
-            if (args.bias) acc += __half2float(args.bias[nn]);
-            y[j] = acc;
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 ws = *reinterpret_cast<const float4*>(wsc + c + 4 * j4);
+            const float4 bs = *reinterpret_cast<const float4*>(bsc + c + 4 * j4);
+            const float wv[4] = {ws.x, ws.y, ws.z, ws.w}, bv[4] = {bs.x, bs.y, bs.z, bs.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 4 * j4 + e;
+              float acc = 0.0f;
+              if (kb_i8 > 0) acc = static_cast<float>(static_cast<int32_t>(ra[j])) * sx * wv[e];
+              if (kb_f16 > 0) acc += __uint_as_float(rp[j]);
+              y[j] = acc + bv[e];
+            }
           }
           store_half32(args.Y + static_cast<size_t>(row) * N + n, y, valid, vec_ok);
         }
