@@ -15,7 +15,12 @@
 // the tile's column scales and bias are staged in shared memory once).  With both products
 // present the 512 TMEM columns hold one int32 and one fp32 accumulator; with only one of
 // them, two accumulator slots alternate so the epilogue of a tile overlaps the next
-// tile's main loop.  Every wait is bounded (ptx.cuh); a wait that gives up writes
+// tile's main loop.  With both products the epilogue works in two phases: it folds the
+// int32 accumulator, the scales, the fp32 outlier term and the bias into fp32 Y written
+// back over the outlier accumulator (tcgen05.st) and releases the int32 columns, so the
+// next tile's int8 MMAs start at once; it then converts and stores Y and releases the
+// fp32 columns, which the next tile needs only for its fp16 MMAs, issued last.
+// Every wait is bounded (ptx.cuh); a wait that gives up writes
 // INT8MM_ERR_TIMEOUT to the status word, and the block drains its in-flight copies and
 // MMAs, frees its tensor memory and exits.
 #include "kernels.cuh"
@@ -77,26 +82,6 @@ __device__ __forceinline__ bool epi_any(bool v) {
 
 __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
-}
-
-__device__ __forceinline__ void store_half32(__half* dst, const float (&y)[32], int valid,
-                                             bool vec_ok) {
-  if (vec_ok && valid == 32) {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __half2 h = __floats2half2_rn(y[v * 8 + 2 * e], y[v * 8 + 2 * e + 1]);
-        w[e] = *reinterpret_cast<const uint32_t*>(&h);
-      }
-      reinterpret_cast<uint4*>(dst)[v] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < valid) dst[j] = __float2half_rn(y[j]);
-  }
 }
 
 }  // namespace
@@ -197,6 +182,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_i8 = tmem + (both ? 0u : slot * 256u);
         const uint32_t d_f32 = tmem + (both ? 256u : slot * 256u);
         for (int kb = 0; kb < kb_total; ++kb) {
+          if (both && kb == kb_i8) {  // the fp32 columns: free once the last tile's Y is out
+            if (!mbar_wait_bounded(&S.tmem_empty[1], (static_cast<uint32_t>(it) & 1u) ^ 1u,
+                                   abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
           if (!mbar_wait_bounded(&S.full[stage], phase, abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_addr(S.a[stage]);
@@ -257,32 +250,104 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float sx = (args.Y && row_ok) ? args.xscale[row] : 0.0f;
       const float* wsc = S.wscale[it & 1];
       const float* bsc = S.bias[it & 1];
-      for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 32) {
-        uint32_t ra[32], rp[32];
+      if (both) {
+        // phase 1: Y in fp32 over the outlier accumulator, then the int32 columns are free
+        for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 16) {
+          uint32_t ra[16], rp[16];
+          __syncwarp();
+          tmem_ld16(t_i8 + c, ra);
+          tmem_ld16(t_f32 + c, rp);
+          tmem_ld_wait();
+          const int n = n0 + c;
+          const int valid = min(16, N - n);
+          if (row_ok && valid > 0 && args.C) {
+            int32_t* dst = args.C + static_cast<size_t>(row) * N + n;
+            if (valid == 16 && (N % 4) == 0) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                reinterpret_cast<int4*>(dst)[v] =
+                    make_int4(ra[4 * v], ra[4 * v + 1], ra[4 * v + 2], ra[4 * v + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (j < valid) dst[j] = static_cast<int32_t>(ra[j]);
+            }
+          }
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 ws = *reinterpret_cast<const float4*>(wsc + c + 4 * j4);
+            const float4 bs = *reinterpret_cast<const float4*>(bsc + c + 4 * j4);
+            const float wv[4] = {ws.x, ws.y, ws.z, ws.w}, bv[4] = {bs.x, bs.y, bs.z, bs.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 4 * j4 + e;
+              const float acc = static_cast<float>(static_cast<int32_t>(ra[j])) * sx * wv[e] +
+                                __uint_as_float(rp[j]);
+              rp[j] = __float_as_uint(acc + bv[e]);
+            }
+          }
+          tmem_st16(t_f32 + c, rp);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&S.tmem_empty[0]);
+        // phase 2: Y out, then the fp32 columns are free
+        for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 16) {
+          uint32_t ry[16];
+          __syncwarp();
+          tmem_ld16(t_f32 + c, ry);
+          tmem_ld_wait();
+          const int n = n0 + c;
+          const int valid = min(16, N - n);
+          if (row_ok && valid > 0 && args.Y) {
+            __half* dst = args.Y + static_cast<size_t>(row) * N + n;
+            if (vec_ok && valid == 16) {
+              uint32_t w[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const __half2 h = __floats2half2_rn(__uint_as_float(ry[2 * e]),
+                                                    __uint_as_float(ry[2 * e + 1]));
+                w[e] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+              reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (j < valid) dst[j] = __float2half_rn(__uint_as_float(ry[j]));
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&S.tmem_empty[1]);
+        continue;
+      }
+      for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 16) {
+        uint32_t ra[16], rp[16];
         __syncwarp();  // the tensor-memory loads are warp-collective
-        if (kb_i8 > 0) tmem_ld_32x32b_x32(t_i8 + c, ra);
-        if (kb_f16 > 0) tmem_ld_32x32b_x32(t_f32 + c, rp);
+        if (kb_i8 > 0) tmem_ld16(t_i8 + c, ra);
+        if (kb_f16 > 0) tmem_ld16(t_f32 + c, rp);
         tmem_ld_wait();
         const int n = n0 + c;
-        const int valid = min(32, N - n);
+        const int valid = min(16, N - n);
         if (row_ok && valid > 0 && args.C) {
           int32_t* dst = args.C + static_cast<size_t>(row) * N + n;
-          if (valid == 32 && (N % 4) == 0) {
+          if (valid == 16 && (N % 4) == 0) {
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
+            for (int v = 0; v < 4; ++v)
               reinterpret_cast<int4*>(dst)[v] =
                   make_int4(kb_i8 ? ra[4 * v] : 0, kb_i8 ? ra[4 * v + 1] : 0,
                             kb_i8 ? ra[4 * v + 2] : 0, kb_i8 ? ra[4 * v + 3] : 0);
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
+            for (int j = 0; j < 16; ++j)
               if (j < valid) dst[j] = kb_i8 ? static_cast<int32_t>(ra[j]) : 0;
           }
         }
         if (row_ok && valid > 0 && args.Y) {
-          float y[32];
+          float y[16];
 #pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
+          for (int j4 = 0; j4 < 4; ++j4) {
             const float4 ws = *reinterpret_cast<const float4*>(wsc + c + 4 * j4);
             const float4 bs = *reinterpret_cast<const float4*>(bsc + c + 4 * j4);
             const float wv[4] = {ws.x, ws.y, ws.z, ws.w}, bv[4] = {bs.x, bs.y, bs.z, bs.w};
@@ -295,7 +360,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               y[j] = acc + bv[e];
             }
           }
-          store_half32(args.Y + static_cast<size_t>(row) * N + n, y, valid, vec_ok);
+          __half* dst = args.Y + static_cast<size_t>(row) * N + n;
+          if (vec_ok && valid == 16) {
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const __half2 h = __floats2half2_rn(y[2 * e], y[2 * e + 1]);
+              w[e] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (j < valid) dst[j] = __float2half_rn(y[j]);
+          }
         }
       }
       tc_fence_before();
