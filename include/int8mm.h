@@ -108,9 +108,12 @@ int int8_linear_forward(const void *X, int M, int K, const int8_t *Wq, const flo
  *
  * int8_linear_quantize: the activation side.  For M > 16: outlier columns, per-row scales,
  *   int8 activations and the compacted fp16 outlier operands (activations and
- *   W_hat = fp16(Wq * w_scale)), written into the workspace.  For M <= 16 (few tokens, the
- *   weight-streaming regime, K <= 32768) it enqueues nothing: one kernel in
- *   int8_linear_matmul quantizes the activations next to the tensor cores.
+ *   W_hat = fp16(Wq * w_scale)), written into the workspace.  For few tokens (the
+ *   weight-streaming regime): with M <= 8, K % 128 == 0 and K <= 8192 it enqueues nothing (one
+ *   kernel in int8_linear_matmul does the whole layer); with M <= 16 otherwise under the same
+ *   K limits it enqueues one kernel that quantizes the activations once into the workspace;
+ *   for longer rows with M <= 16 it enqueues nothing (one kernel quantizes next to the tensor
+ *   cores).
  * int8_linear_matmul: the rest -- the int8 and fp16 products and the fused epilogue --
  *   reading what int8_linear_quantize left in the workspace.
  */
