@@ -224,9 +224,8 @@ int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_s
     if (small_path_fits(M, K)) return INT8MM_OK;  // one kernel does everything: see run_matmul
   }
   int rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
-                                        effective_threshold(threshold), p.mask,
-                                        at<__half>(workspace, p.L.pmax),
-                                        at<int32_t>(workspace, p.L.strip), stream, pdl_first));
+                                        effective_threshold(threshold), p.mask, stream,
+                                        pdl_first));
   if (rc) return rc;
   RowQuantArgs rq;
   rq.X = static_cast<const __half*>(X);
@@ -376,9 +375,7 @@ int int8_quantize_rows(const void* X, int M, int K, float threshold, int8_t* Xq,
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   uint32_t* mask = at<uint32_t>(workspace, L.mask);
   if ((rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
-                                         effective_threshold(threshold), mask,
-                                         at<__half>(workspace, L.pmax),
-                                         at<int32_t>(workspace, L.strip), stream, false))))
+                                         effective_threshold(threshold), mask, stream, false))))
     return rc;
   RowQuantArgs rq = {};
   rq.X = static_cast<const __half*>(X);

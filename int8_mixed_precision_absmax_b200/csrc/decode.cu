@@ -121,34 +121,45 @@ __device__ __forceinline__ float h2f(uint32_t word, int hi) {
 // rne(x * r) with r = 1/sx rounded to nearest equals rne(fl(x / sx)) unless x * r lies within
 // 2^-15 of a half-integer (the exact x * r is within 2^-17 of x / sx for |x / sx| <= 128, the
 // rounded quotient within 2^-18); there the quotient itself (__fdiv_rn) is rounded.
-// rne(x * r) comes from one fused multiply-add with 1.5 * 2^23, whose low bits then hold the
-// integer.  A regular column has |x| <= the row maximum, so |x / sx| <= 127 * (1 + 2^-22) and
-// the code needs no clamp; outlier columns are masked out after the fact.
+// tb = fl(x * r + 1.5 * 2^23) = 1.5 * 2^23 + rne(x * r) exactly, and as 1.5 * 2^23 has a zero
+// low byte, the low byte of tb's bits is the two's-complement code.  d = x * r - rne(x * r)
+// (one more FMA, rounding error <= 2^-25) has |d| <= 1/2, so "near a half-integer" is
+// |d| > 1/2 - 2^-15.  A regular column has |x| <= the row maximum, so |x / sx| <=
+// 127 (1 + 2^-22) and the code needs no clamp; outlier columns are masked out after the fact.
 __device__ __forceinline__ uint32_t keep_mask(uint32_t bits4) {  // bit e set -> byte e = 0
   return ~(((bits4 * 0x204081u) & 0x01010101u) * 0xFFu);
 }
 __device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, uint32_t bits) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kNear = 0.5f - 0x1p-15f;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   float x[8];
-  int qv[8];
-  uint32_t near_tie = 0;
+  uint32_t qb[8];
+  bool near_tie = false;
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e / 2]));
+    x[e] = f.x;
+    x[e + 1] = f.y;
+  }
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    x[e] = h2f(w[e / 2], e & 1);
     const float tb = __fmaf_rn(x[e], rcp, kRound);
-    qv[e] = __float_as_int(tb) - 0x4B400000;
-    const float d = fabsf(__fmaf_rn(x[e], rcp, -(tb - kRound)));
-    near_tie |= (fabsf(d - 0.5f) <= 0x1p-15f ? 1u : 0u) << e;
+    qb[e] = __float_as_uint(tb);
+    const float d = __fmaf_rn(x[e], rcp, -(tb - kRound));
+    near_tie |= fabsf(d) > kNear && !((bits >> e) & 1u);
   }
-  near_tie &= ~bits;
   if (near_tie) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if ((near_tie >> e) & 1u) qv[e] = __float2int_rn(__fdiv_rn(x[e], sc));
+    for (int e = 0; e < 8; ++e) {
+      const float tb = __fmaf_rn(x[e], rcp, kRound);
+      const float d = __fmaf_rn(x[e], rcp, -(tb - kRound));
+      if (fabsf(d) > kNear && !((bits >> e) & 1u))
+        qb[e] = static_cast<uint32_t>(__float2int_rn(__fdiv_rn(x[e], sc)));
+    }
   }
-  const uint32_t lo = __byte_perm(__byte_perm(qv[0], qv[1], 0x0040), __byte_perm(qv[2], qv[3], 0x0040), 0x5410);
-  const uint32_t hi = __byte_perm(__byte_perm(qv[4], qv[5], 0x0040), __byte_perm(qv[6], qv[7], 0x0040), 0x5410);
+  const uint32_t lo = __byte_perm(__byte_perm(qb[0], qb[1], 0x0040), __byte_perm(qb[2], qb[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(qb[4], qb[5], 0x0040), __byte_perm(qb[6], qb[7], 0x0040), 0x5410);
   return make_uint2(lo & keep_mask(bits & 0xFu), hi & keep_mask(bits >> 4));
 }
 

@@ -21,9 +21,6 @@ namespace i8mm {
 //   xq       int8[M*K]      quantized activations (0 in outlier columns)
 //   xo       half[M*ldo]    outlier activations, compacted, zero-padded to a multiple of 64
 //   wo       half[N*ldo]    outlier weights fp16(Wq*w_scale), compacted, zero-padded
-//   pmax     half[ceil(M/256)*K]   per-256-row-block column maxima |X| (outlier search)
-//   strip    int32[ceil(K/64)]     per-64-column-strip arrival counters of the outlier
-//                                  search (zero between calls: the last block resets them)
 // ldo = K rounded up to 64 (the fp16 operand tiles are 64 elements deep).
 // The few-token path (M <= kSmallMP) adds: int8 activations padded to 16 rows and to a
 // multiple of 256 columns (few_xq, int8[16*kpad]), the fp16 values of the outlier columns
@@ -34,11 +31,8 @@ constexpr int kSmallBN = 128;            // output channels per tile (M of the M
 constexpr int kSmallMaxSplits = 8;       // CTAs per cluster (portable cluster size)
 constexpr int kSmallMaxKbPerSplit = 16;  // 128-byte k-blocks of X / Xq one CTA keeps in smem
 
-constexpr int kColRowBlock = 256;  // rows per block of the outlier-column search
-constexpr int kColStrip = 64;      // columns per block of the outlier-column search
-
 struct WorkspaceLayout {
-  size_t header, mask, cols, xscale, xq, xo, wo, pmax, strip, few_xq, few_xo, few_sx, total;
+  size_t header, mask, cols, xscale, xq, xo, wo, few_xq, few_xo, few_sx, total;
   int ldo;
 };
 
@@ -55,9 +49,6 @@ inline WorkspaceLayout workspace_layout(int M, int N, int K) {
   L.xq = off;     off = align256(off + static_cast<size_t>(M) * K);
   L.xo = off;     off = align256(off + static_cast<size_t>(M) * L.ldo * sizeof(__half));
   L.wo = off;     off = align256(off + static_cast<size_t>(N) * L.ldo * sizeof(__half));
-  L.pmax = off;
-  off = align256(off + static_cast<size_t>((M + kColRowBlock - 1) / kColRowBlock) * K * sizeof(__half));
-  L.strip = off;  off = align256(off + static_cast<size_t>((K + kColStrip - 1) / kColStrip) * sizeof(int32_t));
   L.few_xq = L.few_xo = L.few_sx = off;
   if (M <= kSmallMP) {
     const size_t kpad = static_cast<size_t>((K + 255) / 256) * 256;
@@ -77,10 +68,8 @@ inline WorkspaceLayout workspace_layout(int M, int N, int K) {
 cudaError_t launch_quant_weight(const __half* W, int N, int K, int8_t* Wq, float* w_scale,
                                 cudaStream_t stream);
 
-// pmax: [ceil(M/256)][K] partial column maxima; strip: [ceil(K/64)] counters, zero on entry
-// and on exit.
 cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint32_t* mask,
-                           __half* pmax, int32_t* strip, cudaStream_t stream, bool pdl);
+                           cudaStream_t stream, bool pdl);
 
 cudaError_t launch_outlier_weights(const int8_t* Wq, const float* w_scale, int N, int K,
                                    const int32_t* cols, const int32_t* n_out, __half* W_hat,

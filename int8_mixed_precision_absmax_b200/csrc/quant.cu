@@ -52,39 +52,46 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 // |x| <= absmax = 127 s, packed little-endian, outlier columns (bits) set to 0.
 // With r = 1/s rounded to nearest, the exact x * r is within 2^-17 of x / s (|x / s| <= 128)
 // and the rounded quotient within 2^-18, so rne(x * r) = rne(fl(x / s)) unless x * r lies
-// within 2^-15 of a half-integer; there the quotient itself (__fdiv_rn) is rounded.  rne(x * r)
-// comes from one fused multiply-add with 1.5 * 2^23, whose low bits then hold the integer;
-// |x / s| <= 127 (1 + 2^-22) on regular columns, so the code needs no clamp.
+// within 2^-15 of a half-integer; there the quotient itself (__fdiv_rn) is rounded.
+// tb = fl(x * r + 1.5 * 2^23) = 1.5 * 2^23 + rne(x * r) exactly, and as 1.5 * 2^23 has a zero
+// low byte, the low byte of tb's bits is the two's-complement code.  d = x * r - rne(x * r)
+// (one more FMA, rounding error <= 2^-25) has |d| <= 1/2, so "near a half-integer" is
+// |d| > 1/2 - 2^-15.  |x / s| <= 127 (1 + 2^-22) on regular columns: no clamp is needed.
 __device__ __forceinline__ uint32_t keep_mask(uint32_t bits4) {  // bit e set -> byte e = 0
   return ~(((bits4 * 0x204081u) & 0x01010101u) * 0xFFu);
 }
 __device__ __forceinline__ uint2 quantize_chunk_fast(const uint4& v, float s, float rcp,
                                                      uint32_t bits) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kNear = 0.5f - 0x1p-15f;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   float x[8];
-  int qv[8];
-  uint32_t near_tie = 0;
+  uint32_t qb[8];
+  bool near_tie = false;
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e / 2]));
+    x[e] = f.x;
+    x[e + 1] = f.y;
+  }
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    if ((e & 1) == 0) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e / 2]));
-      x[e] = f.x;
-      x[e + 1] = f.y;
-    }
     const float tb = __fmaf_rn(x[e], rcp, kRound);
-    qv[e] = __float_as_int(tb) - 0x4B400000;
-    const float d = fabsf(__fmaf_rn(x[e], rcp, -(tb - kRound)));
-    near_tie |= (fabsf(d - 0.5f) <= 0x1p-15f ? 1u : 0u) << e;
+    qb[e] = __float_as_uint(tb);
+    const float d = __fmaf_rn(x[e], rcp, -(tb - kRound));
+    near_tie |= fabsf(d) > kNear && !((bits >> e) & 1u);
   }
-  near_tie &= ~bits;
   if (near_tie) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if ((near_tie >> e) & 1u) qv[e] = __float2int_rn(__fdiv_rn(x[e], s));
+    for (int e = 0; e < 8; ++e) {
+      const float tb = __fmaf_rn(x[e], rcp, kRound);
+      const float d = __fmaf_rn(x[e], rcp, -(tb - kRound));
+      if (fabsf(d) > kNear && !((bits >> e) & 1u))
+        qb[e] = static_cast<uint32_t>(__float2int_rn(__fdiv_rn(x[e], s)));
+    }
   }
-  const uint32_t lo = __byte_perm(__byte_perm(qv[0], qv[1], 0x0040), __byte_perm(qv[2], qv[3], 0x0040), 0x5410);
-  const uint32_t hi = __byte_perm(__byte_perm(qv[4], qv[5], 0x0040), __byte_perm(qv[6], qv[7], 0x0040), 0x5410);
+  const uint32_t lo = __byte_perm(__byte_perm(qb[0], qb[1], 0x0040), __byte_perm(qb[2], qb[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(qb[4], qb[5], 0x0040), __byte_perm(qb[6], qb[7], 0x0040), 0x5410);
   return make_uint2(lo & keep_mask(bits & 0xFu), hi & keep_mask(bits >> 4));
 }
 
@@ -142,45 +149,55 @@ cudaError_t launch_quant_weight(const __half* W, int N, int K, int8_t* Wq, float
 
 // ------------------------------------------------------------------ outlier columns
 //
-// Block (strip, rb) takes columns [64 strip, +64) of rows [256 rb, +256): thread (r, c) =
-// (tid / 8, tid % 8) reads the 16-byte chunk c of the strip in rows 256 rb + r + 32 u,
-// u = 0..7, all eight loads in flight.  The block's column maxima (fp16, exact) go to
-// pmax[rb][column]; the last block of the strip to arrive (counted in strip[s], which it
-// sets back to zero) takes the maximum over the row blocks and writes the strip's two mask
-// words.  No two blocks write the same word, so the mask needs no clearing.
+// A cluster of 8 CTAs owns a strip of 64 columns; CTA r of the cluster takes rows
+// r, r + 8, ...: thread (l, c) = (tid / 8, tid % 8) reads the 16-byte chunk c of the strip in
+// 16 of those rows at a time (all 16 loads in flight; one batch covers M <= 4096).  Each CTA reduces its column maxima
+// (fp16, exact) into its shared memory; after one cluster barrier CTA 0 takes the maximum over
+// the 8 CTAs through distributed shared memory and writes the strip's two mask words.  No two
+// clusters write the same word, so the mask needs no clearing.
 
 constexpr int kCMThreads = 256;
-constexpr int kCMRowLanes = kCMThreads / 8;           // 32
-constexpr int kCMUnroll = kColRowBlock / kCMRowLanes;  // 8
+constexpr int kCMCluster = 8;
+constexpr int kCMStrip = 64;                       // columns per cluster
+constexpr int kCMRowLanes = kCMThreads / 8;        // 32 row lanes x 8 chunks of 8 columns
+constexpr int kCMUnroll = 8;                       // loads in flight per thread
+
+__device__ __forceinline__ uint32_t cm_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
 
 __global__ void __launch_bounds__(kCMThreads) colmask_kernel(const __half* __restrict__ X, int M,
                                                              int K, float threshold,
-                                                             uint32_t* __restrict__ mask,
-                                                             __half* __restrict__ pmax,
-                                                             int32_t* __restrict__ strip_cnt) {
+                                                             uint32_t* __restrict__ mask) {
   __shared__ __half2 red[kCMThreads / 32][8][4];
-  __shared__ int last;
+  __shared__ __half cmax_local[kCMStrip];  // this CTA's column maxima (read by CTA 0)
   grid_dependency_wait();
-  const int strip = blockIdx.x, rb = blockIdx.y, nrb = gridDim.y;
-  const int c = threadIdx.x & 7, r = threadIdx.x >> 3;
-  const int col0 = strip * kColStrip + c * 8;
+  const int strip = blockIdx.x / kCMCluster;
+  const int rank = static_cast<int>(cm_cluster_rank());
+  const int c = threadIdx.x & 7, l = threadIdx.x >> 3;
+  const int col0 = strip * kCMStrip + c * 8;
   __half2 m[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) m[e] = __float2half2_rn(0.0f);
   if (col0 < K) {  // K % 8 == 0: a chunk is entirely inside or outside the matrix
-    uint4 v[kCMUnroll];
+    // rows i = rank + 8 (l + 32 u): consecutive lanes of a warp read neighbouring chunks
+    for (int base = rank + kCMCluster * l; base < M; base += kCMCluster * kCMRowLanes * kCMUnroll) {
+      uint4 v[kCMUnroll];
 #pragma unroll
-    for (int u = 0; u < kCMUnroll; ++u) {
-      const int i = rb * kColRowBlock + r + u * kCMRowLanes;
-      v[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (i < M) v[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(i) * K + col0));
-    }
+      for (int u = 0; u < kCMUnroll; ++u) {
+        const int i = base + u * kCMCluster * kCMRowLanes;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < M) v[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(i) * K + col0));
+      }
 #pragma unroll
-    for (int u = 0; u < kCMUnroll; ++u) {
-      m[0] = habs2_max(m[0], v[u].x);
-      m[1] = habs2_max(m[1], v[u].y);
-      m[2] = habs2_max(m[2], v[u].z);
-      m[3] = habs2_max(m[3], v[u].w);
+      for (int u = 0; u < kCMUnroll; ++u) {
+        m[0] = habs2_max(m[0], v[u].x);
+        m[1] = habs2_max(m[1], v[u].y);
+        m[2] = habs2_max(m[2], v[u].z);
+        m[3] = habs2_max(m[3], v[u].w);
+      }
     }
   }
   grid_launch_dependents();
@@ -196,7 +213,7 @@ __global__ void __launch_bounds__(kCMThreads) colmask_kernel(const __half* __res
     for (int e = 0; e < 4; ++e) red[warp][lane][e] = m[e];
   }
   __syncthreads();
-  if (threadIdx.x < kColStrip) {  // thread j: column 64 strip + j
+  if (threadIdx.x < kCMStrip) {  // thread j: column 64 strip + j
     const int j = threadIdx.x, cg = j / 8, ce = (j % 8) / 2, hi = j % 2;
     __half h = __float2half_rn(0.0f);
 #pragma unroll
@@ -204,44 +221,51 @@ __global__ void __launch_bounds__(kCMThreads) colmask_kernel(const __half* __res
       const __half2 v = red[w][cg][ce];
       h = __hmax(h, hi ? __high2half(v) : __low2half(v));
     }
-    const int col = strip * kColStrip + j;
-    if (col < K) pmax[static_cast<size_t>(rb) * K + col] = h;
-    __threadfence();
+    cmax_local[j] = h;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    const int done = atomicAdd(&strip_cnt[strip], 1);
-    last = done == nrb - 1;
-  }
-  __syncthreads();
-  if (!last) return;
-  // the strip's last block: every row block's maxima are in pmax
-  __threadfence();
-  if (threadIdx.x < kColStrip) {
-    const int col = strip * kColStrip + threadIdx.x;
-    float cmax = 0.0f;
-    if (col < K)
-      for (int b = 0; b < nrb; ++b)
-        cmax = fmaxf(cmax, __half2float(__ldcg(pmax + static_cast<size_t>(b) * K + col)));
-    const uint32_t bits = __ballot_sync(0xffffffffu, cmax > threshold);
+  // warp 0 releases the CTA's shared-memory writes for all threads (cumulative); every warp
+  // arrives with one instruction
+  if (warp == 0) asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+  else asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+  if (rank == 0 && threadIdx.x < kCMStrip) {  // whole warps 0, 1
+    const uint32_t local = static_cast<uint32_t>(__cvta_generic_to_shared(&cmax_local[threadIdx.x]));
+    unsigned short hv[kCMCluster];
+#pragma unroll
+    for (int q = 0; q < kCMCluster; ++q) {
+      uint32_t remote;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(q));
+      asm volatile("ld.shared::cluster.u16 %0, [%1];" : "=h"(hv[q]) : "r"(remote));
+    }
+    float cm = 0.0f;
+#pragma unroll
+    for (int q = 0; q < kCMCluster; ++q) cm = fmaxf(cm, __half2float(__ushort_as_half(hv[q])));
+    const uint32_t bits = __ballot_sync(0xffffffffu, cm > threshold);
     const int word = strip * 2 + threadIdx.x / 32;
-    if ((threadIdx.x & 31) == 0 && word * 32 < K) mask[word] = bits;
+    if (lane == 0 && word * 32 < K) mask[word] = bits;
   }
-  if (threadIdx.x == 0) strip_cnt[strip] = 0;
+  // no CTA leaves while CTA 0 may still read its shared memory
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
 
 cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint32_t* mask,
-                           __half* pmax, int32_t* strip, cudaStream_t stream, bool pdl) {
+                           cudaStream_t stream, bool pdl) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((K + kColStrip - 1) / kColStrip, (M + kColRowBlock - 1) / kColRowBlock);
+  cfg.gridDim = dim3(((K + kCMStrip - 1) / kCMStrip) * kCMCluster);
   cfg.blockDim = dim3(kCMThreads);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kCMCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, colmask_kernel, X, M, K, threshold, mask, pmax, strip);
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, colmask_kernel, X, M, K, threshold, mask);
 }
 
 // ------------------------------------------------------------------ rows + outlier operands
@@ -464,10 +488,11 @@ __host__ __device__ inline int rowquant_tpr(int K) {
 __global__ void __launch_bounds__(kRQThreads) rowquant_kernel(const RowQuantArgs a, int row_blocks) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
   RowQuantShared& S = *reinterpret_cast<RowQuantShared*>(rq_smem);
-  grid_dependency_wait();
   const int words = (a.K + 31) / 32;
   const int tpr = rowquant_tpr(a.K);
-  // the rows' loads go out before the mask prologue, which waits on its own loads
+  // The rows' loads go out before the wait on the column search: X is not written by that
+  // kernel, and whatever wrote X was complete before the column search (which waited for it)
+  // let this launch start.
   const bool row_block = static_cast<int>(blockIdx.x) < row_blocks;
   const int chunks = a.K / 8;
   uint4 v[kRQRegChunks];
@@ -481,6 +506,7 @@ __global__ void __launch_bounds__(kRQThreads) rowquant_kernel(const RowQuantArgs
       if (i < a.M && c < chunks) v[u] = __ldg(row + c);
     }
   }
+  grid_dependency_wait();  // the outlier mask is complete from here on
   load_mask_prefix(S, a.mask, words);
   grid_launch_dependents();
   if (blockIdx.x == 0) {
