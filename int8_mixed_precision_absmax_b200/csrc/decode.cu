@@ -84,12 +84,11 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-// Remote shared-memory loads; ordered after the writes they read by a cluster barrier (volatile:
-// they must not move above it).  Callers issue a batch before using any result.
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
+// Remote shared-memory stores and loads, ordered against the other side by a cluster barrier
+// (volatile: they must not move across it).  Callers issue a batch of loads before using any
+// result.
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 __device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
   uint4 v;
@@ -202,8 +201,8 @@ __device__ __forceinline__ uint32_t mask2(uint32_t word, uint32_t bits, int h) {
 
 struct DecodeShared {
   uint64_t full[kDWarps];      // one weight box per 16-channel tile
-  float part[kDWarps][kDTok];  // row maxima of this CTA's slice, per warp
-  float slice_max[kDTok];      // row maxima of this CTA's slice (read cluster-wide)
+  float part[kDWarps][kDTok];   // row maxima of this CTA's slice, per warp
+  float all_max[kDSplit][kDTok];  // row maxima of every slice (written by the slice's CTA)
   float sx[kDTok];
   float rcp[kDTok];
   int zero_row[kDTok];
@@ -325,13 +324,17 @@ __global__ void __launch_bounds__(kDThreads, 3)
     sh.part[warp][2 * p + 1] = rm1;
   }
   __syncthreads();
-  if (tid < kDTok) {
+  if (warp == 0) {
+    // this slice's row maxima into every CTA of the cluster (lane: token lane % 8, CTAs
+    // lane / 8 and lane / 8 + 4); warp 0's release below covers its own remote stores
+    const int i = lane % kDTok;
     float m = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kDWarps; ++w) m = fmaxf(m, sh.part[w][tid]);
-    sh.slice_max[tid] = m;
+    for (int w = 0; w < kDWarps; ++w) m = fmaxf(m, sh.part[w][i]);
+    const uint32_t local = smem_addr(&sh.all_max[r][i]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) st_cluster_f32(map_rank(local, lane / kDTok + 4 * h), m);
   }
-  __syncthreads();
   cluster_arrive_cta();
 
   // this warp's k-blocks and the k-steps among them holding an outlier column (bit
@@ -360,13 +363,9 @@ __global__ void __launch_bounds__(kDThreads, 3)
   cluster_wait();  // every slice's row maxima are in its shared memory
 
   if (tid < kDTok) {
-    const uint32_t local = smem_addr(&sh.slice_max[tid]);
-    float mv[kDSplit];
-#pragma unroll
-    for (int s = 0; s < kDSplit; ++s) mv[s] = ld_cluster_f32(map_rank(local, s));
     float m = 0.0f;
 #pragma unroll
-    for (int s = 0; s < kDSplit; ++s) m = fmaxf(m, mv[s]);
+    for (int s = 0; s < kDSplit; ++s) m = fmaxf(m, sh.all_max[s][tid]);
     const float sc = __fdiv_rn(m, 127.0f);
     sh.sx[tid] = tid < M ? sc : 0.0f;
     sh.rcp[tid] = (tid < M && m > 0.0f) ? __frcp_rn(sc) : 0.0f;
@@ -468,36 +467,44 @@ __global__ void __launch_bounds__(kDThreads, 3)
     stage_p[c1 + 1] = pf[m][3];
   }
   __syncthreads();
+  // sum over the k-parts of each tile pair, in place into the part-0 slots: stage[pair * kParts]
+  for (int e = tid; e < P * 32 * kDTok; e += kDThreads) {
+    const int pr = e / (32 * kDTok), off = e % (32 * kDTok);
+    int32_t si = stage_i[(pr * kParts) * 32 * kDTok + off];
+    float sp = stage_p[(pr * kParts) * 32 * kDTok + off];
+#pragma unroll
+    for (int h = 1; h < kParts; ++h) {
+      si += stage_i[(pr * kParts + h) * 32 * kDTok + off];
+      sp += stage_p[(pr * kParts + h) * 32 * kDTok + off];
+    }
+    stage_i[(pr * kParts) * 32 * kDTok + off] = si;
+    stage_p[(pr * kParts) * 32 * kDTok + off] = sp;
+  }
+  __syncthreads();
   cluster_arrive_cta();
   cluster_wait();  // every slice's partial sums are in its shared memory
 
   // ---- CTA r finishes channels [r * kRed, (r + 1) * kRed) of the group.  Thread (channel,
-  // token quad, kind) sums the int32 (kind 0) or fp32 (kind 1) partials of the 8 slices and
-  // the k-parts in a fixed order; the two kinds meet through a shuffle.
+  // token quad, kind) sums the int32 (kind 0) or fp32 (kind 1) partials of the 8 slices in a
+  // fixed order; the two kinds meet through a shuffle.
   if (tid < 4 * kRed) {  // whole warps: 4 * kRed is 64 or 32
     const int kind = tid & 1, quad = (tid >> 1) & 1, cl = r * kRed + (tid >> 2);
     const int pr = cl / 32, cr = cl % 32;
     const uint8_t* stage = kind ? reinterpret_cast<const uint8_t*>(stage_p)
                                 : reinterpret_cast<const uint8_t*>(stage_i);
-    uint4 v[kParts][kDSplit];
+    uint4 v[kDSplit];
+    const uint32_t local = smem_addr(stage + ((((pr * kParts) * 32 + cr) * kDTok + 4 * quad) * 4));
 #pragma unroll
-    for (int h = 0; h < kParts; ++h) {
-      const uint32_t local =
-          smem_addr(stage + ((((pr * kParts + h) * 32 + cr) * kDTok + 4 * quad) * 4));
-#pragma unroll
-      for (int q = 0; q < kDSplit; ++q) v[h][q] = ld_cluster_v4(map_rank(local, q));
-    }
+    for (int q = 0; q < kDSplit; ++q) v[q] = ld_cluster_v4(map_rank(local, q));
     uint32_t sum[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int h = 0; h < kParts; ++h)
+    for (int q = 0; q < kDSplit; ++q) {
+      const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
 #pragma unroll
-      for (int q = 0; q < kDSplit; ++q) {
-        const uint32_t w[4] = {v[h][q].x, v[h][q].y, v[h][q].z, v[h][q].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          sum[e] = kind ? __float_as_uint(__uint_as_float(sum[e]) + __uint_as_float(w[e]))
-                        : sum[e] + w[e];
-      }
+      for (int e = 0; e < 4; ++e)
+        sum[e] = kind ? __float_as_uint(__uint_as_float(sum[e]) + __uint_as_float(w[e]))
+                      : sum[e] + w[e];
+    }
     uint32_t other[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) other[e] = __shfl_xor_sync(0xffffffffu, sum[e], 1);
