@@ -122,8 +122,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
 
-  // Everything above overlaps the previous kernel; inputs are read only after this.
+  // Everything above overlaps the previous kernel; inputs are read only after this.  The next
+  // launch may then start its own prologue (it waits for this grid before reading anything).
   grid_dependency_wait();
+  grid_launch_dependents();
 
   const int M = args.M, N = args.N, K = args.K;
   const int n_out = args.n_out ? *args.n_out : 0;

@@ -173,11 +173,22 @@ __global__ void __launch_bounds__(kCMThreads) colmask_kernel(const __half* __res
                                                              uint32_t* __restrict__ mask) {
   __shared__ __half2 red[kCMThreads / 32][8][4];
   __shared__ __half cmax_local[kCMStrip];  // this CTA's column maxima (read by CTA 0)
-  grid_dependency_wait();
   const int strip = blockIdx.x / kCMCluster;
   const int rank = static_cast<int>(cm_cluster_rank());
   const int c = threadIdx.x & 7, l = threadIdx.x >> 3;
   const int col0 = strip * kCMStrip + c * 8;
+  // Ask L2 for this CTA's rows of the strip before waiting for the previous launch.  L2 is
+  // where global memory is kept coherent, so this is safe even while that launch may still be
+  // writing X: its stores land in the same lines, and X is read only after the wait.
+  if (strip * kCMStrip < K) {
+    const int seg = min(kCMStrip, K - strip * kCMStrip) * 2;  // bytes of the row segment
+    for (int i = rank + kCMCluster * threadIdx.x; i < M; i += kCMCluster * kCMThreads)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                       reinterpret_cast<uint64_t>(X + static_cast<size_t>(i) * K + strip * kCMStrip)),
+                   "r"(seg)
+                   : "memory");
+  }
+  grid_dependency_wait();
   __half2 m[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) m[e] = __float2half2_rn(0.0f);
