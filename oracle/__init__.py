@@ -54,9 +54,11 @@ def _load():
             lib.oracle_outlier_weights.argtypes = [p, p, i64, i64, p, i32, p]
             lib.oracle_linear_forward.argtypes = [p, i64, i64, p, p, p, i64, f32, p]
             lib.oracle_linear_forward_rows.argtypes = [p, i64, i64, p, p, p, i64, f32, p, i64, p, p]
+            lib.oracle_linear_forward_rows_w16.argtypes = [p, i64, i64, p, p, p, p, i64, f32, p,
+                                                           i64, p, p]
             for name in ("oracle_quant_weight", "oracle_outlier_columns", "oracle_quantize_rows",
                          "oracle_gemm_i32", "oracle_outlier_weights", "oracle_linear_forward",
-                         "oracle_linear_forward_rows"):
+                         "oracle_linear_forward_rows", "oracle_linear_forward_rows_w16"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -150,6 +152,30 @@ def linear_forward(X, Wq, sw, bias, threshold: float):
     _check(_load().oracle_linear_forward(_ptr(X), M, K, _ptr(Wq), _ptr(sw), _ptr(b), N,
                                          float(threshold), _ptr(Y)), "oracle_linear_forward")
     return Y
+
+
+def linear_forward_rows_w16(X, Wq, sw, W16, bias, threshold: float, rows):
+    """As linear_forward_rows, with the outlier columns' weights taken from the kept fp16
+    weights W16 (has_fp16_weights=True)."""
+    X = _c(X, np.float16)
+    Wq = _c(Wq, np.int8)
+    sw = _c(sw, np.float32)
+    W16 = _c(W16, np.float16)
+    b = None if bias is None else _c(bias, np.float16)
+    rows = _c(rows, np.int64)
+    M, K = X.shape
+    N = Wq.shape[0]
+    Y = np.empty((len(rows), N), np.float16)
+    A = np.empty((len(rows), N), np.int32)
+    _check(_load().oracle_linear_forward_rows_w16(_ptr(X), M, K, _ptr(Wq), _ptr(sw), _ptr(W16),
+                                                  _ptr(b), N, float(threshold), _ptr(rows),
+                                                  len(rows), _ptr(Y), _ptr(A)),
+           "oracle_linear_forward_rows_w16")
+    return Y, A
+
+
+def linear_forward_w16(X, Wq, sw, W16, bias, threshold: float):
+    return linear_forward_rows_w16(X, Wq, sw, W16, bias, threshold, np.arange(X.shape[0]))[0]
 
 
 def linear_forward_rows(X, Wq, sw, bias, threshold: float, rows):

@@ -201,10 +201,12 @@ int oracle_outlier_weights(const int8_t *Wq, const float *w_scale, int64_t N, in
 
 /* ------------------------------------------------------------------ the layer */
 
-int oracle_linear_forward_rows(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,
-                               const float *w_scale, const uint16_t *bias, int64_t N,
-                               float threshold, const int64_t *rows, int64_t n_rows,
-                               uint16_t *Y_rows, int32_t *A_rows)
+/* W16 (nullable): the layer's own fp16 weights [N, K]; when given, the outlier columns take
+ * their weights from it instead of rebuilding them from the int8 weights. */
+static int forward_rows(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,
+                        const float *w_scale, const uint16_t *W16, const uint16_t *bias,
+                        int64_t N, float threshold, const int64_t *rows, int64_t n_rows,
+                        uint16_t *Y_rows, int32_t *A_rows)
 {
     if (!X || !Wq || !w_scale || !rows || !Y_rows || M <= 0 || N <= 0 || K <= 0 || n_rows < 0)
         return ORACLE_EINVAL;
@@ -223,7 +225,10 @@ int oracle_linear_forward_rows(const uint16_t *X, int64_t M, int64_t K, const in
     if (status == 0 && n_out > 0) {
         W_hat = (uint16_t *)malloc((size_t)N * (size_t)n_out * sizeof(uint16_t));
         if (!W_hat) status = ORACLE_EINVAL;
-        else status = oracle_outlier_weights(Wq, w_scale, N, K, cols, n_out, W_hat);
+        else if (W16) {
+            for (int64_t n = 0; n < N; ++n)
+                for (int32_t o = 0; o < n_out; ++o) W_hat[n * n_out + o] = W16[n * K + cols[o]];
+        } else status = oracle_outlier_weights(Wq, w_scale, N, K, cols, n_out, W_hat);
     }
 
     if (status == 0) {
@@ -255,6 +260,26 @@ int oracle_linear_forward_rows(const uint16_t *X, int64_t M, int64_t K, const in
     free(cols);
     free(mask);
     return status;
+}
+
+int oracle_linear_forward_rows(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,
+                               const float *w_scale, const uint16_t *bias, int64_t N,
+                               float threshold, const int64_t *rows, int64_t n_rows,
+                               uint16_t *Y_rows, int32_t *A_rows)
+{
+    return forward_rows(X, M, K, Wq, w_scale, NULL, bias, N, threshold, rows, n_rows, Y_rows,
+                        A_rows);
+}
+
+int oracle_linear_forward_rows_w16(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,
+                                   const float *w_scale, const uint16_t *W16,
+                                   const uint16_t *bias, int64_t N, float threshold,
+                                   const int64_t *rows, int64_t n_rows, uint16_t *Y_rows,
+                                   int32_t *A_rows)
+{
+    if (!W16) return ORACLE_EINVAL;
+    return forward_rows(X, M, K, Wq, w_scale, W16, bias, N, threshold, rows, n_rows, Y_rows,
+                        A_rows);
 }
 
 int oracle_linear_forward(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,

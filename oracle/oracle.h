@@ -75,6 +75,16 @@ int oracle_linear_forward_rows(const uint16_t *X, int64_t M, int64_t K, const in
                                float threshold, const int64_t *rows, int64_t n_rows,
                                uint16_t *Y_rows, int32_t *A_rows);
 
+/* The layer that keeps its fp16 weights ([P5] section "如何在 PyTorch 2.9 中启用 LLM.int8
+ * 推理": has_fp16_weights=True): as oracle_linear_forward_rows, except that the fp16 term uses
+ * the kept weights of the outlier columns, W_hat[n,j] = W16[n,j], instead of rebuilding them
+ * from Wq.  W16: binary16 [N, K], the weights Wq and w_scale were quantized from. */
+int oracle_linear_forward_rows_w16(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,
+                                   const float *w_scale, const uint16_t *W16,
+                                   const uint16_t *bias, int64_t N, float threshold,
+                                   const int64_t *rows, int64_t n_rows, uint16_t *Y_rows,
+                                   int32_t *A_rows);
+
 #ifdef __cplusplus
 }
 #endif
