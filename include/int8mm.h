@@ -102,6 +102,21 @@ int int8_linear_forward(const void *X, int M, int K, const int8_t *Wq, const flo
                         size_t ws_bytes, int8mm_stream_t stream);
 
 /*
+ * The layer that keeps its fp16 weights ([P5] section "如何在 PyTorch 2.9 中启用 LLM.int8
+ * 推理", has_fp16_weights=True): as int8_linear_forward, except that the outlier term reads
+ * the layer's own fp16 weights, sum_{j in O} X[i,j] * W16[n,j], in place of the rebuilt
+ * W_hat = fp16(Wq * w_scale).  The int8 term is unchanged (Wq and w_scale still come from
+ * int8_quant_weight of the same weights).
+ *   W16        [in]  binary16 [N, K], row-major, 16-byte aligned, read only at the outlier
+ *                    columns; NULL is rejected (INT8MM_ERR_NULL)
+ * Every other argument, the workspace and the error codes are as for int8_linear_forward.
+ */
+int int8_linear_forward_fp16w(const void *X, int M, int K, const int8_t *Wq,
+                              const float *w_scale, const void *W16, const void *bias, int N,
+                              float threshold, void *Y, void *workspace, size_t ws_bytes,
+                              int8mm_stream_t stream);
+
+/*
  * The two halves of int8_linear_forward, for callers that time or schedule them apart:
  * int8_linear_forward is exactly int8_linear_quantize followed by int8_linear_matmul with
  * the same arguments, workspace and stream.  Arguments are as for int8_linear_forward.

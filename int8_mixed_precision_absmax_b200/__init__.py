@@ -27,7 +27,7 @@ __all__ = [
     "int8_linear_quantize", "int8_linear_matmul", "int8_linear_forward_acc",
     "int8_quantize_rows", "int8_gemm_i32", "int8_outlier_weights",
     "int8_read_device_status", "int8_status_string", "int8_linear_forward_noalloc",
-    "Int8Linear", "DEFAULT_THRESHOLD",
+    "int8_linear_forward_fp16w", "Int8Linear", "DEFAULT_THRESHOLD",
 ]
 
 DEFAULT_THRESHOLD = 6.0
@@ -72,10 +72,11 @@ def load_library():
         lib.int8_outlier_weights.argtypes = [p, p, i, i, p, p, p, p]
         lib.int8_read_device_status.argtypes = [p, p]
         lib.int8_linear_forward_noalloc.argtypes = [p, i, i, p, p, p, i, f, p, p, p]
+        lib.int8_linear_forward_fp16w.argtypes = [p, i, i, p, p, p, p, i, f, p, p, sz, p]
         for name in ("int8_quant_weight", "int8_linear_forward", "int8_linear_quantize",
                      "int8_linear_matmul", "int8_linear_forward_acc", "int8_quantize_rows",
                      "int8_gemm_i32", "int8_outlier_weights", "int8_read_device_status",
-                     "int8_linear_forward_noalloc"):
+                     "int8_linear_forward_noalloc", "int8_linear_forward_fp16w"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -164,6 +165,36 @@ def int8_linear_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor
         _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(bias), N, float(threshold), _ptr(Y),
         _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream, X.device))),
         "int8_linear_forward")
+    return Y
+
+
+def int8_linear_forward_fp16w(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                              W16: torch.Tensor, bias: torch.Tensor | None,
+                              threshold: float = DEFAULT_THRESHOLD, Y: torch.Tensor | None = None,
+                              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """int8_linear_forward for a layer that keeps its fp16 weights W16 [N, K]: the outlier
+    columns are multiplied by W16 itself rather than by fp16(Wq * w_scale)."""
+    _need(X, torch.float16, "X", 2)
+    _need(Wq, torch.int8, "Wq", 2)
+    _need(w_scale, torch.float32, "w_scale", 1)
+    _need(W16, torch.float16, "W16", 2)
+    M, K = X.shape
+    N = Wq.shape[0]
+    if tuple(W16.shape) != (N, K):
+        raise ValueError(f"W16 must be [{N}, {K}], got {tuple(W16.shape)}")
+    if bias is not None:
+        _need(bias, torch.float16, "bias", 1)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    _need(Y, torch.float16, "Y", 2)
+    if workspace is None:
+        n = int8_linear_workspace_size(M, N, K)
+        workspace = torch.zeros(max(n, 256), dtype=torch.uint8, device=X.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    _check(load_library().int8_linear_forward_fp16w(
+        _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(W16), _ptr(bias), N, float(threshold),
+        _ptr(Y), _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream, X.device))),
+        "int8_linear_forward_fp16w")
     return Y
 
 
@@ -301,20 +332,24 @@ def int8_read_device_status(dev_status: torch.Tensor, stream=None) -> int:
 
 
 class Int8Linear:
-    """An LLM.int8() linear layer holding int8 weights only (no fp16 copy).
+    """An LLM.int8() linear layer.
 
-    Mirrors ``Linear8bitLt(in_features, out_features, bias, has_fp16_weights=False,
-    threshold)``: the fp16 weight is quantized once per output channel at construction,
-    then every call quantizes its activations per row on the fly and routes the columns
-    whose magnitude exceeds ``threshold`` through fp16.
+    Mirrors ``Linear8bitLt(in_features, out_features, bias, has_fp16_weights, threshold)``:
+    the fp16 weight is quantized once per output channel at construction, then every call
+    quantizes its activations per row on the fly and routes the columns whose magnitude
+    exceeds ``threshold`` through fp16.  With ``has_fp16_weights=False`` (the default) only
+    the int8 weights are kept and the outlier columns use fp16(Wq * w_scale); with True the
+    layer also keeps the fp16 weight and the outlier columns use it.
     """
 
     def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None,
-                 threshold: float = DEFAULT_THRESHOLD):
+                 threshold: float = DEFAULT_THRESHOLD, has_fp16_weights: bool = False):
         if math.isnan(threshold):
             raise ValueError("threshold is NaN")
         self.out_features, self.in_features = weight.shape
-        self.Wq, self.w_scale = int8_quant_weight(weight.contiguous())
+        weight = weight.to(torch.float16).contiguous()
+        self.Wq, self.w_scale = int8_quant_weight(weight)
+        self.W16 = weight if has_fp16_weights else None
         self.bias = None if bias is None else bias.to(torch.float16).contiguous()
         self.threshold = float(threshold)
         self._workspace = None
@@ -330,6 +365,10 @@ class Int8Linear:
         lead = X.shape[:-1]
         X2 = X.reshape(-1, self.in_features).contiguous()
         ws = self._ws(X2.shape[0], X2.device)
-        Y = int8_linear_forward(X2, self.Wq, self.w_scale, self.bias, self.threshold, Y=out,
-                                workspace=ws)
+        if self.W16 is not None:
+            Y = int8_linear_forward_fp16w(X2, self.Wq, self.w_scale, self.W16, self.bias,
+                                          self.threshold, Y=out, workspace=ws)
+        else:
+            Y = int8_linear_forward(X2, self.Wq, self.w_scale, self.bias, self.threshold, Y=out,
+                                    workspace=ws)
         return Y.reshape(*lead, self.out_features)

@@ -135,8 +135,10 @@ int plan_forward(int M, int N, int K, const int8_t* Wq, const float* w_scale, vo
 
 GemvArgs gemv_args(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                    const void* bias, int N, float threshold, void* Y, int32_t* acc,
-                   void* workspace, const ForwardPlan& p, const GemvPlan& gp) {
+                   void* workspace, const ForwardPlan& p, const GemvPlan& gp,
+                   const void* W16 = nullptr) {
   GemvArgs g;
+  g.W16 = static_cast<const __half*>(W16);
   g.X = static_cast<const __half*>(X);
   g.M = M;
   g.K = K;
@@ -162,8 +164,9 @@ GemvArgs gemv_args(const void* X, int M, int K, const int8_t* Wq, const float* w
 
 SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                      const void* bias, int N, float threshold, void* Y, int32_t* acc,
-                     const ForwardPlan& p, const SmallPlan& sp) {
+                     const ForwardPlan& p, const SmallPlan& sp, const void* W16 = nullptr) {
   SmallArgs a;
+  a.W16 = static_cast<const __half*>(W16);
   a.X = static_cast<const __half*>(X);
   a.M = M;
   a.K = K;
@@ -185,7 +188,7 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
 // tile.
 int run_decode(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                const void* bias, int N, float threshold, void* Y, int32_t* acc, int32_t* status,
-               const DecodePlan& dp, cudaStream_t stream, bool pdl) {
+               const DecodePlan& dp, cudaStream_t stream, bool pdl, const void* W16 = nullptr) {
   CUtensorMap map;
   const uint64_t dims[3] = {128, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 128)};
   const uint64_t strides[2] = {static_cast<uint64_t>(K), 128};
@@ -202,6 +205,7 @@ int run_decode(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   a.threshold = effective_threshold(threshold);
   a.Wq = Wq;
   a.w_scale = w_scale;
+  a.W16 = static_cast<const __half*>(W16);
   a.bias = static_cast<const __half*>(bias);
   a.Y = static_cast<__half*>(Y);
   a.acc = acc;
@@ -212,7 +216,7 @@ int run_decode(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
 
 int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale, int N,
                  float threshold, void* workspace, const ForwardPlan& p, cudaStream_t stream,
-                 bool pdl_first) {
+                 bool pdl_first, const void* W16 = nullptr) {
   if (M <= kSmallMP) {
     if (plan_decode(M, N, K).fits) return INT8MM_OK;  // one kernel does everything
     const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
@@ -240,6 +244,7 @@ int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_s
   rq.n_out = p.header + 1;
   rq.Wq = Wq;
   rq.w_scale = w_scale;
+  rq.W16 = static_cast<const __half*>(W16);
   rq.wo = p.wo;
   rq.N = N;
   rq.status = p.header;
@@ -248,16 +253,17 @@ int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_s
 
 int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                const void* bias, int N, float threshold, void* Y, int32_t* acc,
-               void* workspace, const ForwardPlan& p, cudaStream_t stream, bool pdl) {
+               void* workspace, const ForwardPlan& p, cudaStream_t stream, bool pdl,
+               const void* W16 = nullptr) {
   if (M <= kSmallMP) {
     const DecodePlan dp = plan_decode(M, N, K);
     if (dp.fits)
       return run_decode(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p.header, dp, stream,
-                        pdl);
+                        pdl, W16);
     const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
     if (gp.fits) {
       const GemvArgs g = gemv_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace,
-                                   p, gp);
+                                   p, gp, W16);
       // Wq viewed as [K/128 k-blocks][N rows][128 bytes]: one box is 32 rows x 8 k-blocks,
       // each k-block landing as a 128-byte-swizzled 32 x 128 tile
       CUtensorMap map;
@@ -272,7 +278,7 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   }
   if (small_path_fits(M, K)) {
     const SmallPlan sp = plan_small(M, N, K);
-    const SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p, sp);
+    const SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p, sp, W16);
     CUtensorMap map;
     if (!encode_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kSmallBN))
       return INT8MM_ERR_CUDA;
@@ -302,17 +308,20 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
 
 int forward_impl(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                  const void* bias, int N, float threshold, void* Y, int32_t* acc,
-                 void* workspace, size_t ws_bytes, cudaStream_t stream) {
+                 void* workspace, size_t ws_bytes, cudaStream_t stream,
+                 const void* W16 = nullptr) {
   if (!X || !Y) return INT8MM_ERR_NULL;
-  if (!aligned16(X) || !aligned16(Y) || (bias && !aligned16(bias)) || (acc && !aligned16(acc)))
+  if (!aligned16(X) || !aligned16(Y) || (bias && !aligned16(bias)) || (acc && !aligned16(acc)) ||
+      (W16 && !aligned16(W16)))
     return INT8MM_ERR_ALIGN;
   if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
   ForwardPlan p;
   int rc = plan_forward(M, N, K, Wq, w_scale, workspace, ws_bytes, p);
   if (rc) return rc;
-  if ((rc = run_quantize(X, M, K, Wq, w_scale, N, threshold, workspace, p, stream, true)))
+  if ((rc = run_quantize(X, M, K, Wq, w_scale, N, threshold, workspace, p, stream, true, W16)))
     return rc;
-  return run_matmul(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace, p, stream, true);
+  return run_matmul(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace, p, stream, true,
+                    W16);
 }
 
 }  // namespace
@@ -324,6 +333,15 @@ int int8_linear_forward(const void* X, int M, int K, const int8_t* Wq, const flo
                         size_t ws_bytes, int8mm_stream_t stream) {
   return forward_impl(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, workspace, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int int8_linear_forward_fp16w(const void* X, int M, int K, const int8_t* Wq,
+                              const float* w_scale, const void* W16, const void* bias, int N,
+                              float threshold, void* Y, void* workspace, size_t ws_bytes,
+                              int8mm_stream_t stream) {
+  if (!W16) return INT8MM_ERR_NULL;
+  return forward_impl(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, workspace, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), W16);
 }
 
 int int8_linear_forward_acc(const void* X, int M, int K, const int8_t* Wq,

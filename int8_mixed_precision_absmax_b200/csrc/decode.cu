@@ -434,10 +434,28 @@ __global__ void __launch_bounds__(kDThreads, 3)
           const uint32_t b2 = mask2(xr.z, fb, 2), b3 = mask2(xr.w, fb, 3);
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
-            mma_f16_16816(pf[m], what2(w[m][0].x, 0, swr[m][0]), what2(w[m][1].x, 0, swr[m][1]),
-                          what2(w[m][0].x, 1, swr[m][0]), what2(w[m][1].x, 1, swr[m][1]), b0, b1);
-            mma_f16_16816(pf[m], what2(w[m][0].y, 0, swr[m][0]), what2(w[m][1].y, 0, swr[m][1]),
-                          what2(w[m][0].y, 1, swr[m][0]), what2(w[m][1].y, 1, swr[m][1]), b2, b3);
+            uint32_t ha[2][4];  // rows g, g + 8: fp16 weights of this step's 8 columns
+            if (a.W16) {        // the layer's kept fp16 weights
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int n = n0 + 32 * pair + 16 * m + 8 * h + g;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (n < N)
+                  v = __ldg(reinterpret_cast<const uint4*>(
+                      a.W16 + static_cast<size_t>(n) * K + col0 + kb * 128 + 32 * j + 8 * tig));
+                ha[h][0] = v.x; ha[h][1] = v.y; ha[h][2] = v.z; ha[h][3] = v.w;
+              }
+            } else {            // fp16(Wq * w_scale) from the resident int8 tile
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                ha[h][0] = what2(w[m][h].x, 0, swr[m][h]);
+                ha[h][1] = what2(w[m][h].x, 1, swr[m][h]);
+                ha[h][2] = what2(w[m][h].y, 0, swr[m][h]);
+                ha[h][3] = what2(w[m][h].y, 1, swr[m][h]);
+              }
+            }
+            mma_f16_16816(pf[m], ha[0][0], ha[1][0], ha[0][1], ha[1][1], b0, b1);
+            mma_f16_16816(pf[m], ha[0][2], ha[1][2], ha[0][3], ha[1][3], b2, b3);
           }
         }
       }

@@ -494,16 +494,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
     float P = 0.0f;
     for (int o = 0; o < n_out; ++o) {
       const int j = o < staged ? sh.cols[o] : __ldcg(a.cols + o);
-      int8_t q;
-      if (resident) {
-        const int kb = j / 128;
-        const uint8_t* tile = ring + static_cast<size_t>(kb / kBoxKb) * kBoxBytes +
-                              (kb % kBoxKb) * (kCh * 128);
-        q = static_cast<int8_t>(tile[sw128_offset(c, j % 128)]);
+      float wv;
+      if (a.W16) {
+        wv = __half2float(a.W16[static_cast<size_t>(n) * a.K + j]);
       } else {
-        q = a.Wq[static_cast<size_t>(n) * a.K + j];
+        int8_t q;
+        if (resident) {
+          const int kb = j / 128;
+          const uint8_t* tile = ring + static_cast<size_t>(kb / kBoxKb) * kBoxBytes +
+                                (kb % kBoxKb) * (kCh * 128);
+          q = static_cast<int8_t>(tile[sw128_offset(c, j % 128)]);
+        } else {
+          q = a.Wq[static_cast<size_t>(n) * a.K + j];
+        }
+        wv = __half2float(__float2half_rn(static_cast<float>(q) * swn));
       }
-      const float wv = __half2float(__float2half_rn(static_cast<float>(q) * swn));
       P += wv * __half2float(o < staged ? sh.xo[o][i] : a.xo[static_cast<size_t>(o) * kSmallMP + i]);
     }
     const float bb = sh.bias[c];

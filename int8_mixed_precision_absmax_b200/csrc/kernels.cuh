@@ -88,6 +88,7 @@ struct RowQuantArgs {
   // outlier-weight gather (extra blocks after the M row blocks); wo nullable
   const int8_t* Wq;
   const float* w_scale;
+  const __half* W16;    // nullable: the layer's fp16 weights [N, K] for the outlier columns
   __half* wo;
   int N;
   int32_t* status;
@@ -100,6 +101,7 @@ struct SmallArgs {
   float threshold;       // already clamped to >= 0
   const int8_t* Wq;
   const float* w_scale;
+  const __half* W16;     // nullable: the layer's fp16 weights [N, K] for the outlier term
   const __half* bias;
   __half* Y;
   int32_t* acc;          // nullable: also write the int32 accumulators
@@ -121,6 +123,7 @@ struct GemvArgs {
   float threshold;       // already clamped to >= 0
   const int8_t* Wq;
   const float* w_scale;
+  const __half* W16;     // nullable: the layer's fp16 weights [N, K] for the outlier term
   const __half* bias;
   __half* Y;
   int32_t* acc;          // nullable: also write the int32 accumulators
@@ -152,6 +155,7 @@ struct DecodeArgs {
   float threshold;       // already clamped to >= 0
   const int8_t* Wq;
   const float* w_scale;
+  const __half* W16;     // nullable: the layer's fp16 weights [N, K] for the outlier term
   const __half* bias;
   __half* Y;
   int32_t* acc;          // nullable: also write the int32 accumulators

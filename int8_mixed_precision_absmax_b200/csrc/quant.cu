@@ -444,7 +444,8 @@ __device__ void quantize_rows_block(const RowQuantArgs& a, RowQuantShared& S, in
   }
 }
 
-// Extra blocks: W_hat[n, r] = fp16(float(Wq[n, col(r)]) * w_scale[n]), zero-padded to 64.
+// Extra blocks: W_hat[n, r] = fp16(float(Wq[n, col(r)]) * w_scale[n]), zero-padded to 64 (or
+// the kept fp16 weight W16[n, col(r)] when the layer has one).
 // The outliers are taken in windows of kGatherSmemCols: the block lists the window's columns
 // in shared memory, then thread u writes the 8 consecutive entries (one 16-byte store) of
 // channel u / groups, group u % groups of the window.
@@ -469,15 +470,23 @@ __device__ void gather_weights(const RowQuantArgs& a, RowQuantShared& S, int wor
       const int n = static_cast<int>(u / groups);
       const int r0 = R0 + static_cast<int>(u % groups) * 8;
       uint32_t h[4] = {0u, 0u, 0u, 0u};
-      if (r0 < n_out) {
+      if (r0 < n_out && a.W16 != nullptr) {  // the layer's own fp16 weights
+        const unsigned short* hrow =
+            reinterpret_cast<const unsigned short*>(a.W16) + static_cast<size_t>(n) * a.K;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (r0 + e < n_out)
+            h[e / 2] |= static_cast<uint32_t>(hrow[S.cols[r0 + e - R0]]) << (16 * (e & 1));
+      } else if (r0 < n_out) {  // rebuilt from the int8 weights
         const float sc = a.w_scale[n];
         const int8_t* wrow = a.Wq + static_cast<size_t>(n) * a.K;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int r = r0 + e;
           if (r < n_out) {
-            const __half hv = __float2half_rn(static_cast<float>(wrow[S.cols[r - R0]]) * sc);
-            h[e / 2] |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * (e & 1));
+            const float w = static_cast<float>(wrow[S.cols[r - R0]]) * sc;
+            h[e / 2] |= static_cast<uint32_t>(__half_as_ushort(__float2half_rn(w)))
+                        << (16 * (e & 1));
           }
         }
       }

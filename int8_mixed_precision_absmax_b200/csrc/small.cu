@@ -351,8 +351,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             q0 = w0row[j];
             q1 = w1row[j];
           }
-          const float w0 = __half2float(__float2half_rn(static_cast<float>(q0) * s0));
-          const float w1 = __half2float(__float2half_rn(static_cast<float>(q1) * s1));
+          float w0 = __half2float(__float2half_rn(static_cast<float>(q0) * s0));
+          float w1 = __half2float(__float2half_rn(static_cast<float>(q1) * s1));
+          if (a.W16) {  // the layer's kept fp16 weights of the outlier column
+            w0 = g0 < a.N ? __half2float(a.W16[static_cast<size_t>(g0) * a.K + j]) : 0.0f;
+            w1 = g1 < a.N ? __half2float(a.W16[static_cast<size_t>(g1) * a.K + j]) : 0.0f;
+          }
           const __half* xc = x_slice + (j - col_begin);
 #pragma unroll
           for (int i = 0; i < kSmallMP; ++i)

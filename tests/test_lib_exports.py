@@ -87,3 +87,14 @@ def test_argument_checks_need_no_device(lib):
     assert L.int8_quantize_rows(FAKE, 4, 32, math.nan, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20,
                                 null) == -4
     assert L.int8_read_device_status(null, null) == -1
+
+
+def test_fp16_weight_entry_point_checks_its_weights(lib):
+    L = lib
+    # the kept fp16 weights are required and must be 16-byte aligned
+    assert L.int8_linear_forward_fp16w(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, FAKE, FAKE,
+                                       1 << 20, None) == -1
+    assert L.int8_linear_forward_fp16w(FAKE, 4, 32, FAKE, FAKE, ctypes.c_void_p(0x10002), None,
+                                       8, 6.0, FAKE, FAKE, 1 << 20, None) == -3
+    assert L.int8_linear_forward_fp16w(FAKE, 4, 32, FAKE, FAKE, FAKE, None, 8, math.nan, FAKE,
+                                       FAKE, 1 << 20, None) == -4
