@@ -289,8 +289,8 @@ def forward_path(M: int, N: int, K: int):
     api.cu with the plan functions of decode.cu, gemv.cu and small.cu)."""
     if M <= 8 and K % 128 == 0 and K <= 8192:
         return {"name": "decode", "launches": 1, "quantize": [],
-                "matmul": "decode_kernel (one launch: 8-CTA cluster per 128 channels, split-K, "
-                          "mma.sync int8 + fp16 outlier term, partial sums through DSMEM)"}
+                "matmul": "decode_kernel (one launch: one CTA per 32 channels over all of K, X "
+                          "statistics in every CTA, mma.sync int8 + fp16 outlier term)"}
     if M <= 16:
         if K % 128 == 0 and K <= 8192:
             return {"name": "few_tokens", "launches": 2, "quantize": ["few_quant_kernel"],

@@ -184,16 +184,14 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
 }
 
 // The one-launch few-token layer: Wq viewed as [K/128 k-blocks][N rows][128 bytes], one box
-// is 16 rows x (a slice of) k-blocks, each k-block landing as a 128-byte-swizzled 16 x 128
-// tile.
+// is 16 rows x every k-block, each k-block landing as a 128-byte-swizzled 16 x 128 tile.
 int run_decode(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                const void* bias, int N, float threshold, void* Y, int32_t* acc, int32_t* status,
                const DecodePlan& dp, cudaStream_t stream, bool pdl, const void* W16 = nullptr) {
   CUtensorMap map;
   const uint64_t dims[3] = {128, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 128)};
   const uint64_t strides[2] = {static_cast<uint64_t>(K), 128};
-  const uint32_t box[3] = {128, static_cast<uint32_t>(dp.tile_rows),
-                           static_cast<uint32_t>(dp.nqmax)};
+  const uint32_t box[3] = {128, 16, static_cast<uint32_t>(K / 128)};
   if (!encode_tmap_3d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, dims, strides, box,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return INT8MM_ERR_CUDA;
@@ -209,7 +207,6 @@ int run_decode(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   a.bias = static_cast<const __half*>(bias);
   a.Y = static_cast<__half*>(Y);
   a.acc = acc;
-  a.nqmax = dp.nqmax;
   a.status = status;
   return launch_status(launch_decode(map, a, dp, stream, pdl));
 }

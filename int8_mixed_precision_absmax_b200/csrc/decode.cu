@@ -1,38 +1,40 @@
 // decode.cu -- the LLM.int8() layer for up to 8 tokens in one launch (the decode regime).
 //
 // With M <= 8 the layer reads every byte of Wq once and does at most 8 multiply-adds per
-// byte, so its time is the weight stream and the latency of the few steps that depend on X.
-// One launch does the whole layer, built so that back-to-back layers keep HBM busy and the
-// X-dependent chain stays short:
+// byte, so its time is the weight stream plus the latency of the steps that depend on X.
+// One launch does the whole layer, and every CTA works on its own, with no exchange between
+// CTAs:
 //
-//   * A thread-block cluster of 8 CTAs owns a group of G output channels (G = 128, or 64
-//     for K > 4096) and splits K eight ways: CTA r owns the r-th eighth of the 128-byte
-//     k-blocks.  Its Wq tile (G rows x K/8 bytes, 64 KB) is copied by TMA into shared memory,
-//     one box per 16-channel MMA tile, before the CTA waits for the previous launch on the
-//     stream; the CTA then lets the next launch start.  A CTA needs about 70 KB of shared
-//     memory, so CTAs of the next layer sit beside this layer's and stream their weights
-//     while this layer computes.
-//   * CTA r reads only its slice of X.  It finds the outlier columns of the slice,
-//     max_i |x| > threshold ([P2] "8位量化实战：离群值处理与显存优化避坑指南" section 2.3)
-//     -- a column lies in one slice, so this needs no exchange -- and the row maxima over its
-//     regular columns.  The eight CTAs exchange those maxima through distributed shared
-//     memory, giving sx = max / 127 per row, and each writes q = rne(x / sx) clamped to
-//     [-127, 127], 0 in outlier columns ([P5] "PyTorch 2.9 支持 LLM.int8()" item 2), for its
-//     own slice into its own shared memory.
-//   * Each warp takes one 16-channel tile (and for K > 4096 half of the slice's k-steps) and
-//     forms acc[n, i] = sum_k Wq[n,k] q[i,k] exactly with the int8 warp-level MMA m16n8k32
-//     (16 channels x 8 tokens; a tcgen05 MMA takes the same time at N = 8 tokens as at
-//     N = 256, so at this shape it would idle).  In a k-step holding an outlier column it
-//     also runs the fp16 MMA m16n8k16 on W_hat = fp16(Wq * w_scale) and the fp16 activations
-//     of the outlier columns (zero elsewhere): the fp16 term of the decomposition, with fp32
-//     accumulation ([P5] "如何在 PyTorch 2.9 中启用 LLM.int8 推理": no fp16 weights kept).
-//   * The partial sums of the eight slices meet through distributed shared memory: CTA r
-//     sums channels [r G/8, (r+1) G/8) over the cluster in a fixed order and writes
-//     Y = fp16(acc * sx * w_scale + P + bias).
+//   * A CTA owns 16 T output channels (T = 2 for K <= 4096, else 1) and all of K.  Its Wq
+//     rows (16 T x K bytes, at most 128 KB) are copied by TMA into shared memory, one box
+//     per 16-channel MMA tile, before the CTA waits for the previous launch on the stream;
+//     the CTA then lets the next launch start.
+//   * Each CTA reads the whole of X (8 x K fp16, 64 KB at K = 4096, from L2) and finds by
+//     itself what the layer needs of it.  Thread t holds 8-column chunks of X for all 8
+//     tokens in registers, so the column maxima need no exchange: a column is an outlier
+//     when max_i |x| > threshold ([P2] "8位量化实战：离群值处理与显存优化避坑指南" section
+//     2.3).  The row maxima over the regular columns meet in one block-wide reduction, giving
+//     sx = max / 127 per row, and every thread writes q = rne(x / sx) in [-127, 127], 0 in
+//     outlier columns ([P5] "PyTorch 2.9 支持 LLM.int8()" item 2), for its chunks into shared
+//     memory.  Repeating this work in every CTA measured faster than sharing it across a
+//     thread-block cluster (the remote stores and the cluster barrier cost more than the
+//     quantization they save), and it runs while the weights are still arriving.
+//   * Warp w takes the w-th sixteenth of the k-blocks for all T tiles and forms
+//     acc[n, i] = sum_k Wq[n,k] q[i,k] exactly with the int8 warp-level MMA m16n8k32
+//     (16 channels x 8 tokens; a CTA owns 32 channels, fewer than the 64 rows a tcgen05 MMA
+//     needs).  Its k-steps holding an outlier column then run, one at a time, the fp16 MMA
+//     m16n8k16 on the outlier weights and the fp16 activations of the outlier columns (zero
+//     elsewhere, kept in shared memory since the statistics pass): the fp16 term of the
+//     decomposition, with fp32 accumulation.  The outlier weights are W_hat =
+//     fp16(Wq * w_scale) ([P5] "如何在 PyTorch 2.9 中启用 LLM.int8 推理",
+//     has_fp16_weights=False), or the layer's own fp16 weights when it keeps them.
+//   * The 16 warps' partial sums meet in shared memory; thread (token, channel) sums them in
+//     a fixed order and writes Y = fp16(acc * sx * w_scale + P + bias).
 //
-// Each thread's fragments cover 8 consecutive bytes of K per 32-wide k-step (the MMA's k
-// positions are permuted the same way in both operands, which leaves the dot product as it
-// is), so a fragment is one 8-byte shared-memory load.
+// Each lane's fragments cover 8 consecutive bytes of K per 32-wide k-step, chosen so that the
+// 16 lanes of a half-warp read 16 different bank pairs of the swizzled weight rows and of the
+// codes (the MMA's k positions are permuted the same way in both operands, which leaves the
+// dot product as it is); a fragment is one 8-byte shared-memory load.
 //
 // The weights and scales are read before the wait on the previous launch: they must not be
 // written by the launch just before this one on the stream while it can still be running.
@@ -43,60 +45,13 @@ namespace i8mm {
 
 namespace {
 
-constexpr int kDThreads = 256;
+constexpr int kDThreads = 512;
 constexpr int kDWarps = kDThreads / 32;
-constexpr int kDTok = 8;               // tokens (MMA N)
-constexpr int kDSplit = 8;             // CTAs per cluster = slices of K
-constexpr int kDMaxKb = 64;            // K <= 8192
-constexpr int kDMaxItems = 2;          // (chunk, token pair) items of the slice per thread
-constexpr size_t kDSmemBudget = 74 * 1024;  // three CTAs per SM
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// Split cluster barrier (per thread): every thread of the cluster arrives once per phase and
-// waits before arriving again.
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
-}
-// Arrive without ordering this thread's earlier memory operations: for the exit barrier, whose
-// only job is to keep this CTA's shared memory alive while its peers still read it (each
-// thread has used the values of its remote loads before it arrives), and for the threads of a
-// CTA whose shared-memory writes thread 0 releases for all of them after a __syncthreads
-// (release is cumulative).
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
-}
-// After a __syncthreads: warp 0 releases the CTA's shared-memory writes for all threads, the
-// other warps arrive relaxed.  Every warp takes one branch as a whole: a warp never splits
-// its arrival across two barrier instructions.
-__device__ __forceinline__ void cluster_arrive_cta() {
-  if (threadIdx.x < 32) cluster_arrive();
-  else cluster_arrive_relaxed();
-}
-__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-// Remote shared-memory stores and loads, ordered against the other side by a cluster barrier
-// (volatile: they must not move across it).  Callers issue a batch of loads before using any
-// result.
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
+constexpr int kDTok = 8;                // tokens (MMA N)
+constexpr int kDMaxKb = 64;             // K <= 8192
+constexpr int kDMaxTiles = 2;
+constexpr int kDOutChunks = 64;         // 8-column chunks with an outlier kept in shared memory
+constexpr size_t kDSmemMax = 227 * 1024;
 
 // Ask L2 to fetch `bytes` (a multiple of 16) at a 16-byte aligned global address.  L2 is where
 // global memory is kept coherent, so this is safe even for data the previous launch may still
@@ -111,30 +66,28 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
 }
 
-__device__ __forceinline__ float h2f(uint32_t word, int hi) {
-  return __half2float(
-      __ushort_as_half(static_cast<unsigned short>(hi ? (word >> 16) : (word & 0xFFFFu))));
+// 8 codes of one row chunk, packed little-endian, then ANDed with `keep` (zero bytes in outlier
+// columns).  rne(x * r) with r = 1/sx rounded to nearest equals rne(fl(x / sx)) unless x * r
+// lies within 2^-15 of a half-integer (the exact x * r is within 2^-17 of x / sx for
+// |x / sx| <= 128, the rounded quotient within 2^-18); there the quotient itself (__fdiv_rn)
+// is rounded.  tb = fl(x * r + 1.5 * 2^23) = 1.5 * 2^23 + rne(x * r) exactly, and as
+// 1.5 * 2^23 has a zero low byte, the low byte of tb's bits is the two's-complement code.
+// d = x * r - rne(x * r) (one more FMA, rounding error <= 2^-25) has |d| <= 1/2, so "near a
+// half-integer" is |d| > 1/2 - 2^-15, tested once for the 8 values through max |d|.  A
+// regular column has |x| <= the row maximum, so |x / sx| <= 127 (1 + 2^-22) and the code needs
+// no clamp; an outlier column may take the exact route needlessly, and its code is masked.
+__device__ __forceinline__ uint2 keep_masks(uint32_t bits) {  // bit e set -> byte e = 0
+  const uint32_t lo = ~((((bits & 0xFu) * 0x204081u) & 0x01010101u) * 0xFFu);
+  const uint32_t hi = ~((((bits >> 4) * 0x204081u) & 0x01010101u) * 0xFFu);
+  return make_uint2(lo, hi);
 }
-
-// 8 codes of one row chunk, packed little-endian, outlier columns (bits) set to 0.
-// rne(x * r) with r = 1/sx rounded to nearest equals rne(fl(x / sx)) unless x * r lies within
-// 2^-15 of a half-integer (the exact x * r is within 2^-17 of x / sx for |x / sx| <= 128, the
-// rounded quotient within 2^-18); there the quotient itself (__fdiv_rn) is rounded.
-// tb = fl(x * r + 1.5 * 2^23) = 1.5 * 2^23 + rne(x * r) exactly, and as 1.5 * 2^23 has a zero
-// low byte, the low byte of tb's bits is the two's-complement code.  d = x * r - rne(x * r)
-// (one more FMA, rounding error <= 2^-25) has |d| <= 1/2, so "near a half-integer" is
-// |d| > 1/2 - 2^-15.  A regular column has |x| <= the row maximum, so |x / sx| <=
-// 127 (1 + 2^-22) and the code needs no clamp; outlier columns are masked out after the fact.
-__device__ __forceinline__ uint32_t keep_mask(uint32_t bits4) {  // bit e set -> byte e = 0
-  return ~(((bits4 * 0x204081u) & 0x01010101u) * 0xFFu);
-}
-__device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, uint32_t bits) {
+__device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, uint2 keep) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   constexpr float kNear = 0.5f - 0x1p-15f;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   float x[8];
   uint32_t qb[8];
-  bool near_tie = false;
+  float dmax = 0.0f;
 #pragma unroll
   for (int e = 0; e < 8; e += 2) {
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e / 2]));
@@ -145,21 +98,19 @@ __device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, 
   for (int e = 0; e < 8; ++e) {
     const float tb = __fmaf_rn(x[e], rcp, kRound);
     qb[e] = __float_as_uint(tb);
-    const float d = __fmaf_rn(x[e], rcp, -(tb - kRound));
-    near_tie |= fabsf(d) > kNear && !((bits >> e) & 1u);
+    dmax = fmaxf(dmax, fabsf(__fmaf_rn(x[e], rcp, -(tb - kRound))));
   }
-  if (near_tie) {
+  if (dmax > kNear) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float tb = __fmaf_rn(x[e], rcp, kRound);
-      const float d = __fmaf_rn(x[e], rcp, -(tb - kRound));
-      if (fabsf(d) > kNear && !((bits >> e) & 1u))
+      if (fabsf(__fmaf_rn(x[e], rcp, -(tb - kRound))) > kNear)
         qb[e] = static_cast<uint32_t>(__float2int_rn(__fdiv_rn(x[e], sc)));
     }
   }
   const uint32_t lo = __byte_perm(__byte_perm(qb[0], qb[1], 0x0040), __byte_perm(qb[2], qb[3], 0x0040), 0x5410);
   const uint32_t hi = __byte_perm(__byte_perm(qb[4], qb[5], 0x0040), __byte_perm(qb[6], qb[7], 0x0040), 0x5410);
-  return make_uint2(lo & keep_mask(bits & 0xFu), hi & keep_mask(bits >> 4));
+  return make_uint2(lo & keep.x, hi & keep.y);
 }
 
 // D(16 x 8, int32) += A(16 x 32, int8, row-major) * B(32 x 8, int8, column-major)
@@ -183,12 +134,19 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// fp16(float(code) * scale) for bytes (2h, 2h+1) of an int8 word, packed as a half2 word
+// fp16(float(code) * scale) for bytes (2h, 2h+1) of an int8 word, packed as a half2 word.
+// float(code) is read off the bits 0x4B0000vv with vv = code + 128 (the float 2^23 + vv, exact)
+// less 2^23 + 128: a byte permute, a XOR and an add instead of integer-to-float conversions.
+__device__ __forceinline__ float code_to_float(uint32_t word, uint32_t byte_sel) {
+  uint32_t bits;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(bits) : "r"(word), "r"(0x4B000000u), "r"(byte_sel));
+  return __uint_as_float(bits ^ 0x80u) - 8388736.0f;  // 2^23 + 128
+}
 __device__ __forceinline__ uint32_t what2(uint32_t word, int h, float scale) {
-  const float lo = static_cast<float>(static_cast<int8_t>((word >> (16 * h)) & 0xFFu));
-  const float hi = static_cast<float>(static_cast<int8_t>((word >> (16 * h + 8)) & 0xFFu));
-  const __half2 v = __halves2half2(__float2half_rn(__fmul_rn(lo, scale)),
-                                   __float2half_rn(__fmul_rn(hi, scale)));
+  // selector: byte 2h (or 2h + 1) of word, then bytes 1..3 of 0x4B000000
+  const float lo = code_to_float(word, 0x7650u + 2u * h);
+  const float hi = code_to_float(word, 0x7651u + 2u * h);
+  const __half2 v = __floats2half2_rn(__fmul_rn(lo, scale), __fmul_rn(hi, scale));
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
@@ -200,354 +158,355 @@ __device__ __forceinline__ uint32_t mask2(uint32_t word, uint32_t bits, int h) {
 }
 
 struct DecodeShared {
-  uint64_t full[kDWarps];      // one weight box per 16-channel tile
-  float part[kDWarps][kDTok];   // row maxima of this CTA's slice, per warp
-  float all_max[kDSplit][kDTok];  // row maxima of every slice (written by the slice's CTA)
+  uint64_t full[kDMaxTiles];    // one weight box per 16-channel tile
+  uint4 part[kDWarps];          // per-warp row maxima: word e holds tokens 2e, 2e + 1 (fp16)
   float sx[kDTok];
-  float rcp[kDTok];
-  int zero_row[kDTok];
-  uint8_t flags[kDMaxKb / kDSplit * 16];  // outlier bits of the slice's 8-column chunks
+  uint8_t flags[kDMaxKb * 16];  // outlier bits of each 8-column chunk of X
+  uint8_t oslot[kDMaxKb * 16];  // chunk with an outlier -> its slot in xo (0xFF: not kept)
+  uint4 xo[kDOutChunks][kDTok];  // fp16 X of the chunks with an outlier, per token
+  int n_ochunks;
   int abort;
 };
 
-// [Wq tiles: tiles x 16 rows x nqmax k-blocks x 128 B | int8 codes: 8 rows x (nqmax x 128
-//  + 32) B]
-size_t decode_smem_bytes(int tiles, int nqmax) {
-  return 1024 + static_cast<size_t>(tiles) * 16 * 128 * nqmax +
-         static_cast<size_t>(kDTok) * (128 * nqmax + 32);
+// partial sums of the 16 warps, [warp][token][stage_ld] per kind (int32, then fp32); the
+// 4-word pad keeps the fragment stores free of bank conflicts
+__host__ __device__ constexpr int stage_ld(int T) { return 16 * T + 4; }
+__host__ __device__ constexpr int stage_bytes(int T) { return 2 * kDWarps * kDTok * stage_ld(T) * 4; }
+// bytes of one tile: 16 rows x K/128 k-blocks x 128 B
+__host__ __device__ inline int tile_bytes(int K) { return 16 * K; }
+__host__ __device__ inline int weight_area(int T, int K) {
+  return T * tile_bytes(K) > stage_bytes(T) ? T * tile_bytes(K) : stage_bytes(T);
 }
 
-// P = pairs of 16-channel tiles per CTA; the 8 warps are P pairs x (8 / P) parts of the
-// slice's k-blocks.
-template <int P>
-__global__ void __launch_bounds__(kDThreads, 3)
+// [Wq tiles: T x K/128 k-blocks x 16 rows x 128 B (or the staged sums) | codes: 8 x (K + 16) B]
+size_t decode_smem_bytes(int T, int K) {
+  return 1024 + static_cast<size_t>(weight_area(T, K)) + static_cast<size_t>(kDTok) * (K + 16);
+}
+
+// T 16-channel tiles per CTA; each thread holds up to kItems 8-column chunks of X
+template <int T, int kItems>
+__global__ void __launch_bounds__(kDThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap map_wq, const DecodeArgs a) {
-  constexpr int kParts = kDWarps / P;   // k-parts of the slice
-  constexpr int kTiles = 2 * P;         // 16-channel tiles per CTA (and per cluster)
-  constexpr int kG = 16 * kTiles;       // channels per cluster
-  constexpr int kRed = kG / kDSplit;    // channels each CTA finishes
+  constexpr int kC = 16 * T;  // channels per CTA
+  constexpr int kLd = stage_ld(T);
   extern __shared__ uint8_t decode_smem_raw[];
   __shared__ DecodeShared sh;
   uint8_t* wt = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(decode_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int nqmax = a.nqmax;
-  const int tile_bytes = 16 * 128 * nqmax;
-  uint8_t* xq_s = wt + kTiles * tile_bytes;  // [token][xq_ld] int8
-  const int xq_ld = nqmax * 128 + 32;        // +32: the 8 token rows start in different banks
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int r = static_cast<int>(cluster_rank());
-  const int n0 = (blockIdx.x / kDSplit) * kG;
   const int M = a.M, K = a.K, N = a.N;
   const int KB = K / 128;
-  const int lo = r * KB / kDSplit, nq = (r + 1) * KB / kDSplit - lo;  // this CTA's k-blocks
+  const int tb = tile_bytes(K);
+  uint8_t* xq_s = wt + weight_area(T, K);  // [token][xq_ld] int8
+  const int xq_ld = K + 16;                // +16: token rows g and g + 1 start 4 banks apart
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int g = lane >> 2, tig = lane & 3;
+  const int n0 = blockIdx.x * kC;
   volatile int* abort = &sh.abort;
 
+  if (tid < M) {  // CTA b asks L2 for the (b mod 8)-th eighth of each row of X, ahead of Wq
+    const int seg = K / 8;
+    prefetch_l2(a.X + static_cast<size_t>(tid) * K + (blockIdx.x % 8) * seg,
+                static_cast<uint32_t>(seg * 2));
+  }
   if (tid == 0) {
-    for (int t = 0; t < kTiles; ++t) mbar_init(&sh.full[t], 1);
+    for (int t = 0; t < T; ++t) mbar_init(&sh.full[t], 1);
     sh.abort = 0;
+    sh.n_ochunks = 0;
     fence_mbarrier_init();
     prefetch_tmap(&map_wq);
   }
   __syncthreads();
-  if (tid == 0 && nq > 0) {  // the weight stream starts before the previous launch ends
-    for (int t = 0; t < kTiles; ++t) {
-      mbar_arrive_expect_tx(&sh.full[t], static_cast<uint32_t>(tile_bytes));
-      tma_load_3d(&map_wq, wt + static_cast<size_t>(t) * tile_bytes, &sh.full[t], 0,
-                  n0 + 16 * t, lo);
+  if (tid == 0) {  // the weight stream starts before the previous launch ends
+    for (int t = 0; t < T; ++t) {
+      mbar_arrive_expect_tx(&sh.full[t], static_cast<uint32_t>(tb));
+      tma_load_3d(&map_wq, wt + static_cast<size_t>(t) * tb, &sh.full[t], 0, n0 + 16 * t, 0);
     }
   }
-  const int g = lane >> 2, tig = lane & 3;
-  const int pair = warp / kParts, part = warp % kParts;  // tiles 2 pair, 2 pair + 1
-  float swr[2][2];
+  float swr[T][2];  // scales of the fragment rows g, g + 8 of each tile
 #pragma unroll
-  for (int m = 0; m < 2; ++m)
+  for (int t = 0; t < T; ++t)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int n = n0 + 32 * pair + 16 * m + 8 * h + g;
-      swr[m][h] = n < N ? a.w_scale[n] : 0.0f;
+      const int n = n0 + 16 * t + 8 * h + g;
+      swr[t][h] = n < N ? a.w_scale[n] : 0.0f;
     }
-  if (tid < M && nq > 0) prefetch_l2(a.X + static_cast<size_t>(tid) * K + lo * 128, nq * 256);
+  // the epilogue's (token, channel): thread tid < 8 kC
+  const int ec = tid % kC, ei = tid / kC;
+  const bool e_live = tid < kDTok * kC && ei < M && n0 + ec < N;
+  const float e_sw = e_live ? a.w_scale[n0 + ec] : 0.0f;
+  const float e_bias = (e_live && a.bias) ? __half2float(a.bias[n0 + ec]) : 0.0f;
   grid_launch_dependents();
   grid_dependency_wait();  // X (the previous layer's output) is complete from here on
 
-  // ---- this CTA's slice of X.  Item (chunk c of 8 columns, token pair p): the 4 lanes of
-  // a chunk hold its 8 tokens.  The raw values stay in registers for the quantization.
-  const int p = lane & 3;
-  const int col0 = lo * 128;
-  float rm0 = 0.0f, rm1 = 0.0f;  // row maxima of tokens 2p, 2p+1 over regular columns
-  uint4 xv[kDMaxItems][2];
-  uint32_t xbits[kDMaxItems];
+  // ---- X: thread tid holds chunks c = tid + 512 u (8 columns x 8 tokens each) in registers
+  const int chunks = K / 8;
+  // fp16 x: |x| > t exactly when |x| > (t rounded down to fp16)
+  const __half2 th2 = __half2half2(__float2half_rd(a.threshold));
+  const __half2 zero2 = __float2half2_rn(0.0f);
+  uint4 xv[kItems][kDTok];
+  uint2 xkeep[kItems];
+  __half2 rm[kDTok / 2];  // row maxima over regular columns, tokens (2e, 2e + 1)
 #pragma unroll
-  for (int it = 0; it < kDMaxItems; ++it) {
-    const int item = tid + it * kDThreads;
-    xbits[it] = 0u;
-    xv[it][0] = xv[it][1] = make_uint4(0u, 0u, 0u, 0u);
-    if (item < nq * 64) {  // warp-uniform: nq * 64 is a multiple of 64
-      const int c = item >> 2;
-      const int col = col0 + c * 8;
-      if (2 * p < M)
-        xv[it][0] = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(2 * p) * K + col));
-      if (2 * p + 1 < M)
-        xv[it][1] = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(2 * p + 1) * K + col));
-      const uint32_t w0[4] = {xv[it][0].x, xv[it][0].y, xv[it][0].z, xv[it][0].w};
-      const uint32_t w1[4] = {xv[it][1].x, xv[it][1].y, xv[it][1].z, xv[it][1].w};
-      uint32_t bits = 0;
+  for (int e = 0; e < kDTok / 2; ++e) rm[e] = zero2;
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int c = tid + it * kDThreads;
+    xkeep[it] = make_uint2(0u, 0u);
+#pragma unroll
+    for (int i = 0; i < kDTok; ++i) xv[it][i] = make_uint4(0u, 0u, 0u, 0u);
+    if (c < chunks) {
+#pragma unroll
+      for (int i = 0; i < kDTok; ++i)
+        if (i < M)
+          xv[it][i] = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * K + 8 * c));
+      uint32_t keep[4];  // |x| of the regular columns: 0x7FFF per regular half, 0 per outlier
+      uint32_t bits = 0u;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        __half2 m = __hmax2(__habs2(*reinterpret_cast<const __half2*>(&w0[e])),
-                            __habs2(*reinterpret_cast<const __half2*>(&w1[e])));
+        uint32_t cm = (&xv[it][0].x)[e] & 0x7FFF7FFFu;
 #pragma unroll
-        for (int o = 1; o <= 2; o <<= 1) {
-          const uint32_t other = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t*>(&m), o);
-          m = __hmax2(m, *reinterpret_cast<const __half2*>(&other));
+        for (int i = 1; i < kDTok; ++i) {
+          const uint32_t v = (&xv[it][i].x)[e] & 0x7FFF7FFFu;
+          const __half2 m = __hmax2(*reinterpret_cast<const __half2*>(&cm),
+                                    *reinterpret_cast<const __half2*>(&v));
+          cm = *reinterpret_cast<const uint32_t*>(&m);
         }
-        if (__low2float(m) > a.threshold) bits |= 1u << (2 * e);
-        if (__high2float(m) > a.threshold) bits |= 1u << (2 * e + 1);
+        const uint32_t gt = __hgt2_mask(*reinterpret_cast<const __half2*>(&cm), th2);
+        keep[e] = ~gt & 0x7FFF7FFFu;
+        bits |= ((gt & 1u) | ((gt >> 15) & 2u)) << (2 * e);
+      }
+      xkeep[it] = keep_masks(bits);
+      sh.flags[c] = static_cast<uint8_t>(bits);
+      if (bits != 0u) {  // keep the chunk's fp16 values for the outlier term
+        const int slot = atomicAdd(&sh.n_ochunks, 1);
+        sh.oslot[c] = static_cast<uint8_t>(slot < kDOutChunks ? slot : 0xFF);
+        if (slot < kDOutChunks)
+#pragma unroll
+          for (int i = 0; i < kDTok; ++i) sh.xo[slot][i] = xv[it][i];
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if ((bits >> e) & 1u) continue;
-        rm0 = fmaxf(rm0, fabsf(h2f(w0[e / 2], e & 1)));
-        rm1 = fmaxf(rm1, fabsf(h2f(w1[e / 2], e & 1)));
+      for (int i = 0; i < kDTok; i += 2) {
+        uint32_t m0 = (&xv[it][i].x)[0] & keep[0], m1 = (&xv[it][i + 1].x)[0] & keep[0];
+#pragma unroll
+        for (int e = 1; e < 4; ++e) {
+          const uint32_t v0 = (&xv[it][i].x)[e] & keep[e], v1 = (&xv[it][i + 1].x)[e] & keep[e];
+          const __half2 h0 = __hmax2(*reinterpret_cast<const __half2*>(&m0),
+                                     *reinterpret_cast<const __half2*>(&v0));
+          const __half2 h1 = __hmax2(*reinterpret_cast<const __half2*>(&m1),
+                                     *reinterpret_cast<const __half2*>(&v1));
+          m0 = *reinterpret_cast<const uint32_t*>(&h0);
+          m1 = *reinterpret_cast<const uint32_t*>(&h1);
+        }
+        const __half2 h0 = *reinterpret_cast<const __half2*>(&m0);
+        const __half2 h1 = *reinterpret_cast<const __half2*>(&m1);
+        rm[i / 2] = __hmax2(rm[i / 2], __halves2half2(__hmax(__low2half(h0), __high2half(h0)),
+                                                      __hmax(__low2half(h1), __high2half(h1))));
       }
-      xbits[it] = bits;
-      if (p == 0) sh.flags[c] = static_cast<uint8_t>(bits);
     }
   }
+  {  // the block's row maxima
+    uint32_t r4[4];
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    rm0 = fmaxf(rm0, __shfl_xor_sync(0xffffffffu, rm0, o));
-    rm1 = fmaxf(rm1, __shfl_xor_sync(0xffffffffu, rm1, o));
-  }
-  if (lane < 4) {
-    sh.part[warp][2 * p] = rm0;
-    sh.part[warp][2 * p + 1] = rm1;
+    for (int e = 0; e < 4; ++e) r4[e] = *reinterpret_cast<const uint32_t*>(&rm[e]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, r4[e], o);
+        const __half2 m = __hmax2(*reinterpret_cast<const __half2*>(&r4[e]),
+                                  *reinterpret_cast<const __half2*>(&other));
+        r4[e] = *reinterpret_cast<const uint32_t*>(&m);
+      }
+    if (lane == 0) sh.part[warp] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
   }
   __syncthreads();
-  if (warp == 0) {
-    // this slice's row maxima into every CTA of the cluster (lane: token lane % 8, CTAs
-    // lane / 8 and lane / 8 + 4); warp 0's release below covers its own remote stores
-    const int i = lane % kDTok;
-    float m = 0.0f;
+  // lane i < 8 of every warp: sx and 1/sx of token i, then shared across the warp
+  float sx_l = 0.0f, rcp_l = 0.0f;
+  if (lane < kDTok) {
+    __half m = __float2half_rn(0.0f);
 #pragma unroll
-    for (int w = 0; w < kDWarps; ++w) m = fmaxf(m, sh.part[w][i]);
-    const uint32_t local = smem_addr(&sh.all_max[r][i]);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) st_cluster_f32(map_rank(local, lane / kDTok + 4 * h), m);
+    for (int w = 0; w < kDWarps; ++w) {
+      const uint32_t word = (&sh.part[w].x)[lane >> 1];
+      const __half2 h2 = *reinterpret_cast<const __half2*>(&word);
+      m = __hmax(m, (lane & 1) ? __high2half(h2) : __low2half(h2));
+    }
+    const float mf = __half2float(m);
+    sx_l = __fdiv_rn(mf, 127.0f);
+    rcp_l = mf > 0.0f ? __frcp_rn(sx_l) : 0.0f;
+    if (warp == 0) sh.sx[lane] = sx_l;
   }
-  cluster_arrive_cta();
 
   // this warp's k-blocks and the k-steps among them holding an outlier column (bit
-  // 4 (kb - kb_begin) + j); the fp16 activations of the first two such steps are fetched now,
-  // while the cluster exchanges its row maxima
-  const int kb_begin = part * nq / kParts, kb_end = (part + 1) * nq / kParts;
+  // 4 (kb - kb_begin) + j).  Lane (g, tig) of k-step j of a k-block covers its 8 columns
+  // 16 (4 (tig / 2) + j) + 8 (tig % 2) .. + 7 (the chunk 8 (tig / 2) + 2 j + tig % 2), a
+  // permutation of the block's 128 columns that both MMA operands follow; with it the 16 lanes
+  // of a half-warp read 16 different bank pairs of the swizzled weight rows and of the codes.
+  const int kb_begin = warp * KB / kDWarps, kb_end = (warp + 1) * KB / kDWarps;
   const int nsteps = 4 * (kb_end - kb_begin);
-  const uint32_t ow = lane < nsteps
-      ? *reinterpret_cast<const uint32_t*>(&sh.flags[(4 * kb_begin + lane) * 4]) : 0u;
+  uint32_t ow = 0u;
+  if (lane < nsteps) {
+    const int kb = kb_begin + lane / 4, j = lane % 4;
+    const uint16_t* f2 = reinterpret_cast<const uint16_t*>(sh.flags);
+    ow = f2[(kb * 16 + 2 * j) / 2] | f2[(kb * 16 + 8 + 2 * j) / 2];
+  }
   const uint32_t outlier_steps = __ballot_sync(0xffffffffu, ow != 0u);
-  const __half* xg = a.X + static_cast<size_t>(g) * K + col0 + 8 * tig;
-  uint4 xo_pre[2];
+  const int lane_col = 64 * (tig >> 1) + 8 * (tig & 1);  // + 16 j within a k-block
+
+  // ---- int8 codes: xq_s[token][column].  A row with no regular value has 1/sx = 0 and
+  // codes 0.
   {
-    uint32_t rest = outlier_steps;
+    float sxv[kDTok], rcpv[kDTok];
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      xo_pre[n] = make_uint4(0u, 0u, 0u, 0u);
-      if (rest != 0u) {
-        const int st = __ffs(rest) - 1;
-        rest &= rest - 1u;
-        if (g < M)
-          xo_pre[n] = __ldg(reinterpret_cast<const uint4*>(xg + (kb_begin + st / 4) * 128 + 32 * (st % 4)));
-      }
+    for (int i = 0; i < kDTok; ++i) {
+      sxv[i] = __shfl_sync(0xffffffffu, sx_l, i);
+      rcpv[i] = __shfl_sync(0xffffffffu, rcp_l, i);
     }
-  }
-  cluster_wait();  // every slice's row maxima are in its shared memory
-
-  if (tid < kDTok) {
-    float m = 0.0f;
 #pragma unroll
-    for (int s = 0; s < kDSplit; ++s) m = fmaxf(m, sh.all_max[s][tid]);
-    const float sc = __fdiv_rn(m, 127.0f);
-    sh.sx[tid] = tid < M ? sc : 0.0f;
-    sh.rcp[tid] = (tid < M && m > 0.0f) ? __frcp_rn(sc) : 0.0f;
-    sh.zero_row[tid] = (tid >= M) || m == 0.0f;
-  }
-  __syncthreads();
-  // ---- int8 codes of the slice: xq_s[token][column of the slice]
+    for (int it = 0; it < kItems; ++it) {
+      const int c = tid + it * kDThreads;
+      if (c < chunks) {
 #pragma unroll
-  for (int it = 0; it < kDMaxItems; ++it) {
-    const int item = tid + it * kDThreads;
-    if (item < nq * 64) {
-      const int c = item >> 2;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int i = 2 * p + h;
-        const uint2 code = sh.zero_row[i] ? make_uint2(0u, 0u)
-                                          : quantize8(xv[it][h], sh.sx[i], sh.rcp[i], xbits[it]);
-        *reinterpret_cast<uint2*>(xq_s + i * xq_ld + c * 8) = code;
+        for (int i = 0; i < kDTok; ++i)
+          *reinterpret_cast<uint2*>(xq_s + i * xq_ld + c * 8) =
+              quantize8(xv[it][i], sxv[i], rcpv[i], xkeep[it]);
       }
     }
   }
   __syncthreads();
 
-  // ---- this warp: tiles 2 pair + m (m = 0, 1) over k-blocks [kb_begin, kb_end)
-  int d[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-  float pf[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+  // ---- this warp: every tile over k-blocks [kb_begin, kb_end)
+  int d[T][2][4];  // two accumulator chains per tile (even and odd k-steps) halve the MMA
+                   // dependency chain
+  float pf[T][4];
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      d[t][0][e] = d[t][1][e] = 0;
+      pf[t][e] = 0.0f;
+    }
   bool ok = true;
   if (kb_begin < kb_end) {
     bool landed = true;
     if (lane == 0)
-      landed = mbar_wait_bounded(&sh.full[2 * pair], 0, abort) &&
-               mbar_wait_bounded(&sh.full[2 * pair + 1], 0, abort);
+      for (int t = 0; t < T; ++t) landed = landed && mbar_wait_bounded(&sh.full[t], 0, abort);
     ok = __shfl_sync(0xffffffffu, landed ? 1 : 0, 0) != 0;
-    mbar_try_wait(&sh.full[2 * pair], 0);  // each lane observes the completed phases
-    mbar_try_wait(&sh.full[2 * pair + 1], 0);
+    for (int t = 0; t < T; ++t) mbar_try_wait(&sh.full[t], 0);  // each lane observes the phase
   }
   if (ok && kb_begin < kb_end) {
     // rows g and g + 8 of the swizzled 16 x 128 tiles: one address per k-step of a k-block
-    const uint8_t* wrow[2][4];
+    const uint8_t* wrow[T][4];
 #pragma unroll
-    for (int m = 0; m < 2; ++m)
+    for (int t = 0; t < T; ++t)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        wrow[m][j] = wt + (2 * pair + m) * tile_bytes + g * 128 +
-                     (((2 * j + (tig >> 1)) ^ g) << 4) + (tig & 1) * 8 + kb_begin * (16 * 128);
-    const uint8_t* xrow = xq_s + g * xq_ld + 8 * tig + kb_begin * 128;
-    int n_out = 0;
+        wrow[t][j] = wt + t * tb + g * 128 + (((4 * (tig >> 1) + j) ^ g) << 4) +
+                     (tig & 1) * 8 + kb_begin * (16 * 128);
+    const uint8_t* xrow = xq_s + g * xq_ld + lane_col + kb_begin * 128;
     for (int kb = kb_begin; kb < kb_end; ++kb) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint2 xb = *reinterpret_cast<const uint2*>(xrow + 32 * j);
-        uint2 w[2][2];
+        const uint2 xb = *reinterpret_cast<const uint2*>(xrow + 16 * j);
+        uint2 w[T][2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          w[m][0] = *reinterpret_cast<const uint2*>(wrow[m][j]);
-          w[m][1] = *reinterpret_cast<const uint2*>(wrow[m][j] + 1024);
-          mma_s8_16832(d[m], w[m][0].x, w[m][1].x, w[m][0].y, w[m][1].y, xb.x, xb.y);
-        }
-        if ((outlier_steps >> ((kb - kb_begin) * 4 + j)) & 1u) {
-          // fp16 term: this k-step's outlier columns only (the other activations are zero)
-          const uint32_t fb = sh.flags[kb * 16 + 4 * j + tig];
-          uint4 xr = n_out == 0 ? xo_pre[0] : xo_pre[1];
-          if (n_out >= 2 && g < M) xr = __ldg(reinterpret_cast<const uint4*>(xg + kb * 128 + 32 * j));
-          ++n_out;
-          const uint32_t b0 = mask2(xr.x, fb, 0), b1 = mask2(xr.y, fb, 1);
-          const uint32_t b2 = mask2(xr.z, fb, 2), b3 = mask2(xr.w, fb, 3);
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            uint32_t ha[2][4];  // rows g, g + 8: fp16 weights of this step's 8 columns
-            if (a.W16) {        // the layer's kept fp16 weights
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int n = n0 + 32 * pair + 16 * m + 8 * h + g;
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (n < N)
-                  v = __ldg(reinterpret_cast<const uint4*>(
-                      a.W16 + static_cast<size_t>(n) * K + col0 + kb * 128 + 32 * j + 8 * tig));
-                ha[h][0] = v.x; ha[h][1] = v.y; ha[h][2] = v.z; ha[h][3] = v.w;
-              }
-            } else {            // fp16(Wq * w_scale) from the resident int8 tile
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                ha[h][0] = what2(w[m][h].x, 0, swr[m][h]);
-                ha[h][1] = what2(w[m][h].x, 1, swr[m][h]);
-                ha[h][2] = what2(w[m][h].y, 0, swr[m][h]);
-                ha[h][3] = what2(w[m][h].y, 1, swr[m][h]);
-              }
-            }
-            mma_f16_16816(pf[m], ha[0][0], ha[1][0], ha[0][1], ha[1][1], b0, b1);
-            mma_f16_16816(pf[m], ha[0][2], ha[1][2], ha[0][3], ha[1][3], b2, b3);
-          }
+        for (int t = 0; t < T; ++t) {
+          w[t][0] = *reinterpret_cast<const uint2*>(wrow[t][j]);
+          w[t][1] = *reinterpret_cast<const uint2*>(wrow[t][j] + 1024);
+          mma_s8_16832(d[t][j & 1], w[t][0].x, w[t][1].x, w[t][0].y, w[t][1].y, xb.x, xb.y);
         }
       }
 #pragma unroll
-      for (int m = 0; m < 2; ++m)
+      for (int t = 0; t < T; ++t)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) wrow[m][j] += 16 * 128;
+        for (int j = 0; j < 4; ++j) wrow[t][j] += 16 * 128;
       xrow += 128;
+    }
+    // fp16 term: the warp's k-steps holding an outlier column, one at a time (the code exists
+    // once, so the rare steps cost no instruction fetches per unrolled copy); only the
+    // outlier columns' activations are nonzero
+    uint32_t rest = outlier_steps;
+#pragma unroll 1
+    while (rest != 0u) {
+      const int st = __ffs(rest) - 1;
+      rest &= rest - 1u;
+      const int kb = kb_begin + st / 4, j = st % 4;
+      const int ch = kb * 16 + 8 * (tig >> 1) + 2 * j + (tig & 1);  // this lane's chunk
+      const uint32_t fb = sh.flags[ch];
+      uint4 xr = make_uint4(0u, 0u, 0u, 0u);
+      if (fb != 0u) {
+        const int slot = sh.oslot[ch];
+        if (slot < kDOutChunks) xr = sh.xo[slot][g];
+        else if (g < M)
+          xr = __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(g) * K + 8 * ch));
+      }
+      const uint32_t b0 = mask2(xr.x, fb, 0), b1 = mask2(xr.y, fb, 1);
+      const uint32_t b2 = mask2(xr.z, fb, 2), b3 = mask2(xr.w, fb, 3);
+      const uint8_t* wb = wt + g * 128 + (((4 * (tig >> 1) + j) ^ g) << 4) + (tig & 1) * 8 +
+                          kb * (16 * 128);
+#pragma unroll
+      for (int t = 0; t < T; ++t) {
+        uint32_t ha[2][4];  // rows g, g + 8: fp16 weights of this step's 8 columns
+        if (a.W16) {        // the layer's kept fp16 weights
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int n = n0 + 16 * t + 8 * h + g;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (n < N)
+              v = __ldg(reinterpret_cast<const uint4*>(
+                  a.W16 + static_cast<size_t>(n) * K + kb * 128 + lane_col + 16 * j));
+            ha[h][0] = v.x; ha[h][1] = v.y; ha[h][2] = v.z; ha[h][3] = v.w;
+          }
+        } else {            // fp16(Wq * w_scale) from the resident int8 tile
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint2 w = *reinterpret_cast<const uint2*>(wb + t * tb + 1024 * h);
+            ha[h][0] = what2(w.x, 0, swr[t][h]);
+            ha[h][1] = what2(w.x, 1, swr[t][h]);
+            ha[h][2] = what2(w.y, 0, swr[t][h]);
+            ha[h][3] = what2(w.y, 1, swr[t][h]);
+          }
+        }
+        mma_f16_16816(pf[t], ha[0][0], ha[1][0], ha[0][1], ha[1][1], b0, b1);
+        mma_f16_16816(pf[t], ha[0][2], ha[1][2], ha[0][3], ha[1][3], b2, b3);
+      }
     }
   }
   if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);
-  // partial sums of this part of the slice into the weight area (every warp is done reading
-  // it): stage_i / stage_p [warp][32 channels][8 tokens]
+  // partial sums into the weight area (every warp is done reading it)
   __syncthreads();
   int32_t* stage_i = reinterpret_cast<int32_t*>(wt);
-  float* stage_p = reinterpret_cast<float*>(wt + kDWarps * 32 * kDTok * sizeof(int32_t));
+  float* stage_p = reinterpret_cast<float*>(wt + kDWarps * kDTok * kLd * 4);
 #pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    const int c0 = (warp * 32 + 16 * m + g) * kDTok + 2 * tig, c1 = c0 + 8 * kDTok;
-    stage_i[c0] = d[m][0];
-    stage_i[c0 + 1] = d[m][1];
-    stage_i[c1] = d[m][2];
-    stage_i[c1 + 1] = d[m][3];
-    stage_p[c0] = pf[m][0];
-    stage_p[c0 + 1] = pf[m][1];
-    stage_p[c1] = pf[m][2];
-    stage_p[c1 + 1] = pf[m][3];
+  for (int t = 0; t < T; ++t) {
+    const int o = (warp * kDTok + 2 * tig) * kLd + 16 * t + g;
+    stage_i[o] = d[t][0][0] + d[t][1][0];
+    stage_i[o + kLd] = d[t][0][1] + d[t][1][1];
+    stage_i[o + 8] = d[t][0][2] + d[t][1][2];
+    stage_i[o + kLd + 8] = d[t][0][3] + d[t][1][3];
+    stage_p[o] = pf[t][0];
+    stage_p[o + kLd] = pf[t][1];
+    stage_p[o + 8] = pf[t][2];
+    stage_p[o + kLd + 8] = pf[t][3];
   }
   __syncthreads();
-  // sum over the k-parts of each tile pair, in place into the part-0 slots: stage[pair * kParts]
-  for (int e = tid; e < P * 32 * kDTok; e += kDThreads) {
-    const int pr = e / (32 * kDTok), off = e % (32 * kDTok);
-    int32_t si = stage_i[(pr * kParts) * 32 * kDTok + off];
-    float sp = stage_p[(pr * kParts) * 32 * kDTok + off];
+  if (e_live) {  // token ei, channel n0 + ec: the 16 warps in a fixed order
+    int32_t acc = 0;
+    float P = 0.0f;
 #pragma unroll
-    for (int h = 1; h < kParts; ++h) {
-      si += stage_i[(pr * kParts + h) * 32 * kDTok + off];
-      sp += stage_p[(pr * kParts + h) * 32 * kDTok + off];
+    for (int w = 0; w < kDWarps; ++w) {
+      acc += stage_i[(w * kDTok + ei) * kLd + ec];
+      P += stage_p[(w * kDTok + ei) * kLd + ec];
     }
-    stage_i[(pr * kParts) * 32 * kDTok + off] = si;
-    stage_p[(pr * kParts) * 32 * kDTok + off] = sp;
+    const int n = n0 + ec;
+    const float y = static_cast<float>(acc) * sh.sx[ei] * e_sw + P + e_bias;
+    a.Y[static_cast<size_t>(ei) * N + n] = __float2half_rn(y);
+    if (a.acc) a.acc[static_cast<size_t>(ei) * N + n] = sh.abort ? 0 : acc;
   }
-  __syncthreads();
-  cluster_arrive_cta();
-  cluster_wait();  // every slice's partial sums are in its shared memory
-
-  // ---- CTA r finishes channels [r * kRed, (r + 1) * kRed) of the group.  Thread (channel,
-  // token quad, kind) sums the int32 (kind 0) or fp32 (kind 1) partials of the 8 slices in a
-  // fixed order; the two kinds meet through a shuffle.
-  if (tid < 4 * kRed) {  // whole warps: 4 * kRed is 64 or 32
-    const int kind = tid & 1, quad = (tid >> 1) & 1, cl = r * kRed + (tid >> 2);
-    const int pr = cl / 32, cr = cl % 32;
-    const uint8_t* stage = kind ? reinterpret_cast<const uint8_t*>(stage_p)
-                                : reinterpret_cast<const uint8_t*>(stage_i);
-    uint4 v[kDSplit];
-    const uint32_t local = smem_addr(stage + ((((pr * kParts) * 32 + cr) * kDTok + 4 * quad) * 4));
-#pragma unroll
-    for (int q = 0; q < kDSplit; ++q) v[q] = ld_cluster_v4(map_rank(local, q));
-    uint32_t sum[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int q = 0; q < kDSplit; ++q) {
-      const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        sum[e] = kind ? __float_as_uint(__uint_as_float(sum[e]) + __uint_as_float(w[e]))
-                      : sum[e] + w[e];
-    }
-    uint32_t other[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) other[e] = __shfl_xor_sync(0xffffffffu, sum[e], 1);
-    const int n = n0 + cl;
-    if (kind == 0 && n < N) {
-      const float swn = a.w_scale[n];
-      const float bb = a.bias ? __half2float(a.bias[n]) : 0.0f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * quad + e;
-        if (i >= M) continue;
-        const int acc = static_cast<int>(sum[e]);
-        const float y = static_cast<float>(acc) * sh.sx[i] * swn + __uint_as_float(other[e]) + bb;
-        a.Y[static_cast<size_t>(i) * N + n] = __float2half_rn(y);
-        if (a.acc) a.acc[static_cast<size_t>(i) * N + n] = sh.abort ? 0 : acc;
-      }
-    }
-  }
-  cluster_arrive_relaxed();  // this CTA is done reading its peers' shared memory
-  if (tid == 0 && nq > 0) {
+  if (tid == 0) {
     // every copy this CTA started has landed before it exits (normally long ago)
     int dummy = 0;
-    for (int t = 0; t < kTiles; ++t) mbar_wait_bounded(&sh.full[t], 0, &dummy);
+    for (int t = 0; t < T; ++t) mbar_wait_bounded(&sh.full[t], 0, &dummy);
   }
-  cluster_wait();  // no CTA leaves while a peer may still read its shared memory
 }
 
 }  // namespace
@@ -555,17 +514,11 @@ __global__ void __launch_bounds__(kDThreads, 3)
 DecodePlan plan_decode(int M, int N, int K) {
   DecodePlan p = {};
   p.fits = false;
-  if (M > kDTok || K % 128 != 0 || K / 128 > kDMaxKb || N <= 0) return p;
-  const int KB = K / 128;
-  p.cluster = kDSplit;
-  p.nqmax = (KB + kDSplit - 1) / kDSplit;
-  p.wpm = K <= 4096 ? 4 : 2;  // pairs of 16-channel tiles per CTA
-  const int tiles = 2 * p.wpm;
-  p.tile_rows = 16;
-  p.smem = decode_smem_bytes(tiles, p.nqmax);
-  const int groups = (N + 16 * tiles - 1) / (16 * tiles);
-  p.ctas = groups * kDSplit;
-  p.fits = p.smem + sizeof(DecodeShared) <= kDSmemBudget;
+  if (M > kDTok || K % 128 != 0 || K / 128 > kDMaxKb || N <= 0 || M <= 0) return p;
+  p.tiles = K <= 4096 ? 2 : 1;
+  p.smem = decode_smem_bytes(p.tiles, K);
+  p.ctas = (N + 16 * p.tiles - 1) / (16 * p.tiles);
+  p.fits = p.smem + sizeof(DecodeShared) <= kDSmemMax;
   return p;
 }
 
@@ -575,13 +528,16 @@ cudaError_t launch_decode(const CUtensorMap& map_wq, const DecodeArgs& a, const 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev != configured_device) {
-    e = cudaFuncSetAttribute(decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kDSmemBudget));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kDSmemBudget));
-    if (e != cudaSuccess) return e;
+  if (dev != configured_device) {  // all the shared memory a CTA may have beside the static
+    for (const void* k : {reinterpret_cast<const void*>(decode_kernel<2, 1>),
+                          reinterpret_cast<const void*>(decode_kernel<1, 2>)}) {
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, k);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kDSmemMax - fa.sharedSizeBytes));
+      if (e != cudaSuccess) return e;
+    }
     configured_device = dev;
   }
   cudaLaunchConfig_t cfg = {};
@@ -589,17 +545,14 @@ cudaError_t launch_decode(const CUtensorMap& map_wq, const DecodeArgs& a, const 
   cfg.blockDim = dim3(kDThreads);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 2 : 1;
-  return p.wpm == 4 ? cudaLaunchKernelEx(&cfg, decode_kernel<4>, map_wq, a)
-                     : cudaLaunchKernelEx(&cfg, decode_kernel<2>, map_wq, a);
+  cfg.numAttrs = pdl ? 1 : 0;
+  // K <= 4096: two tiles, one chunk of X per thread; up to 8192: one tile, two chunks
+  return p.tiles == 2 ? cudaLaunchKernelEx(&cfg, decode_kernel<2, 1>, map_wq, a)
+                      : cudaLaunchKernelEx(&cfg, decode_kernel<1, 2>, map_wq, a);
 }
 
 }  // namespace i8mm

@@ -159,14 +159,11 @@ struct DecodeArgs {
   const __half* bias;
   __half* Y;
   int32_t* acc;          // nullable: also write the int32 accumulators
-  int nqmax;             // k-blocks of the largest slice of K (one slice per CTA of a cluster)
   int32_t* status;
 };
 struct DecodePlan {
-  int cluster;           // CTAs per cluster = slices of K
-  int wpm;               // pairs of 16-channel tiles per CTA (the kernel's P)
-  int tile_rows;         // rows of Wq per TMA box
-  int ctas, nqmax;
+  int tiles;             // 16-channel tiles per CTA (the kernel's T)
+  int ctas;
   size_t smem;
   bool fits;
 };
