@@ -403,27 +403,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
         wrow[t][j] = wt + t * tb + g * 128 + (((4 * (tig >> 1) + j) ^ g) << 4) +
                      (tig & 1) * 8 + kb_begin * (16 * 128);
     const uint8_t* xrow = xq_s + g * xq_ld + lane_col + kb_begin * 128;
-    for (int kb = kb_begin; kb < kb_end; ++kb) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint2 xb = *reinterpret_cast<const uint2*>(xrow + 16 * j);
-        uint2 w[T][2];
-#pragma unroll
-        for (int t = 0; t < T; ++t) {
-          w[t][0] = *reinterpret_cast<const uint2*>(wrow[t][j]);
-          w[t][1] = *reinterpret_cast<const uint2*>(wrow[t][j] + 1024);
-          mma_s8_16832(d[t][j & 1], w[t][0].x, w[t][1].x, w[t][0].y, w[t][1].y, xb.x, xb.y);
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < T; ++t)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) wrow[t][j] += 16 * 128;
-      xrow += 128;
-    }
-    // fp16 term: the warp's k-steps holding an outlier column, one at a time (the code exists
-    // once, so the rare steps cost no instruction fetches per unrolled copy); only the
-    // outlier columns' activations are nonzero
+    // fp16 term first: the warp's k-steps holding an outlier column, one at a time in a rolled
+    // loop (its code exists once); only the outlier columns' activations are nonzero.  Then
+    // the int8 k-steps.
     uint32_t rest = outlier_steps;
 #pragma unroll 1
     while (rest != 0u) {
@@ -469,6 +451,24 @@ __global__ void __launch_bounds__(kDThreads, 1)
         mma_f16_16816(pf[t], ha[0][0], ha[1][0], ha[0][1], ha[1][1], b0, b1);
         mma_f16_16816(pf[t], ha[0][2], ha[1][2], ha[0][3], ha[1][3], b2, b3);
       }
+    }
+    for (int kb = kb_begin; kb < kb_end; ++kb) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint2 xb = *reinterpret_cast<const uint2*>(xrow + 16 * j);
+        uint2 w[T][2];
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+          w[t][0] = *reinterpret_cast<const uint2*>(wrow[t][j]);
+          w[t][1] = *reinterpret_cast<const uint2*>(wrow[t][j] + 1024);
+          mma_s8_16832(d[t][j & 1], w[t][0].x, w[t][1].x, w[t][0].y, w[t][1].y, xb.x, xb.y);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < T; ++t)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) wrow[t][j] += 16 * 128;
+      xrow += 128;
     }
   }
   if (!ok) report(a.status, INT8MM_ERR_TIMEOUT);

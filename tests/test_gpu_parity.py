@@ -254,6 +254,27 @@ def test_forward_accumulators_and_y(M, K, N, n_out, t):
         assert not acc.any()
 
 
+@pytest.mark.parametrize("M,K,N,cols,t", [
+    (8, 2048, 512, list(range(640, 704)), 6.0),       # 64 outlier columns in 8 chunks
+    (8, 2048, 512, list(range(640, 705)), 6.0),       # 65 columns: fp16 MMAs instead
+    (6, 4096, 384, list(range(3, 4096, 57)), 6.0),    # 72 chunks with an outlier
+    (7, 1024, 200, [0, 1, 2, 1023], 6.0),             # first and last columns
+])
+def test_decode_outlier_term_routes(M, K, N, cols, t):
+    """The one-launch decode kernel computes the fp16 term on CUDA cores for up to 64 outlier
+    columns (all within 64 chunks of 8) and with fp16 MMAs beyond; both against the oracle."""
+    rng = np.random.default_rng(M * K + N + len(cols))
+    X = rng.standard_normal((M, K))
+    X[:, cols] *= rng.uniform(10, 40, size=len(cols))
+    X[0, cols] = rng.uniform(20, 40, size=len(cols)) * rng.choice([-1, 1], size=len(cols))
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+    b = (rng.standard_normal(N) * 0.01).astype(np.float16)
+    X = X.astype(np.float16)
+    _, found = oracle.outlier_columns(X, t)
+    np.testing.assert_array_equal(found, np.array(sorted(cols)))
+    check_forward_acc(X, W, b, t)
+
+
 def test_decode_workload_full_forward():
     w, X, W, b, _ = workload_inputs("decode_q_proj")
     Y, acc = check_forward_acc(X, W, b, w.threshold)
