@@ -56,9 +56,15 @@ def _load():
             lib.oracle_linear_forward_rows.argtypes = [p, i64, i64, p, p, p, i64, f32, p, i64, p, p]
             lib.oracle_linear_forward_rows_w16.argtypes = [p, i64, i64, p, p, p, p, i64, f32, p,
                                                            i64, p, p]
+            lib.oracle_quantize_tensor.argtypes = [p, i64, i64, p, p, p]
+            lib.oracle_linear_forward_rows_ex.argtypes = [p, i64, i64, p, p, p, p, i64, f32,
+                                                          ctypes.c_int, p, i64, p, p]
+            lib.oracle_activation_stats.argtypes = [p, i64, i64, p, p]
             for name in ("oracle_quant_weight", "oracle_outlier_columns", "oracle_quantize_rows",
                          "oracle_gemm_i32", "oracle_outlier_weights", "oracle_linear_forward",
-                         "oracle_linear_forward_rows", "oracle_linear_forward_rows_w16"):
+                         "oracle_linear_forward_rows", "oracle_linear_forward_rows_w16",
+                         "oracle_quantize_tensor", "oracle_linear_forward_rows_ex",
+                         "oracle_activation_stats"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -193,3 +199,57 @@ def linear_forward_rows(X, Wq, sw, bias, threshold: float, rows):
                                               float(threshold), _ptr(rows), len(rows), _ptr(Y),
                                               _ptr(A)), "oracle_linear_forward_rows")
     return Y, A
+
+
+def quantize_tensor(X, mask):
+    """One activation scale for the whole of X ([P5] item 2 as its snippet is written): absmax
+    over every row and the regular columns, / 127.  Returns Xq and the scale of every row (all
+    equal)."""
+    X = _c(X, np.float16)
+    mask = _c(mask, np.uint32)
+    M, K = X.shape
+    Xq = np.empty((M, K), np.int8)
+    sx = np.empty(M, np.float32)
+    _check(_load().oracle_quantize_tensor(_ptr(X), M, K, _ptr(mask), _ptr(Xq), _ptr(sx)),
+           "oracle_quantize_tensor")
+    return Xq, sx
+
+
+def linear_forward_rows_ex(X, Wq, sw, bias, threshold: float, rows, W16=None,
+                           per_tensor: bool = False):
+    """linear_forward_rows with the kept fp16 weights (W16, nullable) and the per-tensor
+    activation scale as options."""
+    X = _c(X, np.float16)
+    Wq = _c(Wq, np.int8)
+    sw = _c(sw, np.float32)
+    W16 = None if W16 is None else _c(W16, np.float16)
+    b = None if bias is None else _c(bias, np.float16)
+    rows = _c(rows, np.int64)
+    M, K = X.shape
+    N = Wq.shape[0]
+    Y = np.empty((len(rows), N), np.float16)
+    A = np.empty((len(rows), N), np.int32)
+    _check(_load().oracle_linear_forward_rows_ex(_ptr(X), M, K, _ptr(Wq), _ptr(sw), _ptr(W16),
+                                                 _ptr(b), N, float(threshold), int(per_tensor),
+                                                 _ptr(rows), len(rows), _ptr(Y), _ptr(A)),
+           "oracle_linear_forward_rows_ex")
+    return Y, A
+
+
+def linear_forward_tensor(X, Wq, sw, bias, threshold: float, W16=None):
+    """The layer with one activation scale for the whole of X."""
+    return linear_forward_rows_ex(X, Wq, sw, bias, threshold, np.arange(X.shape[0]), W16=W16,
+                                  per_tensor=True)[0]
+
+
+def activation_stats(X):
+    """[P2] section 5.1: (max |X|, the 0.99 quantile of |X|, max / (q99 + 1e-6), column
+    absmax [K])."""
+    X = _c(X, np.float16)
+    M, K = X.shape
+    col = np.empty(K, np.float32)
+    out = np.empty(3, np.float64)
+    _check(_load().oracle_activation_stats(_ptr(X), M, K, _ptr(col), _ptr(out)),
+           "oracle_activation_stats")
+    return float(out[0]), float(out[1]), float(out[2]), col
+

@@ -136,9 +136,8 @@ int oracle_outlier_columns(const uint16_t *X, int64_t M, int64_t K, float thresh
 
 static int is_outlier(const uint32_t *mask, int64_t j) { return (mask[j / 32] >> (j % 32)) & 1; }
 
-/* one row: absmax over the regular columns, scale, quantize */
-static void quantize_one_row(const uint16_t *x, int64_t K, const uint32_t *mask,
-                             int8_t *q, float *scale)
+/* absmax of one row over the regular columns */
+static float row_absmax(const uint16_t *x, int64_t K, const uint32_t *mask)
 {
     float absmax = 0.0f;
     for (int64_t j = 0; j < K; ++j) {
@@ -146,10 +145,46 @@ static void quantize_one_row(const uint16_t *x, int64_t K, const uint32_t *mask,
         float v = fabsf(half_to_float(x[j]));
         if (v > absmax) absmax = v;
     }
+    return absmax;
+}
+
+/* one row quantized with the absmax given: scale = absmax / 127, q = round(x / scale) */
+static void quantize_with_absmax(const uint16_t *x, int64_t K, const uint32_t *mask,
+                                 float absmax, int8_t *q, float *scale)
+{
     float s = absmax / 127.0f;
     *scale = s;
     for (int64_t j = 0; j < K; ++j)
         q[j] = (is_outlier(mask, j) || absmax == 0.0f) ? 0 : round_clamp_127(half_to_float(x[j]) / s);
+}
+
+/* one row: absmax over the regular columns, scale, quantize */
+static void quantize_one_row(const uint16_t *x, int64_t K, const uint32_t *mask,
+                             int8_t *q, float *scale)
+{
+    quantize_with_absmax(x, K, mask, row_absmax(x, K, mask), q, scale);
+}
+
+/* [P5] section "LLM.int8() 是怎么做到几乎无损的", item 2, as its snippet is written: one
+ * absmax for the whole activation tensor (over the regular columns, as for the rows). */
+static float tensor_absmax(const uint16_t *X, int64_t M, int64_t K, const uint32_t *mask)
+{
+    float absmax = 0.0f;
+    for (int64_t i = 0; i < M; ++i) {
+        float a = row_absmax(X + i * K, K, mask);
+        if (a > absmax) absmax = a;
+    }
+    return absmax;
+}
+
+int oracle_quantize_tensor(const uint16_t *X, int64_t M, int64_t K, const uint32_t *mask,
+                           int8_t *Xq, float *row_scale)
+{
+    if (!X || !mask || !Xq || !row_scale || M <= 0 || K <= 0) return ORACLE_EINVAL;
+    float absmax = tensor_absmax(X, M, K, mask);
+    for (int64_t i = 0; i < M; ++i)
+        quantize_with_absmax(X + i * K, K, mask, absmax, Xq + i * K, row_scale + i);
+    return 0;
 }
 
 int oracle_quantize_rows(const uint16_t *X, int64_t M, int64_t K, const uint32_t *mask,
@@ -205,8 +240,8 @@ int oracle_outlier_weights(const int8_t *Wq, const float *w_scale, int64_t N, in
  * their weights from it instead of rebuilding them from the int8 weights. */
 static int forward_rows(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,
                         const float *w_scale, const uint16_t *W16, const uint16_t *bias,
-                        int64_t N, float threshold, const int64_t *rows, int64_t n_rows,
-                        uint16_t *Y_rows, int32_t *A_rows)
+                        int64_t N, float threshold, int per_tensor, const int64_t *rows,
+                        int64_t n_rows, uint16_t *Y_rows, int32_t *A_rows)
 {
     if (!X || !Wq || !w_scale || !rows || !Y_rows || M <= 0 || N <= 0 || K <= 0 || n_rows < 0)
         return ORACLE_EINVAL;
@@ -231,6 +266,8 @@ static int forward_rows(const uint16_t *X, int64_t M, int64_t K, const int8_t *W
         } else status = oracle_outlier_weights(Wq, w_scale, N, K, cols, n_out, W_hat);
     }
 
+    /* per-tensor scale: one absmax over every row of X, whichever rows are returned */
+    float t_absmax = (status == 0 && per_tensor) ? tensor_absmax(X, M, K, mask) : 0.0f;
     if (status == 0) {
         #pragma omp parallel for schedule(dynamic, 1) reduction(min:status)
         for (int64_t r = 0; r < n_rows; ++r) {
@@ -238,7 +275,8 @@ static int forward_rows(const uint16_t *X, int64_t M, int64_t K, const int8_t *W
             int8_t *xq = (int8_t *)malloc((size_t)K);
             if (!xq) { status = ORACLE_EINVAL; continue; }
             float sx;
-            quantize_one_row(x, K, mask, xq, &sx);
+            if (per_tensor) quantize_with_absmax(x, K, mask, t_absmax, xq, &sx);
+            else quantize_one_row(x, K, mask, xq, &sx);
             for (int64_t n = 0; n < N; ++n) {
                 int32_t a;
                 int rc = dot_i8(xq, Wq + n * K, K, &a);
@@ -267,8 +305,18 @@ int oracle_linear_forward_rows(const uint16_t *X, int64_t M, int64_t K, const in
                                float threshold, const int64_t *rows, int64_t n_rows,
                                uint16_t *Y_rows, int32_t *A_rows)
 {
-    return forward_rows(X, M, K, Wq, w_scale, NULL, bias, N, threshold, rows, n_rows, Y_rows,
-                        A_rows);
+    return forward_rows(X, M, K, Wq, w_scale, NULL, bias, N, threshold, 0, rows, n_rows,
+                        Y_rows, A_rows);
+}
+
+int oracle_linear_forward_rows_ex(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,
+                                  const float *w_scale, const uint16_t *W16,
+                                  const uint16_t *bias, int64_t N, float threshold,
+                                  int per_tensor, const int64_t *rows, int64_t n_rows,
+                                  uint16_t *Y_rows, int32_t *A_rows)
+{
+    return forward_rows(X, M, K, Wq, w_scale, W16, bias, N, threshold, per_tensor != 0, rows,
+                        n_rows, Y_rows, A_rows);
 }
 
 int oracle_linear_forward_rows_w16(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,
@@ -278,7 +326,7 @@ int oracle_linear_forward_rows_w16(const uint16_t *X, int64_t M, int64_t K, cons
                                    int32_t *A_rows)
 {
     if (!W16) return ORACLE_EINVAL;
-    return forward_rows(X, M, K, Wq, w_scale, W16, bias, N, threshold, rows, n_rows, Y_rows,
+    return forward_rows(X, M, K, Wq, w_scale, W16, bias, N, threshold, 0, rows, n_rows, Y_rows,
                         A_rows);
 }
 
@@ -294,4 +342,45 @@ int oracle_linear_forward(const uint16_t *X, int64_t M, int64_t K, const int8_t 
                                             Y, NULL);
     free(rows);
     return status;
+}
+
+/* ------------------------------------------------------------------ activation statistics */
+
+static int cmp_float(const void *a, const void *b)
+{
+    float x = *(const float *)a, y = *(const float *)b;
+    return (x > y) - (x < y);
+}
+
+/* [P2] section 5.1 (statistics before choosing a threshold): the largest |x|, the 0.99
+ * quantile of |x| over every element (order statistics of the sorted values, linear
+ * interpolation between the two around position 0.99 (n - 1)), their ratio
+ * max / (q99 + 1e-6), and the absmax of every column.  out: {max, q99, ratio}. */
+int oracle_activation_stats(const uint16_t *X, int64_t M, int64_t K, float *col_absmax,
+                            double *out)
+{
+    if (!X || !out || M <= 0 || K <= 0) return ORACLE_EINVAL;
+    int64_t n = M * K;
+    float *v = (float *)malloc((size_t)n * sizeof(float));
+    if (!v) return ORACLE_EINVAL;
+    float mx = 0.0f;
+    for (int64_t j = 0; j < K && col_absmax; ++j) col_absmax[j] = 0.0f;
+    for (int64_t i = 0; i < M; ++i)
+        for (int64_t j = 0; j < K; ++j) {
+            float a = fabsf(half_to_float(X[i * K + j]));
+            v[i * K + j] = a;
+            if (a > mx) mx = a;
+            if (col_absmax && a > col_absmax[j]) col_absmax[j] = a;
+        }
+    qsort(v, (size_t)n, sizeof(float), cmp_float);
+    double pos = 0.99 * (double)(n - 1);
+    int64_t lo = (int64_t)floor(pos);
+    double frac = pos - (double)lo;
+    double a = v[lo], b = lo + 1 < n ? v[lo + 1] : v[lo];
+    double q99 = a + frac * (b - a);
+    out[0] = mx;
+    out[1] = q99;
+    out[2] = (double)mx / (q99 + 1e-6);
+    free(v);
+    return 0;
 }

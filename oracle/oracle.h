@@ -85,6 +85,28 @@ int oracle_linear_forward_rows_w16(const uint16_t *X, int64_t M, int64_t K, cons
                                    const int64_t *rows, int64_t n_rows, uint16_t *Y_rows,
                                    int32_t *A_rows);
 
+/* [P5] section "LLM.int8() 是怎么做到几乎无损的", item 2, with its snippet's granularity: one
+ * scale for the whole activation tensor, absmax over every row and the regular columns,
+ * divided by 127; each row quantized with it as oracle_quantize_rows does.  row_scale[i] holds
+ * that one scale for every row. */
+int oracle_quantize_tensor(const uint16_t *X, int64_t M, int64_t K, const uint32_t *mask,
+                           int8_t *Xq, float *row_scale);
+
+/* The layer with both options: W16 (nullable) as in oracle_linear_forward_rows_w16, and
+ * per_tensor != 0 for one activation scale over the whole of X (oracle_quantize_tensor). */
+int oracle_linear_forward_rows_ex(const uint16_t *X, int64_t M, int64_t K, const int8_t *Wq,
+                                  const float *w_scale, const uint16_t *W16,
+                                  const uint16_t *bias, int64_t N, float threshold,
+                                  int per_tensor, const int64_t *rows, int64_t n_rows,
+                                  uint16_t *Y_rows, int32_t *A_rows);
+
+/* [P2] section 5.1: statistics of |X| for choosing a threshold.  col_absmax: float [K]
+ * (nullable), the largest |X[i,j]| of each column; out: double [3] = {max |X|, the 0.99
+ * quantile of |X| over all M K values (linear interpolation at position 0.99 (M K - 1) of the
+ * sorted values), max / (q99 + 1e-6)}. */
+int oracle_activation_stats(const uint16_t *X, int64_t M, int64_t K, float *col_absmax,
+                            double *out);
+
 #ifdef __cplusplus
 }
 #endif
