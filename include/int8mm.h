@@ -47,6 +47,10 @@ typedef struct CUstream_st *int8mm_stream_t; /* the same type as cudaStream_t */
 #define INT8MM_ERR_TIMEOUT (-8)      /* device side: a bounded wait gave up */
 #define INT8MM_ERR_OVERFLOW (-9)     /* device side: an outlier count beyond K */
 #define INT8MM_ERR_SCRATCH (-10)     /* shape beyond int8_linear_forward_noalloc's scratch */
+#define INT8MM_ERR_FLAGS (-11)       /* unknown bits in the flags of int8_linear_forward_ex */
+
+/* flags of int8_linear_forward_ex */
+#define INT8MM_PER_TENSOR_SCALE 1u   /* one activation scale for the whole of X */
 
 /* Bytes of the static device scratch behind int8_linear_forward_noalloc (per device). */
 #define INT8MM_NOALLOC_SCRATCH_BYTES (512 * 1024)
@@ -115,6 +119,37 @@ int int8_linear_forward_fp16w(const void *X, int M, int K, const int8_t *Wq,
                               const float *w_scale, const void *W16, const void *bias, int N,
                               float threshold, void *Y, void *workspace, size_t ws_bytes,
                               int8mm_stream_t stream);
+
+/*
+ * int8_linear_forward with every option of the layer:
+ *   W16    [in]  NULL, or the layer's fp16 weights as for int8_linear_forward_fp16w
+ *   flags  [in]  0, or INT8MM_PER_TENSOR_SCALE: one activation scale for the whole of X,
+ *                sx = (max over every row i and regular column j of |X[i,j]|) / 127, every
+ *                row quantized with it ([P5] section "LLM.int8() 是怎么做到几乎无损的", item 2,
+ *                as its snippet is written; the default one-per-row scale follows the
+ *                vector-wise reading of [P2]).  Other bits: INT8MM_ERR_FLAGS.
+ *   acc    [out] NULL, or int32 [M, N]: the int8 accumulators, as int8_linear_forward_acc
+ * Every other argument, the workspace and the error codes are as for int8_linear_forward.
+ */
+int int8_linear_forward_ex(const void *X, int M, int K, const int8_t *Wq, const float *w_scale,
+                           const void *W16, const void *bias, int N, float threshold,
+                           unsigned flags, void *Y, int32_t *acc, void *workspace,
+                           size_t ws_bytes, int8mm_stream_t stream);
+
+/*
+ * Statistics of the layer's input for choosing the threshold ([P2] section 5.1, which
+ * compares the largest |x| with its 0.99 quantile: a ratio far above 1 flags outliers), over
+ * every element of X:
+ *   out        [out] double [3] (device): max |X|; q99 = the 0.99 quantile of |X| (the sorted
+ *                    values interpolated linearly at position 0.99 (M K - 1)); max / (q99 + 1e-6)
+ *   col_absmax [out] float32 [K], or NULL: max_i |X[i,j]| of each column (a column is an
+ *                    outlier when this exceeds the threshold)
+ *   workspace  [scratch] ws_bytes >= int8_activation_stats_workspace_size(), 256-byte aligned
+ * M K must be below 2^32.  NaN or infinite inputs give unspecified statistics.
+ */
+size_t int8_activation_stats_workspace_size(void);
+int int8_activation_stats(const void *X, int M, int K, float *col_absmax, double *out,
+                          void *workspace, size_t ws_bytes, int8mm_stream_t stream);
 
 /*
  * The two halves of int8_linear_forward, for callers that time or schedule them apart:

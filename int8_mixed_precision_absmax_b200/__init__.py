@@ -27,10 +27,12 @@ __all__ = [
     "int8_linear_quantize", "int8_linear_matmul", "int8_linear_forward_acc",
     "int8_quantize_rows", "int8_gemm_i32", "int8_outlier_weights",
     "int8_read_device_status", "int8_status_string", "int8_linear_forward_noalloc",
-    "int8_linear_forward_fp16w", "Int8Linear", "DEFAULT_THRESHOLD",
+    "int8_linear_forward_fp16w", "int8_linear_forward_ex", "PER_TENSOR_SCALE",
+    "int8_activation_stats", "Int8Linear", "DEFAULT_THRESHOLD",
 ]
 
 DEFAULT_THRESHOLD = 6.0
+PER_TENSOR_SCALE = 1  # int8_linear_forward_ex flag: one activation scale for the whole of X
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libint8mm.so")
 _lib = None
@@ -73,10 +75,16 @@ def load_library():
         lib.int8_read_device_status.argtypes = [p, p]
         lib.int8_linear_forward_noalloc.argtypes = [p, i, i, p, p, p, i, f, p, p, p]
         lib.int8_linear_forward_fp16w.argtypes = [p, i, i, p, p, p, p, i, f, p, p, sz, p]
+        lib.int8_linear_forward_ex.argtypes = [p, i, i, p, p, p, p, i, f, ctypes.c_uint, p, p,
+                                               p, sz, p]
+        lib.int8_activation_stats_workspace_size.argtypes = []
+        lib.int8_activation_stats_workspace_size.restype = sz
+        lib.int8_activation_stats.argtypes = [p, i, i, p, p, p, sz, p]
         for name in ("int8_quant_weight", "int8_linear_forward", "int8_linear_quantize",
                      "int8_linear_matmul", "int8_linear_forward_acc", "int8_quantize_rows",
                      "int8_gemm_i32", "int8_outlier_weights", "int8_read_device_status",
-                     "int8_linear_forward_noalloc", "int8_linear_forward_fp16w"):
+                     "int8_linear_forward_noalloc", "int8_linear_forward_fp16w",
+                     "int8_linear_forward_ex", "int8_activation_stats"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -196,6 +204,56 @@ def int8_linear_forward_fp16w(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.
         _ptr(Y), _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream, X.device))),
         "int8_linear_forward_fp16w")
     return Y
+
+
+def int8_linear_forward_ex(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                           bias: torch.Tensor | None, threshold: float = DEFAULT_THRESHOLD,
+                           W16: torch.Tensor | None = None, per_tensor: bool = False,
+                           Y: torch.Tensor | None = None, acc: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The layer with every option: the kept fp16 weights W16 (or None), one activation scale
+    for the whole of X (per_tensor), and the int32 accumulators written to acc (or not)."""
+    _need(X, torch.float16, "X", 2)
+    _need(Wq, torch.int8, "Wq", 2)
+    _need(w_scale, torch.float32, "w_scale", 1)
+    M, K = X.shape
+    N = Wq.shape[0]
+    if W16 is not None:
+        _need(W16, torch.float16, "W16", 2)
+        if tuple(W16.shape) != (N, K):
+            raise ValueError(f"W16 must be [{N}, {K}], got {tuple(W16.shape)}")
+    if bias is not None:
+        _need(bias, torch.float16, "bias", 1)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    _need(Y, torch.float16, "Y", 2)
+    if acc is not None:
+        _need(acc, torch.int32, "acc", 2)
+    if workspace is None:
+        n = int8_linear_workspace_size(M, N, K)
+        workspace = torch.zeros(max(n, 256), dtype=torch.uint8, device=X.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    flags = PER_TENSOR_SCALE if per_tensor else 0
+    _check(load_library().int8_linear_forward_ex(
+        _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(W16), _ptr(bias), N, float(threshold),
+        flags, _ptr(Y), _ptr(acc), _ptr(workspace), workspace.numel(),
+        ctypes.c_void_p(_stream(stream, X.device))), "int8_linear_forward_ex")
+    return Y
+
+
+def int8_activation_stats(X: torch.Tensor, stream=None):
+    """Statistics of |X| for choosing the threshold: (max, q99, max / (q99 + 1e-6)) as a
+    float64 tensor of 3 on the device, and the column absmax [K] (float32)."""
+    _need(X, torch.float16, "X", 2)
+    M, K = X.shape
+    out = torch.empty(3, dtype=torch.float64, device=X.device)
+    col = torch.empty(K, dtype=torch.float32, device=X.device)
+    ws = torch.empty(int(load_library().int8_activation_stats_workspace_size()),
+                     dtype=torch.uint8, device=X.device)
+    _check(load_library().int8_activation_stats(
+        _ptr(X), M, K, _ptr(col), _ptr(out), _ptr(ws), ws.numel(),
+        ctypes.c_void_p(_stream(stream, X.device))), "int8_activation_stats")
+    return out, col
 
 
 def int8_linear_forward_noalloc(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
@@ -339,11 +397,14 @@ class Int8Linear:
     quantizes its activations per row on the fly and routes the columns whose magnitude
     exceeds ``threshold`` through fp16.  With ``has_fp16_weights=False`` (the default) only
     the int8 weights are kept and the outlier columns use fp16(Wq * w_scale); with True the
-    layer also keeps the fp16 weight and the outlier columns use it.
+    layer also keeps the fp16 weight and the outlier columns use it.  With
+    ``per_tensor_activation=True`` one activation scale serves the whole input (the default is
+    one per row).
     """
 
     def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None,
-                 threshold: float = DEFAULT_THRESHOLD, has_fp16_weights: bool = False):
+                 threshold: float = DEFAULT_THRESHOLD, has_fp16_weights: bool = False,
+                 per_tensor_activation: bool = False):
         if math.isnan(threshold):
             raise ValueError("threshold is NaN")
         self.out_features, self.in_features = weight.shape
@@ -352,6 +413,7 @@ class Int8Linear:
         self.W16 = weight if has_fp16_weights else None
         self.bias = None if bias is None else bias.to(torch.float16).contiguous()
         self.threshold = float(threshold)
+        self.per_tensor_activation = bool(per_tensor_activation)
         self._workspace = None
         self._ws_rows = 0
 
@@ -365,7 +427,10 @@ class Int8Linear:
         lead = X.shape[:-1]
         X2 = X.reshape(-1, self.in_features).contiguous()
         ws = self._ws(X2.shape[0], X2.device)
-        if self.W16 is not None:
+        if self.per_tensor_activation:
+            Y = int8_linear_forward_ex(X2, self.Wq, self.w_scale, self.bias, self.threshold,
+                                       W16=self.W16, per_tensor=True, Y=out, workspace=ws)
+        elif self.W16 is not None:
             Y = int8_linear_forward_fp16w(X2, self.Wq, self.w_scale, self.W16, self.bias,
                                           self.threshold, Y=out, workspace=ws)
         else:

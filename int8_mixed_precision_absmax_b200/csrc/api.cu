@@ -81,6 +81,7 @@ const char* int8_status_string(int status) {
     case INT8MM_ERR_OVERFLOW: return "outlier count out of range";
     case INT8MM_ERR_SCRATCH:
       return "the shape needs more scratch than the library's static buffer holds";
+    case INT8MM_ERR_FLAGS: return "unknown flag bits";
     default: return "unknown status";
   }
 }
@@ -104,6 +105,13 @@ size_t int8_linear_workspace_size(int M, int N, int K) {
 }  // extern "C"
 
 namespace {
+
+// Options of the layer beyond its operands: the kept fp16 weights (nullable) and one
+// activation scale for the whole of X instead of one per row.
+struct LayerOpts {
+  const void* W16 = nullptr;
+  int per_tensor = 0;
+};
 
 struct ForwardPlan {
   WorkspaceLayout L;
@@ -136,9 +144,10 @@ int plan_forward(int M, int N, int K, const int8_t* Wq, const float* w_scale, vo
 GemvArgs gemv_args(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                    const void* bias, int N, float threshold, void* Y, int32_t* acc,
                    void* workspace, const ForwardPlan& p, const GemvPlan& gp,
-                   const void* W16 = nullptr) {
+                   const LayerOpts& o = LayerOpts()) {
   GemvArgs g;
-  g.W16 = static_cast<const __half*>(W16);
+  g.W16 = static_cast<const __half*>(o.W16);
+  g.per_tensor = o.per_tensor;
   g.X = static_cast<const __half*>(X);
   g.M = M;
   g.K = K;
@@ -164,9 +173,11 @@ GemvArgs gemv_args(const void* X, int M, int K, const int8_t* Wq, const float* w
 
 SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                      const void* bias, int N, float threshold, void* Y, int32_t* acc,
-                     const ForwardPlan& p, const SmallPlan& sp, const void* W16 = nullptr) {
+                     const ForwardPlan& p, const SmallPlan& sp,
+                     const LayerOpts& o = LayerOpts()) {
   SmallArgs a;
-  a.W16 = static_cast<const __half*>(W16);
+  a.W16 = static_cast<const __half*>(o.W16);
+  a.per_tensor = o.per_tensor;
   a.X = static_cast<const __half*>(X);
   a.M = M;
   a.K = K;
@@ -187,7 +198,8 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
 // is 16 rows x every k-block, each k-block landing as a 128-byte-swizzled 16 x 128 tile.
 int run_decode(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                const void* bias, int N, float threshold, void* Y, int32_t* acc, int32_t* status,
-               const DecodePlan& dp, cudaStream_t stream, bool pdl, const void* W16 = nullptr) {
+               const DecodePlan& dp, cudaStream_t stream, bool pdl,
+               const LayerOpts& o = LayerOpts()) {
   CUtensorMap map;
   const uint64_t dims[3] = {128, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 128)};
   const uint64_t strides[2] = {static_cast<uint64_t>(K), 128};
@@ -203,29 +215,31 @@ int run_decode(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   a.threshold = effective_threshold(threshold);
   a.Wq = Wq;
   a.w_scale = w_scale;
-  a.W16 = static_cast<const __half*>(W16);
+  a.W16 = static_cast<const __half*>(o.W16);
   a.bias = static_cast<const __half*>(bias);
   a.Y = static_cast<__half*>(Y);
   a.acc = acc;
+  a.per_tensor = o.per_tensor;
   a.status = status;
   return launch_status(launch_decode(map, a, dp, stream, pdl));
 }
 
 int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_scale, int N,
                  float threshold, void* workspace, const ForwardPlan& p, cudaStream_t stream,
-                 bool pdl_first, const void* W16 = nullptr) {
+                 bool pdl_first, const LayerOpts& o = LayerOpts()) {
   if (M <= kSmallMP) {
     if (plan_decode(M, N, K).fits) return INT8MM_OK;  // one kernel does everything
     const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
     if (gp.fits) {
       const GemvArgs g = gemv_args(X, M, K, Wq, w_scale, nullptr, N, threshold, nullptr, nullptr,
-                                   workspace, p, gp);
+                                   workspace, p, gp, o);
       return launch_status(launch_few_quant(g, gp, stream, pdl_first));
     }
     if (small_path_fits(M, K)) return INT8MM_OK;  // one kernel does everything: see run_matmul
   }
+  float* word_max = o.per_tensor ? at<float>(workspace, p.L.wmax) : nullptr;
   int rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
-                                        effective_threshold(threshold), p.mask, stream,
+                                        effective_threshold(threshold), p.mask, word_max, stream,
                                         pdl_first));
   if (rc) return rc;
   RowQuantArgs rq;
@@ -241,9 +255,10 @@ int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_s
   rq.n_out = p.header + 1;
   rq.Wq = Wq;
   rq.w_scale = w_scale;
-  rq.W16 = static_cast<const __half*>(W16);
+  rq.W16 = static_cast<const __half*>(o.W16);
   rq.wo = p.wo;
   rq.N = N;
+  rq.word_max = word_max;
   rq.status = p.header;
   return launch_status(launch_rowquant(rq, stream, true));
 }
@@ -251,16 +266,16 @@ int run_quantize(const void* X, int M, int K, const int8_t* Wq, const float* w_s
 int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                const void* bias, int N, float threshold, void* Y, int32_t* acc,
                void* workspace, const ForwardPlan& p, cudaStream_t stream, bool pdl,
-               const void* W16 = nullptr) {
+               const LayerOpts& o = LayerOpts()) {
   if (M <= kSmallMP) {
     const DecodePlan dp = plan_decode(M, N, K);
     if (dp.fits)
       return run_decode(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p.header, dp, stream,
-                        pdl, W16);
+                        pdl, o);
     const GemvPlan gp = plan_gemv(M, N, K, device_sm_count());
     if (gp.fits) {
       const GemvArgs g = gemv_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace,
-                                   p, gp, W16);
+                                   p, gp, o);
       // Wq viewed as [K/128 k-blocks][N rows][128 bytes]: one box is 32 rows x 8 k-blocks,
       // each k-block landing as a 128-byte-swizzled 32 x 128 tile
       CUtensorMap map;
@@ -275,7 +290,7 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   }
   if (small_path_fits(M, K)) {
     const SmallPlan sp = plan_small(M, N, K);
-    const SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p, sp, W16);
+    const SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, p, sp, o);
     CUtensorMap map;
     if (!encode_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kSmallBN))
       return INT8MM_ERR_CUDA;
@@ -306,19 +321,19 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
 int forward_impl(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                  const void* bias, int N, float threshold, void* Y, int32_t* acc,
                  void* workspace, size_t ws_bytes, cudaStream_t stream,
-                 const void* W16 = nullptr) {
+                 const LayerOpts& o = LayerOpts()) {
   if (!X || !Y) return INT8MM_ERR_NULL;
   if (!aligned16(X) || !aligned16(Y) || (bias && !aligned16(bias)) || (acc && !aligned16(acc)) ||
-      (W16 && !aligned16(W16)))
+      (o.W16 && !aligned16(o.W16)))
     return INT8MM_ERR_ALIGN;
   if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
   ForwardPlan p;
   int rc = plan_forward(M, N, K, Wq, w_scale, workspace, ws_bytes, p);
   if (rc) return rc;
-  if ((rc = run_quantize(X, M, K, Wq, w_scale, N, threshold, workspace, p, stream, true, W16)))
+  if ((rc = run_quantize(X, M, K, Wq, w_scale, N, threshold, workspace, p, stream, true, o)))
     return rc;
   return run_matmul(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace, p, stream, true,
-                    W16);
+                    o);
 }
 
 }  // namespace
@@ -337,8 +352,40 @@ int int8_linear_forward_fp16w(const void* X, int M, int K, const int8_t* Wq,
                               float threshold, void* Y, void* workspace, size_t ws_bytes,
                               int8mm_stream_t stream) {
   if (!W16) return INT8MM_ERR_NULL;
+  LayerOpts o;
+  o.W16 = W16;
   return forward_impl(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, workspace, ws_bytes,
-                      reinterpret_cast<cudaStream_t>(stream), W16);
+                      reinterpret_cast<cudaStream_t>(stream), o);
+}
+
+size_t int8_activation_stats_workspace_size(void) { return stats_workspace_bytes(); }
+
+int int8_activation_stats(const void* X, int M, int K, float* col_absmax, double* out,
+                          void* workspace, size_t ws_bytes, int8mm_stream_t stream) {
+  if (!X || !out) return INT8MM_ERR_NULL;
+  int rc = check_shape(M, 1, K);
+  if (rc) return rc;
+  if (static_cast<long long>(M) * K >= (1ll << 32)) return INT8MM_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(out) || (col_absmax && !aligned16(col_absmax)))
+    return INT8MM_ERR_ALIGN;
+  if (!workspace || !aligned256(workspace) || ws_bytes < stats_workspace_bytes())
+    return INT8MM_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  return launch_status(launch_activation_stats(static_cast<const __half*>(X), M, K, col_absmax,
+                                               out, workspace, device_sm_count(),
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int int8_linear_forward_ex(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
+                           const void* W16, const void* bias, int N, float threshold,
+                           unsigned flags, void* Y, int32_t* acc, void* workspace,
+                           size_t ws_bytes, int8mm_stream_t stream) {
+  if (flags & ~static_cast<unsigned>(INT8MM_PER_TENSOR_SCALE)) return INT8MM_ERR_FLAGS;
+  LayerOpts o;
+  o.W16 = W16;
+  o.per_tensor = (flags & INT8MM_PER_TENSOR_SCALE) ? 1 : 0;
+  return forward_impl(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), o);
 }
 
 int int8_linear_forward_acc(const void* X, int M, int K, const int8_t* Wq,
@@ -390,7 +437,8 @@ int int8_quantize_rows(const void* X, int M, int K, float threshold, int8_t* Xq,
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   uint32_t* mask = at<uint32_t>(workspace, L.mask);
   if ((rc = launch_status(launch_colmask(static_cast<const __half*>(X), M, K,
-                                         effective_threshold(threshold), mask, stream, false))))
+                                         effective_threshold(threshold), mask, nullptr, stream,
+                                         false))))
     return rc;
   RowQuantArgs rq = {};
   rq.X = static_cast<const __half*>(X);

@@ -330,7 +330,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
       const __half2 h2 = *reinterpret_cast<const __half2*>(&word);
       m = __hmax(m, (lane & 1) ? __high2half(h2) : __low2half(h2));
     }
-    const float mf = __half2float(m);
+    float mf = __half2float(m);
+    if (a.per_tensor)  // one scale for all rows: the largest row absmax (rows past M hold 0)
+#pragma unroll
+      for (int o = 1; o < kDTok; o <<= 1) mf = fmaxf(mf, __shfl_xor_sync(0x000000FFu, mf, o));
     sx_l = __fdiv_rn(mf, 127.0f);
     rcp_l = mf > 0.0f ? __frcp_rn(sx_l) : 0.0f;
     if (warp == 0) sh.sx[lane] = sx_l;

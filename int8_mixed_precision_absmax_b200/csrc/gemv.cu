@@ -249,6 +249,9 @@ __global__ void __launch_bounds__(kQThreads) few_quant_kernel(const GemvArgs a) 
     const uint32_t local = smem_addr(&sh.rowmax_local[i]);
     float m = 0.0f;
     for (int q = 0; q < Q; ++q) m = fmaxf(m, ld_cluster_f32(map_rank(local, q)));
+    if (a.per_tensor)  // one scale for all rows: the largest row absmax (rows past M hold 0)
+#pragma unroll
+      for (int o = 1; o < MT; o <<= 1) m = fmaxf(m, __shfl_xor_sync((1u << MT) - 1u, m, o));
     const float sc = __fdiv_rn(m, 127.0f);
     sh.sx[i] = (i < M) ? sc : 0.0f;
     sh.rcp[i] = (i < M && m > 0.0f) ? __frcp_rn(sc) : 0.0f;

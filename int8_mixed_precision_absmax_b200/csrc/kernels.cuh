@@ -32,7 +32,7 @@ constexpr int kSmallMaxSplits = 8;       // CTAs per cluster (portable cluster s
 constexpr int kSmallMaxKbPerSplit = 16;  // 128-byte k-blocks of X / Xq one CTA keeps in smem
 
 struct WorkspaceLayout {
-  size_t header, mask, cols, xscale, xq, xo, wo, few_xq, few_xo, few_sx, total;
+  size_t header, mask, wmax, cols, xscale, xq, xo, wo, few_xq, few_xo, few_sx, total;
   int ldo;
 };
 
@@ -44,6 +44,7 @@ inline WorkspaceLayout workspace_layout(int M, int N, int K) {
   size_t off = 0;
   L.header = off; off = align256(off + 64 * sizeof(int32_t));
   L.mask = off;   off = align256(off + static_cast<size_t>((K + 31) / 32) * sizeof(uint32_t));
+  L.wmax = off;   off = align256(off + static_cast<size_t>((K + 31) / 32) * sizeof(float));
   L.cols = off;   off = align256(off + static_cast<size_t>(K) * sizeof(int32_t));
   L.xscale = off; off = align256(off + static_cast<size_t>(M) * sizeof(float));
   L.xq = off;     off = align256(off + static_cast<size_t>(M) * K);
@@ -68,8 +69,10 @@ inline WorkspaceLayout workspace_layout(int M, int N, int K) {
 cudaError_t launch_quant_weight(const __half* W, int N, int K, int8_t* Wq, float* w_scale,
                                 cudaStream_t stream);
 
+// word_max (nullable): per 32-column word of the mask, the largest |x| over the word's regular
+// columns and every row (the per-tensor activation scale is the largest of them / 127)
 cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint32_t* mask,
-                           cudaStream_t stream, bool pdl);
+                           float* word_max, cudaStream_t stream, bool pdl);
 
 cudaError_t launch_outlier_weights(const int8_t* Wq, const float* w_scale, int N, int K,
                                    const int32_t* cols, const int32_t* n_out, __half* W_hat,
@@ -91,6 +94,7 @@ struct RowQuantArgs {
   const __half* W16;    // nullable: the layer's fp16 weights [N, K] for the outlier columns
   __half* wo;
   int N;
+  const float* word_max;  // nullable: one activation scale for all rows from colmask's maxima
   int32_t* status;
 };
 cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl);
@@ -107,6 +111,7 @@ struct SmallArgs {
   int32_t* acc;          // nullable: also write the int32 accumulators
   int splits;            // CTAs per cluster, each owning a K-slice
   int stages;            // depth of the Wq ring
+  int per_tensor;        // one activation scale for all rows (the largest row absmax)
   int32_t* status;
 };
 struct SmallPlan {
@@ -136,6 +141,7 @@ struct GemvArgs {
   float* sx;             // [16] row scales
   int32_t* cols;         // [K] outlier columns, ascending
   int32_t* n_out;        // outlier count
+  int per_tensor;        // one activation scale for all rows (the largest row absmax)
   int32_t* status;
 };
 struct GemvPlan {
@@ -148,6 +154,13 @@ cudaError_t launch_gemv(const CUtensorMap& map_wq, const GemvArgs& a, const Gemv
                         cudaStream_t stream, bool pdl);
 int device_sm_count();
 
+// Statistics of |X| (stats.cu): column absmax (nullable), and out[3] = {max, q99, ratio}
+// (device doubles); workspace of stats_workspace_bytes() (the |x| histogram).
+size_t stats_workspace_bytes();
+cudaError_t launch_activation_stats(const __half* X, int M, int K, float* col_absmax,
+                                    double* out, void* workspace, int num_sms,
+                                    cudaStream_t stream);
+
 // One-launch layer for M <= 8 tokens (decode.cu): no workspace.
 struct DecodeArgs {
   const __half* X;
@@ -159,6 +172,7 @@ struct DecodeArgs {
   const __half* bias;
   __half* Y;
   int32_t* acc;          // nullable: also write the int32 accumulators
+  int per_tensor;        // one activation scale for all rows (the largest row absmax)
   int32_t* status;
 };
 struct DecodePlan {

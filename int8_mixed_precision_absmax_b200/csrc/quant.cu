@@ -170,7 +170,8 @@ __device__ __forceinline__ uint32_t cm_cluster_rank() {
 
 __global__ void __launch_bounds__(kCMThreads) colmask_kernel(const __half* __restrict__ X, int M,
                                                              int K, float threshold,
-                                                             uint32_t* __restrict__ mask) {
+                                                             uint32_t* __restrict__ mask,
+                                                             float* __restrict__ word_max) {
   __shared__ __half2 red[kCMThreads / 32][8][4];
   __shared__ __half cmax_local[kCMStrip];  // this CTA's column maxima (read by CTA 0)
   const int strip = blockIdx.x / kCMCluster;
@@ -255,6 +256,12 @@ __global__ void __launch_bounds__(kCMThreads) colmask_kernel(const __half* __res
     const uint32_t bits = __ballot_sync(0xffffffffu, cm > threshold);
     const int word = strip * 2 + threadIdx.x / 32;
     if (lane == 0 && word * 32 < K) mask[word] = bits;
+    if (word_max) {  // the largest |x| of the word's regular columns (columns past K hold 0)
+      float rm = cm > threshold ? 0.0f : cm;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, o));
+      if (lane == 0 && word * 32 < K) word_max[word] = rm;
+    }
   }
   // no CTA leaves while CTA 0 may still read its shared memory
   asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
@@ -262,7 +269,7 @@ __global__ void __launch_bounds__(kCMThreads) colmask_kernel(const __half* __res
 }
 
 cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint32_t* mask,
-                           cudaStream_t stream, bool pdl) {
+                           float* word_max, cudaStream_t stream, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(((K + kCMStrip - 1) / kCMStrip) * kCMCluster);
   cfg.blockDim = dim3(kCMThreads);
@@ -276,7 +283,7 @@ cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint3
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, colmask_kernel, X, M, K, threshold, mask);
+  return cudaLaunchKernelEx(&cfg, colmask_kernel, X, M, K, threshold, mask, word_max);
 }
 
 // ------------------------------------------------------------------ rows + outlier operands
@@ -412,6 +419,14 @@ __device__ void quantize_rows_block(const RowQuantArgs& a, RowQuantShared& S, in
   __syncthreads();
   float amax = 0.0f;
   for (int w = rl * (tpr / 32); w < (rl + 1) * (tpr / 32); ++w) amax = fmaxf(amax, S.red[w]);
+  if (a.word_max) {  // one scale for all rows: the largest regular |x| of the whole tensor
+    const int lane = threadIdx.x & 31;
+    float g = 0.0f;
+    for (int w = lane; w < (K + 31) / 32; w += 32) g = fmaxf(g, __ldcg(a.word_max + w));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
+    amax = g;
+  }
   if (!live) return;
   const float s = __fdiv_rn(amax, 127.0f);
   if (lr == 0) a.xscale[i] = s;

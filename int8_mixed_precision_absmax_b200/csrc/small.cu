@@ -386,6 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m = 0.0f;
 #pragma unroll
         for (int r = 0; r < kSmallMaxSplits; ++r) m = fmaxf(m, peer[r]);
+        if (a.per_tensor)  // one scale for all rows: the largest row absmax (rows past M hold 0)
+#pragma unroll
+          for (int o = 1; o < kSmallMP; o <<= 1)
+            m = fmaxf(m, __shfl_xor_sync((1u << kSmallMP) - 1u, m, o));
         const float sc = __fdiv_rn(m, 127.0f);
         sh.sx[tz] = (tz < a.M) ? sc : 0.0f;
         sh.rcp[tz] = (tz < a.M && m > 0.0f) ? __frcp_rn(sc) : 0.0f;

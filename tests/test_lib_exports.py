@@ -44,7 +44,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(-9, 1):
+    for code in range(-11, 1):
         assert i8.int8_status_string(code) not in ("", "unknown status")
     assert i8.int8_status_string(-1234) == "unknown status"
 
@@ -98,3 +98,16 @@ def test_fp16_weight_entry_point_checks_its_weights(lib):
                                        8, 6.0, FAKE, FAKE, 1 << 20, None) == -3
     assert L.int8_linear_forward_fp16w(FAKE, 4, 32, FAKE, FAKE, FAKE, None, 8, math.nan, FAKE,
                                        FAKE, 1 << 20, None) == -4
+
+
+def test_extended_entry_points_check_their_arguments(lib):
+    L = lib
+    # unknown flag bits are rejected before anything else
+    assert L.int8_linear_forward_ex(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 2, FAKE, None,
+                                    FAKE, 1 << 20, None) == -11
+    assert L.int8_linear_forward_ex(None, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 1, FAKE, None,
+                                    FAKE, 1 << 20, None) == -1
+    assert L.int8_activation_stats(None, 4, 32, None, FAKE, FAKE, 1 << 20, None) == -1
+    assert L.int8_activation_stats(FAKE, 4, 40, None, FAKE, FAKE, 1 << 20, None) == -3
+    assert L.int8_activation_stats(FAKE, 4, 32, None, FAKE, FAKE, 16, None) == -5
+    assert L.int8_activation_stats_workspace_size() == 32768 * 4
