@@ -105,12 +105,21 @@ def load_peaks():
             "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+# the sources each timed kernel is built from (its own file and the shared headers)
+KERNEL_SOURCES = {"decode_kernel": "decode.cu", "gemm_kernel": "gemm.cu",
+                  "rowquant_kernel": "quant.cu", "colmask_kernel": "quant.cu",
+                  "gemv_kernel": "gemv.cu", "small_fused_kernel": "small.cu"}
+
+
+def kernel_source_hash(kernel: str | None = None) -> str:
+    """Hash of the sources of `kernel` (of every kernel source when None)."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    names = sorted(n for n in os.listdir(CSRC) if n.endswith((".cu", ".cuh")))
+    if kernel in KERNEL_SOURCES:
+        names = sorted([KERNEL_SOURCES[kernel], "kernels.cuh", "ptx.cuh"])
+    for name in names:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -122,7 +131,7 @@ def recorded_traffic(workload: str, kernel: str):
     with open(path) as f:
         rec = json.load(f)
     e = rec.get(workload, {}).get(kernel)
-    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+    if not e or e.get("kernel_source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
