@@ -485,7 +485,26 @@ __device__ void gather_weights(const RowQuantArgs& a, RowQuantShared& S, int wor
       const int n = static_cast<int>(u / groups);
       const int r0 = R0 + static_cast<int>(u % groups) * 8;
       uint32_t h[4] = {0u, 0u, 0u, 0u};
-      if (r0 < n_out && a.W16 != nullptr) {  // the layer's own fp16 weights
+      // eight outliers in consecutive columns from a multiple of 8 (every column, when the
+      // threshold is 0): one vector load of the row instead of eight
+      const int c0 = r0 < n_out ? S.cols[r0 - R0] : 0;
+      const bool dense = r0 + 8 <= n_out && (c0 & 7) == 0 && S.cols[r0 + 7 - R0] == c0 + 7;
+      if (dense && a.W16 != nullptr) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.W16 + static_cast<size_t>(n) * a.K + c0));
+        h[0] = v.x;
+        h[1] = v.y;
+        h[2] = v.z;
+        h[3] = v.w;
+      } else if (dense) {
+        const uint2 q = __ldg(reinterpret_cast<const uint2*>(a.Wq + static_cast<size_t>(n) * a.K + c0));
+        const float sc = a.w_scale[n];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int8_t code = static_cast<int8_t>(((e < 4 ? q.x : q.y) >> (8 * (e & 3))) & 0xFFu);
+          const float w = static_cast<float>(code) * sc;
+          h[e / 2] |= static_cast<uint32_t>(__half_as_ushort(__float2half_rn(w))) << (16 * (e & 1));
+        }
+      } else if (r0 < n_out && a.W16 != nullptr) {  // the layer's own fp16 weights
         const unsigned short* hrow =
             reinterpret_cast<const unsigned short*>(a.W16) + static_cast<size_t>(n) * a.K;
 #pragma unroll
