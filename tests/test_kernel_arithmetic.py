@@ -1,0 +1,123 @@
+"""The arithmetic shortcuts of the CUDA kernels, checked on the CPU against the plain definitions.
+
+The kernels replace a few operations of the layer by cheaper ones that give the same bits.
+Each test below restates one shortcut in numpy and compares it, exhaustively or over dense
+samples of binary16 inputs, with the definition it stands in for ([P5] "PyTorch 2.9 支持
+LLM.int8()" section "LLM.int8() 是怎么做到几乎无损的", item 2: q = round(x / scale) with
+scale = absmax / 127; [P2] "8位量化实战：离群值处理与显存优化避坑指南" section 2.3: a column
+is an outlier when |x| exceeds the threshold):
+
+* the quantizer (quant.cu quantize_chunk_fast, decode.cu quantize8): q = rne(x * r) with
+  r = 1 / s rounded to nearest, read off the low byte of fl(x * r + 1.5 * 2^23), and the IEEE
+  quotient x / s only where x * r lies within 2^-15 of a half-integer;
+* the threshold test on binary16 values against the threshold rounded down to binary16
+  (decode.cu);
+* int8 codes to float through the bit pattern 0x4B0000vv (decode.cu code_to_float);
+* the byte masks that zero the codes of outlier columns (quant.cu keep_mask, decode.cu
+  keep_masks).
+
+None of this imports the CUDA library or the oracle.
+"""
+import numpy as np
+import pytest
+
+F16_POS = np.arange(0x0000, 0x7C00, dtype=np.uint16).view(np.float16)  # 0 and every finite > 0
+MAGIC = np.float32(12582912.0)  # 1.5 * 2^23
+NEAR = 0.5 - 2.0 ** -15
+
+
+def _absmax_sample(n_random: int, seed: int) -> np.ndarray:
+    """Row maxima: the extremes, powers of two, their neighbours and random binary16 values."""
+    rng = np.random.default_rng(seed)
+    bits = {0x0001, 0x0002, 0x03FF, 0x0400, 0x0401, 0x3BFF, 0x3C00, 0x3C01, 0x4000, 0x57F0,
+            0x5800, 0x7BFE, 0x7BFF}
+    bits |= {0x0400 * e for e in range(1, 31)}
+    bits |= {0x0400 * e - 1 for e in range(1, 31)}
+    bits |= set(rng.integers(1, 0x7C00, size=n_random).tolist())
+    return np.array(sorted(bits), dtype=np.uint16).view(np.float16)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_fast_quantizer_equals_the_ieee_quotient_outside_the_near_tie_window(seed):
+    """Wherever |x * r - rne(x * r)| <= 1/2 - 2^-15 (with 2^-24 to spare for the kernel's rounded
+    residual), rne(x * r) equals rne(fl(x / s)); the codes fit in [-127, 127] without a clamp;
+    and the low byte of fl(x * r + 1.5 * 2^23) is the code in two's complement."""
+    flagged = total = wrong_fast = 0
+    for a in _absmax_sample(150, seed):
+        s = np.float32(a) / np.float32(127.0)          # IEEE float32 division
+        r = np.float32(1.0) / s                         # reciprocal rounded to nearest
+        x = F16_POS[F16_POS <= a].astype(np.float32)
+        x = np.concatenate([x, -x])
+        q_ref = np.rint(x / s)                          # fl(x / s), then ties to even
+        assert np.abs(q_ref).max() <= 127
+        t = x.astype(np.float64) * np.float64(r)        # exact: 11 x 24 significant bits
+        q_fast = np.rint(t)
+        d = t - q_fast                                  # exact
+        safe = np.abs(d) <= NEAR + 2.0 ** -24
+        np.testing.assert_array_equal(q_fast[safe], q_ref[safe])
+        # the low byte of fl(x * r + 1.5 * 2^23): the float32 sum of the exact product
+        tb = (t + np.float64(MAGIC)).astype(np.float32)
+        assert np.array_equal(tb.astype(np.float64) - np.float64(MAGIC), q_fast)
+        low = (tb.view(np.uint32) & 0xFF).astype(np.uint8)
+        np.testing.assert_array_equal(low, q_fast.astype(np.int64).astype(np.int8).view(np.uint8))
+        flagged += int((~safe).sum())
+        total += x.size
+        wrong_fast += int((q_fast != q_ref).sum())
+    # the exact route is taken for a small fraction of the values, never for most of them, and
+    # it is needed: rne(x * r) alone differs from rne(fl(x / s)) somewhere in the sample
+    assert 0 < flagged < total // 50
+    assert wrong_fast > 0
+
+
+def test_magic_constant_low_byte_for_every_int8_code_and_beyond():
+    q = np.arange(-70000, 70001, dtype=np.int64)
+    tb = (q.astype(np.float64) + np.float64(MAGIC)).astype(np.float32)
+    assert np.array_equal(tb.astype(np.float64) - np.float64(MAGIC), q.astype(np.float64))
+    np.testing.assert_array_equal(tb.view(np.uint32) & 0xFF, q & 0xFF)
+
+
+def _half_round_down(t: float) -> np.float16:
+    with np.errstate(over="ignore"):
+        h = np.float16(t)
+    if np.isnan(h) or (np.isfinite(t) and float(h) > t):
+        h = np.nextafter(np.float16(np.inf) if np.isnan(h) else h, np.float16(-np.inf))
+    return np.float16(h)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_threshold_against_its_binary16_round_down(seed):
+    """For every binary16 |x|: |x| > t (in float32) exactly when |x| > t rounded down to
+    binary16, so the kernels compare binary16 values directly."""
+    rng = np.random.default_rng(seed)
+    ts = [0.0, 1e-8, 6e-8, 1e-3, 0.5, 1.0, 5.999999523162842, 6.0, 6.000000476837158, 6.001953125,
+          6.0009765625, 65504.0, 65519.99609375, 65520.0, 1e6, np.inf]
+    ts += rng.uniform(0, 70000, size=300).astype(np.float32).tolist()
+    ts += F16_POS[rng.integers(0, F16_POS.size, size=200)].astype(np.float32).tolist()
+    ax = F16_POS.astype(np.float64)
+    for t in ts:
+        t32 = float(np.float32(t))
+        h = float(_half_round_down(t32))
+        assert h <= t32
+        np.testing.assert_array_equal(ax > t32, ax > h, err_msg=f"threshold {t32}")
+
+
+def test_int8_code_to_float_through_the_0x4b0000vv_pattern():
+    """float(code) = float32 bits (0x4B000000 | byte) ^ 0x80, minus 2^23 + 128, for every code."""
+    codes = np.arange(-128, 128, dtype=np.int64)
+    byte = codes.astype(np.int8).view(np.uint8).astype(np.uint32)
+    bits = (np.uint32(0x4B000000) | byte) ^ np.uint32(0x80)
+    val = bits.view(np.float32).astype(np.float64) - 8388736.0
+    np.testing.assert_array_equal(val, codes.astype(np.float64))
+
+
+def _keep_mask(bits4: int) -> int:
+    return (~((((bits4 * 0x204081) & 0xFFFFFFFF) & 0x01010101) * 0xFF)) & 0xFFFFFFFF
+
+
+def test_keep_mask_zeroes_exactly_the_outlier_bytes():
+    for bits in range(256):
+        lo, hi = _keep_mask(bits & 0xF), _keep_mask(bits >> 4)
+        word = lo | (hi << 32)
+        for e in range(8):
+            byte = (word >> (8 * e)) & 0xFF
+            assert byte == (0x00 if (bits >> e) & 1 else 0xFF), (bits, e, hex(word))
