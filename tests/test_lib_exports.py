@@ -111,3 +111,40 @@ def test_extended_entry_points_check_their_arguments(lib):
     assert L.int8_activation_stats(FAKE, 4, 40, None, FAKE, FAKE, 1 << 20, None) == -3
     assert L.int8_activation_stats(FAKE, 4, 32, None, FAKE, FAKE, 16, None) == -5
     assert L.int8_activation_stats_workspace_size() == 32768 * 4
+
+
+def test_remaining_entry_points_check_their_arguments(lib):
+    L = lib
+    big_k = 65536 + 16  # one 16-column step past the longest supported rows
+    assert L.int8_linear_forward(FAKE, 4, big_k, FAKE, FAKE, None, 8, 6.0, FAKE, FAKE, 1 << 30,
+                                 None) == -2
+    assert L.int8_linear_forward(FAKE, 4, 32, FAKE, FAKE, None, -8, 6.0, FAKE, FAKE, 1 << 20,
+                                 None) == -2
+    # the two halves of the forward
+    assert L.int8_linear_quantize(None, 4, 32, FAKE, FAKE, 8, 6.0, FAKE, 1 << 20, None) == -1
+    assert L.int8_linear_quantize(FAKE, 4, 32, FAKE, FAKE, 8, math.nan, FAKE, 1 << 20, None) == -4
+    assert L.int8_linear_quantize(FAKE, 0, 32, FAKE, FAKE, 8, 6.0, FAKE, 1 << 20, None) == -2
+    assert L.int8_linear_matmul(FAKE, 4, 32, FAKE, FAKE, None, 8, 6.0, None, FAKE, 1 << 20,
+                                None) == -1
+    assert L.int8_linear_matmul(FAKE, 4, 32, FAKE, FAKE, ctypes.c_void_p(0x10008), 8, 6.0, FAKE,
+                                FAKE, 1 << 20, None) == -3
+    # the accumulator output is required by the accumulating forward
+    assert L.int8_linear_forward_acc(FAKE, 4, 32, FAKE, FAKE, None, 8, 6.0, FAKE, None, FAKE,
+                                     1 << 20, None) == -1
+    # the outlier-weight diagnostic
+    assert L.int8_outlier_weights(FAKE, FAKE, 8, 32, None, FAKE, FAKE, None) == -1
+    assert L.int8_outlier_weights(FAKE, FAKE, 8, 40, FAKE, FAKE, FAKE, None) == -3
+
+
+def test_noalloc_entry_point_checks_before_touching_its_scratch(lib):
+    L = lib
+    # beyond the few-token kernels the static scratch serves: a clear error, no device work
+    assert L.int8_linear_forward_noalloc(FAKE, 17, 256, FAKE, FAKE, None, 128, 6.0, FAKE, None,
+                                         None) == -10
+    assert L.int8_linear_forward_noalloc(None, 8, 256, FAKE, FAKE, None, 128, 6.0, FAKE, None,
+                                         None) == -1
+    # the optional status word must be 4-byte aligned
+    assert L.int8_linear_forward_noalloc(FAKE, 8, 256, FAKE, FAKE, None, 128, 6.0, FAKE,
+                                         ctypes.c_void_p(0x10002), None) == -3
+    assert L.int8_linear_forward_noalloc(FAKE, 8, 256, FAKE, FAKE, None, 128, math.nan, FAKE,
+                                         None, None) == -4
