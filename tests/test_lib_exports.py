@@ -148,3 +148,31 @@ def test_noalloc_entry_point_checks_before_touching_its_scratch(lib):
                                          ctypes.c_void_p(0x10002), None) == -3
     assert L.int8_linear_forward_noalloc(FAKE, 8, 256, FAKE, FAKE, None, 128, math.nan, FAKE,
                                          None, None) == -4
+
+
+def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+    """The boundary is a C ABI: the header compiles as C99 with -pedantic, and a C program that
+    takes the address of every declared entry point links against the library (no C++ names
+    or types leak through)."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = declared_functions()
+    src = tmp_path / "abi.c"
+    src.write_text("#include \"int8mm.h\"\n#include <stdio.h>\n"
+                   "typedef void (*fn_t)(void);\n"
+                   "int main(void) {\n  fn_t fns[] = {\n"
+                   + "".join(f"    (fn_t)&{n},\n" for n in names)
+                   + "  };\n  printf(\"%d %s\\n\", (int)(sizeof fns / sizeof fns[0]),"
+                   " int8_status_string(INT8MM_ERR_SCRATCH));\n  return 0;\n}\n")
+    exe = tmp_path / "abi"
+    lib_dir = os.path.dirname(i8.library_path())
+    subprocess.check_call([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                           "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                           "-L", lib_dir, "-l:" + os.path.basename(i8.library_path()),
+                           "-Wl,-rpath," + lib_dir])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert int(out[0]) == len(names)
