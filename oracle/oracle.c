@@ -13,7 +13,7 @@
  *        section 2.3: Y = X_O . W_O (fp16) + quantize(X_R) . quantize(W_R) (int8),
  *        outlier column <=> column max |x| exceeds the threshold (default 6.0).
  *
- * Readings taken where the pages are silent or garbled (each is listed in the design doc):
+ * Readings taken where the pages are silent or garbled:
  *   - one activation scale per ROW of X, taken over the regular columns only;
  *   - "round" is round-half-to-even (torch.round), done with nearbyint/nearbyintf under
  *     the default FE_TONEAREST mode;
