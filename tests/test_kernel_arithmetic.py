@@ -121,3 +121,50 @@ def test_keep_mask_zeroes_exactly_the_outlier_bytes():
         for e in range(8):
             byte = (word >> (8 * e)) & 0xFF
             assert byte == (0x00 if (bits >> e) & 1 else 0xFF), (bits, e, hex(word))
+
+
+def test_decode_fragment_columns_are_one_permutation_for_both_operands():
+    """decode.cu: in k-step j of a 128-column k-block, lane (g, tig) of a warp feeds the int8 MMA
+    m16n8k32 the 8 consecutive columns L = 16 (4 (tig / 2) + j) + 8 (tig % 2) .. L + 7 of weight
+    rows g and g + 8 (read through the 128-byte swizzle: 16-byte chunk c of row r sits at
+    c ^ (r % 8)) and of token g's codes.  The MMA's k positions tig * 4 .. + 3 and 16 + tig * 4
+    .. + 3 then hold the same columns in both operands, so the dot product is unchanged; every
+    column of the k-block is used exactly once over the four k-steps; and the 16 lanes of each
+    half-warp read 16 different 8-byte bank pairs of the weight tile and of the codes (whose rows
+    start 16 bytes apart in bank space: row pitch K + 16 with K a multiple of 128)."""
+    used = []
+    for j in range(4):
+        k_to_col_a, k_to_col_b = {}, {}
+        for lane in range(32):
+            g, tig = lane >> 2, lane & 3
+            L = 16 * (4 * (tig >> 1) + j) + 8 * (tig & 1)
+            for r in (g, g + 8):
+                for half in range(2):                      # bytes 0-3, then 4-7
+                    for e in range(4):
+                        k = 16 * half + 4 * tig + e        # the MMA's k position
+                        # the weight byte the lane loads: swizzled address back to a column
+                        addr = r * 128 + (((4 * (tig >> 1) + j) ^ (r % 8)) << 4) + (tig & 1) * 8 \
+                            + 4 * half + e
+                        col = (((addr % 128) >> 4) ^ (r % 8)) * 16 + (addr % 16)
+                        assert col == L + 4 * half + e
+                        assert k_to_col_a.setdefault((r, k), col) == col
+                        k_to_col_a[("any", k)] = col
+            for half in range(2):
+                for e in range(4):
+                    k_to_col_b[16 * half + 4 * tig + e] = L + 4 * half + e
+        for k, col in k_to_col_b.items():
+            assert k_to_col_a[("any", k)] == col      # the same column in both operands
+        assert sorted(k_to_col_b.values()) == sorted(set(k_to_col_b.values()))
+        used += list(k_to_col_b.values())
+    assert sorted(used) == list(range(128))
+    for K in (128, 1024, 4096, 8192):
+        for j in range(4):
+            for half_warp in (range(16), range(16, 32)):
+                w_pairs, x_pairs = set(), set()
+                for lane in half_warp:
+                    g, tig = lane >> 2, lane & 3
+                    w_addr = g * 128 + (((4 * (tig >> 1) + j) ^ g) << 4) + (tig & 1) * 8
+                    x_addr = g * (K + 16) + 64 * (tig >> 1) + 8 * (tig & 1) + 16 * j
+                    w_pairs.add((w_addr // 8) % 16)
+                    x_pairs.add((x_addr // 8) % 16)
+                assert len(w_pairs) == 16 and len(x_pairs) == 16
