@@ -1,8 +1,6 @@
-"""The output-channel and token splits with the library's kernels on the GPU: one NCCL rank
-(the runs here have one GPU), so the collectives are copies, but the rank runs the whole path:
-for the channel split its slice of the weights quantized and multiplied by the kernels, joined
-by all_gather_into_tensor; for the token split the column maxima from the statistics kernel,
-their MAX all-reduce, the appended outlier row and the forward on the rows plus that row."""
+"""The output-channel split with the library's kernels on the GPU: one NCCL rank (the runs
+here have one GPU), so the gather is a copy, but the rank runs the whole path: its slice of
+the weights quantized and multiplied by the kernels, joined by all_gather_into_tensor."""
 import socket
 
 import numpy as np
@@ -13,7 +11,6 @@ import torch.distributed as dist
 import int8_mixed_precision_absmax_b200 as i8
 import oracle
 from int8_mixed_precision_absmax_b200 import colparallel as cp
-from int8_mixed_precision_absmax_b200 import rowparallel as rp
 from tests.gpu_helpers import assert_y_close, f16_bits, to_dev, to_np
 
 pytestmark = pytest.mark.gpu
@@ -46,20 +43,3 @@ def test_one_rank_split_equals_the_layer(nccl_group, M, K, N):
     assert_y_close(Y, Y_ref, f"split {M}x{K}x{N}")
     if N % 16 == 0:  # no padded channels: the same launches as the unsplit layer
         np.testing.assert_array_equal(f16_bits(Y), f16_bits(Y_one))
-
-
-@pytest.mark.parametrize("M,K,N", [(8, 4096, 4096), (40, 1024, 300)])
-def test_one_rank_token_split_equals_the_layer(nccl_group, M, K, N):
-    """8 rows become 9 with the appended one (the two-launch few-token path), 40 become 41 (the
-    tiled path); Y of the real rows against the oracle of the whole layer."""
-    rng = np.random.default_rng(3 * M + K + N)
-    X = rng.standard_normal((M, K))
-    X[:, rng.choice(K, size=4, replace=False)] *= 30.0
-    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
-    b = (rng.standard_normal(N) * 0.01).astype(np.float16)
-    X = X.astype(np.float16)
-    layer = rp.RowParallelInt8Linear(to_dev(W), to_dev(b), 6.0)
-    Y = to_np(layer(to_dev(X)))
-    assert Y.shape == (M, N)
-    Y_ref = oracle.linear_forward(X, to_np(layer.Wq), to_np(layer.w_scale), b, 6.0)
-    assert_y_close(Y, Y_ref, f"token split {M}x{K}x{N}")
