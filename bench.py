@@ -34,7 +34,7 @@ if ROOT not in sys.path:
 
 METRIC = "int8_linear_forward effective TOPS (2·M·N·K/s) and GB/s vs B200 roofline"
 UNIT = "TOPS"
-DEFAULT_WORKLOAD = "decode_q_proj"
+DEFAULT_WORKLOAD = "ffn_175b_f0.001_t6"
 INT8_OVER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 CSRC = os.path.join(ROOT, "int8_mixed_precision_absmax_b200", "csrc")
 
@@ -51,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch every step from Python")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     return ap.parse_args(argv)
 
@@ -187,6 +189,13 @@ class ClockSampler:
                 return float(v)
             except ValueError:
                 return None
+        # samples under load: power within half of the highest seen in the window (the window
+        # opens and closes with a quarter second of idle GPU)
+        pw = [num(r[3]) for r in rows]
+        top = max([p for p in pw if p is not None], default=None)
+        loaded = [r for r, p in zip(rows, pw) if top is None or (p is not None and p >= 0.5 * top)]
+        if len(loaded) >= 3:
+            rows = loaded
         sm = [num(r[1]) for r in rows if num(r[1]) is not None]
         smax = [num(r[2]) for r in rows if num(r[2]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -284,6 +293,7 @@ def run_reference(args):
         "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "threshold": w.threshold,
                    "parallelism": "rank 0 only (CPU oracle)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "host_cores": os.cpu_count(), "cpu_model": cpu_model(),
                          "sample": desc + f" per step, {steps} steps"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -297,21 +307,24 @@ def forward_path(M: int, N: int, K: int):
     """Which kernels one int8_linear_forward launches for this shape (the library's dispatch:
     api.cu with the plan functions of decode.cu, gemv.cu and small.cu)."""
     if M <= 8 and K % 128 == 0 and K <= 8192:
-        return {"name": "decode", "launches": 1, "quantize": [],
+        return {"name": "decode", "launches": 1, "quantize": [], "kernel": "decode_kernel",
                 "matmul": "decode_kernel (one launch: one CTA per 32 channels over all of K, X "
                           "statistics in every CTA, mma.sync int8 + fp16 outlier term)"}
     if M <= 16:
         if K % 128 == 0 and K <= 8192:
             return {"name": "few_tokens", "launches": 2, "quantize": ["few_quant_kernel"],
+                    "kernel": "gemv_kernel",
                     "matmul": "gemv_kernel (mma.sync int8 + fp16 outlier term)"}
-        return {"name": "cluster", "launches": 1, "quantize": [],
+        return {"name": "cluster", "launches": 1, "quantize": [], "kernel": "small_fused_kernel",
                 "matmul": "small_fused_kernel (tcgen05, one cluster per channel tile)"}
     return {"name": "tiled", "launches": 3, "quantize": ["colmask_kernel", "rowquant_kernel"],
+            "kernel": "gemm_kernel",
             "matmul": "gemm_kernel (int8 + fp16 tcgen05, fused epilogue)"}
 
 
-def graph_time_ms(fn, n: int, device) -> float:
-    """Average device time of fn() replayed back to back from one CUDA graph of n calls."""
+def graph_time_ms(fn, n: int, device, min_ms: float = 200.0) -> float:
+    """Average device time of fn() replayed back to back from one CUDA graph of n calls, over
+    at least `min_ms` of replays (CUDA events on the launching stream)."""
     import torch
     side = torch.cuda.Stream(device)
     side.wait_stream(torch.cuda.current_stream(device))
@@ -328,7 +341,11 @@ def graph_time_ms(fn, n: int, device) -> float:
         g.replay()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 10
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    reps = max(3, min(10000, int(min_ms / max(a.elapsed_time(b), 1e-3))))
     a.record()
     for _ in range(reps):
         g.replay()
@@ -339,8 +356,274 @@ def graph_time_ms(fn, n: int, device) -> float:
     return ms
 
 
+def op_counts(w, n_out: int):
+    """The method's own work: 2 M N (K - |O|) int8 operations and 2 M N |O| fp16 flops."""
+    return 2.0 * w.M * w.N * (w.K - n_out), 2.0 * w.M * w.N * n_out
+
+
+def tensor_roof_s(int8_ops: float, f16_flops: float, peaks) -> float:
+    """Seconds the work takes at the tensor peaks: int8 at the int8 peak, fp16 at the fp16 one."""
+    return int8_ops / (peaks["int8_tops"] * 1e12) + f16_flops / (peaks["f16_tflops"] * 1e12)
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+class Layer:
+    """One workload resident in HBM: rotating copies of X, Wq, w_scale, bias, Y and workspace,
+    enough that every step's operands have left L2 before they are read again."""
+
+    def __init__(self, w, rank: int, device, l2: int):
+        import torch
+        import int8_mixed_precision_absmax_b200 as i8
+        import synth
+        self.w = w
+        X_h, W_h, b_h, _ = synth.make_inputs(w, seed=w.seed + rank)
+        self.X_h, self.b_h = X_h, b_h
+        self.copies = max(1, math.ceil(2 * l2 / w.algorithmic_bytes))
+        X0 = torch.from_numpy(X_h).to(device)
+        Wq0, sw0 = i8.int8_quant_weight(torch.from_numpy(W_h).to(device))
+        del W_h
+        b0 = None if b_h is None else torch.from_numpy(b_h).to(device)
+        c = self.copies
+        self.Xs = [X0] + [X0.clone() for _ in range(c - 1)]
+        self.Wqs = [Wq0] + [Wq0.clone() for _ in range(c - 1)]
+        self.sws = [sw0] + [sw0.clone() for _ in range(c - 1)]
+        self.bs = [b0] + [None if b0 is None else b0.clone() for _ in range(c - 1)]
+        self.Ys = [torch.empty((w.M, w.N), dtype=torch.float16, device=device) for _ in range(c)]
+        self.wss = [i8.new_workspace(w.M, w.N, w.K, device) for _ in range(c)]
+        self.device = device
+        self.path = forward_path(w.M, w.N, w.K)
+
+    def step(self, i: int):
+        import int8_mixed_precision_absmax_b200 as i8
+        c = i % self.copies
+        i8.int8_linear_forward(self.Xs[c], self.Wqs[c], self.sws[c], self.bs[c],
+                               self.w.threshold, Y=self.Ys[c], workspace=self.wss[c])
+
+    def estimate_ms(self) -> float:
+        import torch
+        for i in range(max(self.copies, 3)):
+            self.step(i)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(self.copies, 8)
+        e0.record()
+        for i in range(n):
+            self.step(i)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    def make_runner(self, steps: int, use_graph: bool):
+        """run(n) launches n steps (n <= steps) from CUDA graphs of `copies` steps each."""
+        import torch
+        graphs = []
+        if use_graph:
+            try:
+                chunk = self.copies if steps >= self.copies else steps
+                sizes = [chunk] + ([steps % chunk] if steps % chunk else [])
+                side = torch.cuda.Stream(self.device)
+                side.wait_stream(torch.cuda.current_stream(self.device))
+                with torch.cuda.stream(side):
+                    for i in range(self.copies):
+                        self.step(i)
+                torch.cuda.current_stream(self.device).wait_stream(side)
+                torch.cuda.synchronize()
+                for n in sizes:
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        for i in range(n):
+                            self.step(i)
+                    graphs.append((g, n))
+            except Exception as exc:  # capture unsupported: launch directly
+                print(f"[bench] graph capture failed ({exc}); launching directly",
+                      file=sys.stderr)
+                graphs = []
+
+        def run(n):
+            if graphs:
+                g, chunk = graphs[0]
+                for _ in range(n // chunk):
+                    g.replay()
+                if n % chunk:
+                    graphs[1][0].replay()
+            else:
+                for i in range(n):
+                    self.step(i)
+        run.graphs = graphs
+        run.chunk = graphs[0][1] if graphs else 1
+        return run
+
+    def check_status(self):
+        import torch
+        import int8_mixed_precision_absmax_b200 as i8
+        for ws in self.wss:
+            st = i8.int8_read_device_status(ws[:4].view(torch.int32))
+            if st != 0:
+                raise SystemExit(f"device status {st}: {i8.int8_status_string(st)}")
+
+    def outlier_count(self) -> int:
+        import int8_mixed_precision_absmax_b200 as i8
+        return int(i8.int8_quantize_rows(self.Xs[0], self.w.threshold)[3].item())
+
+    def kernel_times(self):
+        """(activation-side ms, product ms) per step, each replayed alone from its own graph."""
+        import int8_mixed_precision_absmax_b200 as i8
+        c = self.copies
+        n = max(c, 32)
+        if self.path["quantize"]:
+            q_ms = graph_time_ms(lambda i: i8.int8_linear_quantize(
+                self.Xs[i % c], self.Wqs[i % c], self.sws[i % c], self.w.threshold,
+                self.wss[i % c]), n, self.device)
+        else:
+            q_ms = 0.0
+        g_ms = graph_time_ms(lambda i: i8.int8_linear_matmul(
+            self.Xs[i % c], self.Wqs[i % c], self.sws[i % c], self.bs[i % c], self.w.threshold,
+            self.Ys[i % c], self.wss[i % c]), n, self.device)
+        for i in range(c):  # leave every copy's Y from a complete forward
+            self.step(i)
+        return q_ms, g_ms
+
+    def e2e(self, world: int, budget_s: float):
+        """The same metric through the public call, with a pinned host->device copy of X and a
+        device->host copy of Y inside every step."""
+        import torch
+        w = self.w
+        Xh = torch.from_numpy(self.X_h).pin_memory()
+        Yh = torch.empty((w.M, w.N), dtype=torch.float16).pin_memory()
+        c = self.copies
+
+        def one(i):
+            self.Xs[i % c].copy_(Xh, non_blocking=True)
+            self.step(i)
+            Yh.copy_(self.Ys[i % c], non_blocking=True)
+        for i in range(3):
+            one(i)
+        torch.cuda.synchronize()
+        e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_a.record()
+        for i in range(3):
+            one(i)
+        e_b.record()
+        torch.cuda.synchronize()
+        est = e_a.elapsed_time(e_b) / 3
+        n_e = int(max(5, min(20000, budget_s * 1e3 / max(est, 1e-3))))
+        n_e = int(max_over_ranks(float(n_e), self.device))
+        barrier(self.device)
+        e_a.record()
+        for i in range(n_e):
+            one(i)
+        e_b.record()
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(e_a.elapsed_time(e_b) / 1e3, self.device)
+        return {"value": whole_job_rate(w.ops, n_e, world, e2e_s) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
+                "d2h_bytes_per_step": int(Yh.numel() * Yh.element_size()), "steps": n_e,
+                "ms_per_step": e2e_s / n_e * 1e3}
+
+    def roofline(self, n_out: int, q_ms: float, g_ms: float, step_ms: float, peaks):
+        """The product kernel against its roofline, and the whole step against the same."""
+        w = self.w
+        path = self.path
+        few_tokens = path["name"] != "tiled"
+        if few_tokens:
+            # weight streaming: X (fp16) and Wq in, Y out -- the whole step is one kernel pair
+            nbytes = w.algorithmic_bytes
+            achieved = nbytes / (g_ms / 1e3) / 1e9
+            peak = peaks["hbm_gbs"]
+            return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "frac_end_to_end": nbytes / (step_ms / 1e3) / 1e9 / peak,
+                    "kernel": path["kernel"], "kernel_ms": g_ms, "quantize_ms": q_ms,
+                    "algorithmic_bytes": nbytes,
+                    "peak_source": f"{peaks['source']} HBM copy (burst)"}
+        i8_ops, f16_flops = op_counts(w, n_out)
+        t_roof = tensor_roof_s(i8_ops, f16_flops, peaks)
+        work = i8_ops + f16_flops
+        peak = work / t_roof / 1e12  # the int8/fp16 mix at the two peaks
+        achieved = work / (g_ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "frac_end_to_end": t_roof / (step_ms / 1e3),
+                "kernel": path["kernel"], "kernel_ms": g_ms, "quantize_ms": q_ms,
+                "int8_ops": i8_ops, "fp16_flops": f16_flops,
+                "peak_source": (f"{peaks['source']}: int8 = bf16 burst x {INT8_OVER_BF16:g} "
+                                f"({peaks['int8_tops']:.0f} TOPS), fp16 = bf16 burst "
+                                f"({peaks['f16_tflops']:.0f} TFLOP/s); peak = the work's mix")}
+
+
+def measure(layer, world: int, steps: int, warm: int, use_graph: bool, peaks, sampler=None,
+            e2e_budget_s: float = 2.0):
+    """Time exactly `steps` steps (after `warm` untimed ones and graph warm-up), the kernels
+    apart, and the end-to-end variant; returns the numbers of one JSON entry."""
+    import torch
+    w = layer.w
+    for i in range(max(warm, 1)):
+        layer.step(i)
+    torch.cuda.synchronize()
+    run = layer.make_runner(steps, use_graph)
+    for _ in range(2):
+        run(min(steps, layer.copies))
+    torch.cuda.synchronize()
+    if sampler:
+        # keep the GPU busy while the sampler starts, so the clocks it sees are those under load
+        sampler.start()
+        lead = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        lead[0].record()
+        run(min(steps, layer.copies))
+        lead[1].record()
+        torch.cuda.synchronize()
+        per = lead[0].elapsed_time(lead[1]) / min(steps, layer.copies)
+        n_lead = int(max(1, min(1e6, 1000.0 / max(per, 1e-3))))  # about 1 s of steps
+        for _ in range(max(1, n_lead // run.chunk)):
+            run(run.chunk)
+    barrier(layer.device)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    run(steps)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(layer.device)
+    clocks = sampler.stop() if sampler else None
+    max_s = max_over_ranks(t0.elapsed_time(t1) / 1e3, layer.device)
+    layer.check_status()
+    run.graphs.clear()
+    q_ms, g_ms = layer.kernel_times()
+    n_out = layer.outlier_count()
+    step_ms = max_s / steps * 1e3
+    return {
+        "value": whole_job_rate(w.ops, steps, world, max_s) / 1e12,
+        "gbs": whole_job_rate(w.algorithmic_bytes, steps, world, max_s) / 1e9,
+        "ms_per_step": step_ms, "steps": steps, "outlier_cols": n_out,
+        "roofline": layer.roofline(n_out, q_ms, g_ms, step_ms, peaks),
+        "e2e": layer.e2e(world, e2e_budget_s),
+        "gpu_launches": layer.path["launches"] * steps,
+        "clocks": clocks,
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "threshold": w.threshold,
+                   "bias": layer.b_h is not None, "outlier_cols": n_out,
+                   "path": layer.path["name"],
+                   "l2": f"{layer.copies} rotating copies of X, Wq, w_scale, Y and workspace "
+                         f"({layer.copies * w.algorithmic_bytes / 2**20:.0f} MiB of operands, "
+                         f"> 2 x L2)" if layer.copies > 1 else
+                         f"operands ({w.algorithmic_bytes / 2**20:.0f} MiB) larger than 2 x L2"},
+    }
+
+
+# configurations reported beside the headline, each timed for at least this long
+PER_CONFIG = ("decode_q_proj", "prefill_up_proj", "down_proj_13b")
+PER_CONFIG_MIN_S = 1.0
+
+
 def run_ours(args):
-    import numpy as np
     import torch
 
     import int8_mixed_precision_absmax_b200 as i8
@@ -353,217 +636,76 @@ def run_ours(args):
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
     i8.load_library()
-
-    w = synth.WORKLOADS[args.workload]
-    X_h, W_h, b_h, _ = synth.make_inputs(w, seed=w.seed + rank)
     props = torch.cuda.get_device_properties(device)
     l2 = int(getattr(props, "L2_cache_size", 0) or 126 * 2**20)
-
-    # inputs resident in HBM; enough rotating copies that each step's operands left L2
-    step_bytes = w.algorithmic_bytes
-    copies = max(1, math.ceil(2 * l2 / step_bytes))
-    X0 = torch.from_numpy(X_h).to(device)
-    Wq0, sw0 = i8.int8_quant_weight(torch.from_numpy(W_h).to(device))
-    b0 = None if b_h is None else torch.from_numpy(b_h).to(device)
-    Xs = [X0] + [X0.clone() for _ in range(copies - 1)]
-    Wqs = [Wq0] + [Wq0.clone() for _ in range(copies - 1)]
-    sws = [sw0] + [sw0.clone() for _ in range(copies - 1)]
-    bs = [b0] + [None if b0 is None else b0.clone() for _ in range(copies - 1)]
-    Ys = [torch.empty((w.M, w.N), dtype=torch.float16, device=device) for _ in range(copies)]
-    wss = [i8.new_workspace(w.M, w.N, w.K, device) for _ in range(copies)]
-    del W_h
-
-    def step(i):
-        c = i % copies
-        i8.int8_linear_forward(Xs[c], Wqs[c], sws[c], bs[c], w.threshold, Y=Ys[c],
-                               workspace=wss[c])
-
-    warm = max(args.warmup, 0)
-    for i in range(max(warm, 1)):
-        step(i)
-    torch.cuda.synchronize()
-
-    # estimate the step time to size the default step count (about 2 s of device time)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    probe = max(copies, 8)
-    e0.record()
-    for i in range(probe):
-        step(i)
-    e1.record()
-    torch.cuda.synchronize()
-    est_ms = e0.elapsed_time(e1) / probe
-    steps = args.steps if args.steps is not None else max(20, int(2000.0 / max(est_ms, 1e-3)))
-    steps = int(max_over_ranks(float(steps), device))
-
-    # CUDA graphs: one replay = `copies` consecutive steps, plus one for the remainder
+    peaks = load_peaks()
+    peaks["int8_tops"] = peaks["bf16_tflops"] * INT8_OVER_BF16
+    peaks["f16_tflops"] = peaks["bf16_tflops"]
     use_graph = not args.no_graph
-    graphs = []
-    if use_graph:
-        try:
-            chunk = copies if steps >= copies else steps
-            sizes = [chunk] + ([steps % chunk] if steps % chunk else [])
-            side = torch.cuda.Stream(device)
-            side.wait_stream(torch.cuda.current_stream(device))
-            with torch.cuda.stream(side):
-                for i in range(copies):
-                    step(i)
-            torch.cuda.current_stream(device).wait_stream(side)
-            torch.cuda.synchronize()
-            for n in sizes:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    for i in range(n):
-                        step(i)
-                graphs.append((g, n))
-        except Exception as exc:  # capture unsupported: fall back to direct launches
-            print(f"[bench] graph capture failed ({exc}); launching directly", file=sys.stderr)
-            graphs, use_graph = [], False
-
-    def run_steps(n):
-        if use_graph:
-            g, chunk = graphs[0]
-            for _ in range(n // chunk):
-                g.replay()
-            r = n % chunk
-            if r:
-                graphs[1][0].replay()
-        else:
-            for i in range(n):
-                step(i)
-
-    for _ in range(2):  # graph warm-up (the untimed warm-up steps above ran direct launches)
-        run_steps(min(steps, copies))
-    torch.cuda.synchronize()
-
+    warm = max(args.warmup, 0)
     uuid = None
     try:
         uuid = "GPU-" + str(props.uuid)
     except Exception:
         uuid = None
+
+    # ---- the headline: exactly --steps steps (default: about 2 s of device time)
+    w = synth.WORKLOADS[args.workload]
+    layer = Layer(w, rank, device, l2)
+    est_ms = layer.estimate_ms()
+    steps = args.steps if args.steps is not None else max(20, int(2000.0 / max(est_ms, 1e-3)))
+    steps = int(max_over_ranks(float(steps), device))
     sampler = ClockSampler(uuid) if rank == 0 else None
-    if sampler:
-        sampler.start()
-    barrier(device)
-    torch.cuda.synchronize()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_start.record()
-    run_steps(steps)
-    t_end.record()
-    torch.cuda.synchronize()
-    barrier(device)
-    clocks = sampler.stop() if sampler else None
-    elapsed_s = t_start.elapsed_time(t_end) / 1e3
-    max_s = max_over_ranks(elapsed_s, device)
-
-    for ws in wss:
-        st = i8.int8_read_device_status(ws[:4].view(torch.int32))
-        if st != 0:
-            raise SystemExit(f"device status {st}: {i8.int8_status_string(st)}")
-
-    value = whole_job_rate(w.ops, steps, world, max_s) / 1e12
-    gbs = whole_job_rate(step_bytes, steps, world, max_s) / 1e9
-
-    # ---- per-kernel durations, live: the activation side and the product, each replayed
-    # back to back from its own CUDA graph over the rotating copies (CUDA events around the
-    # replays, on the launching stream); the product reads what earlier steps left in each
-    # copy's workspace
-    path = forward_path(w.M, w.N, w.K)
-    if path["quantize"]:
-        q_ms = graph_time_ms(lambda i: i8.int8_linear_quantize(
-            Xs[i % copies], Wqs[i % copies], sws[i % copies], w.threshold, wss[i % copies]),
-            max(copies, 32), device)
-    else:
-        q_ms = 0.0
-    g_ms = graph_time_ms(lambda i: i8.int8_linear_matmul(
-        Xs[i % copies], Wqs[i % copies], sws[i % copies], bs[i % copies], w.threshold,
-        Ys[i % copies], wss[i % copies]), max(copies, 32), device)
-    for c in range(copies):  # leave every copy's Y from a complete forward
-        step(c)
-    torch.cuda.synchronize()
-
-    peaks = load_peaks()
-    tensor_bound = w.ops / step_bytes > (peaks["bf16_tflops"] * INT8_OVER_BF16 * 1e12) / (peaks["hbm_gbs"] * 1e9)
-    # algorithmic bytes of the matmul kernel: its operands and output, each once
-    n_out = int(i8.int8_quantize_rows(Xs[0], w.threshold)[3].item())
-    pad = (n_out + 63) // 64 * 64 if n_out else 0
-    few_tokens = w.M <= 16
-    kernel = path["matmul"]
-    if few_tokens:  # reads X (fp16) and Wq, writes Y
-        gemm_bytes = (2 * w.M * w.K + w.N * w.K + 4 * w.N + 2 * w.M * w.N
-                      + (2 * w.N if b_h is not None else 0))
-    else:           # reads Xq, Wq and the fp16 outlier operands, writes Y
-        gemm_bytes = (w.M * w.K + w.N * w.K + 4 * (w.M + w.N) + 2 * w.M * w.N
-                      + 2 * pad * (w.M + w.N) + (2 * w.N if b_h is not None else 0))
-    if tensor_bound:
-        achieved = w.ops / (g_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops"] * INT8_OVER_BF16
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "kernel": kernel,
-                "kernel_ms": g_ms, "quantize_ms": q_ms,
-                "peak_source": f"{peaks['source']} bf16 x {INT8_OVER_BF16:g} (int8:bf16 nominal)"}
-    else:
-        achieved = gemm_bytes / (g_ms / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "kernel": kernel,
-                "kernel_ms": g_ms, "quantize_ms": q_ms, "algorithmic_bytes": gemm_bytes,
-                "peak_source": f"{peaks['source']} HBM copy"}
-    roof["traffic"] = recorded_traffic(w.name, kernel.split()[0])
-
-    # ---- end to end through the public API: pinned H2D of X, forward, D2H of Y
-    Xh = torch.from_numpy(X_h).pin_memory()
-    Yh = torch.empty((w.M, w.N), dtype=torch.float16).pin_memory()
-    n_e = max(10, min(steps, 2000))
-    for i in range(3):
-        Xs[0].copy_(Xh, non_blocking=True)
-        step(0)
-        Yh.copy_(Ys[0], non_blocking=True)
-    torch.cuda.synchronize()
-    barrier(device)
-    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_a.record()
-    for i in range(n_e):
-        c = i % copies
-        Xs[c].copy_(Xh, non_blocking=True)
-        step(c)
-        Yh.copy_(Ys[c], non_blocking=True)
-    e_b.record()
-    torch.cuda.synchronize()
-    e2e_s = max_over_ranks(e_a.elapsed_time(e_b) / 1e3, device)
-    e2e = {"value": whole_job_rate(w.ops, n_e, world, e2e_s) / 1e12, "unit": UNIT,
-           "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
-           "d2h_bytes_per_step": int(Yh.numel() * Yh.element_size()), "steps": n_e}
+    head = measure(layer, world, steps, warm, use_graph, peaks, sampler)
+    head["roofline"]["traffic"] = recorded_traffic(w.name, layer.path["kernel"])
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        Wq_h = Wqs[0].cpu().numpy()
-        sw_h = sws[0].cpu().numpy()
-        rate, t, desc, threads, _ = oracle_sample_rate(w, X_h, Wq_h, sw_h, b_h, args.cpu_budget_s)
+        Wq_h = layer.Wqs[0].cpu().numpy()
+        sw_h = layer.sws[0].cpu().numpy()
+        rate, t, desc, threads, _ = oracle_sample_rate(w, layer.X_h, Wq_h, sw_h, layer.b_h,
+                                                       args.cpu_budget_s)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": desc + f", {t:.1f} s"}
+               "host_cores": os.cpu_count(), "cpu_model": cpu_model(),
+               "sample": desc + f", {t:.1f} s; OpenMP over the sampled rows"}
+    del layer
+    torch.cuda.empty_cache()
+
+    # ---- the other configurations: each timed for at least PER_CONFIG_MIN_S
+    per_config = {}
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            if name == w.name:
+                continue
+            pw = synth.WORKLOADS[name]
+            pl = Layer(pw, rank, device, l2)
+            p_est = pl.estimate_ms()
+            p_steps = int(max_over_ranks(float(max(20, int(PER_CONFIG_MIN_S * 1e3 / max(p_est, 1e-3)))),
+                                         device))
+            r = measure(pl, world, p_steps, warm, use_graph, peaks, None, e2e_budget_s=1.0)
+            r["roofline"]["traffic"] = recorded_traffic(pw.name, pl.path["kernel"])
+            r.pop("clocks", None)
+            per_config[name] = r
+            del pl
+            torch.cuda.empty_cache()
 
     if rank == 0:
+        cfg = dict(head["config"])
+        cfg["launch"] = "CUDA graph replay" if use_graph else "direct launches"
+        cfg["parallelism"] = f"{world} independent replica(s), one per GPU"
+        cfg["clocks_window"] = ("nvidia-smi every 200 ms over about 1 s of the same steps run "
+                                "back to back just before the timed ones, and over the timed ones")
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
-            "warmup": warm, "ms_per_step": max_s / steps * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "gbs": gbs,
-            "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N,
-                       "threshold": w.threshold, "bias": b_h is not None,
-                       "outlier_cols": n_out,
-                       "l2": f"{copies} rotating copies of X, Wq, w_scale, Y and workspace "
-                             f"({copies * step_bytes / 2**20:.0f} MiB of operands > 2 x L2)",
-                       "launch": "CUDA graph replay" if use_graph else "direct launches",
-                       "path": path["name"],
-                       "parallelism": f"{world} independent replica(s), one per GPU"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": path["launches"] * steps,
-            "clocks": clocks,
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic", "gbs": head["gbs"], "config": cfg,
+            "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+            "per_config": per_config,
         }
         print(json.dumps(line), flush=True)
 
-    graphs.clear()
     import torch.distributed as dist
     if dist.is_initialized():
         dist.destroy_process_group()

@@ -20,6 +20,13 @@
  *     Kernel-side failures (a bounded wait that gave up) are written as a negative code
  *     to a device status word and read with int8_read_device_status().
  *   - Results are deterministic: the same inputs give the same bits on every call.
+ *   - The forward's kernels are launched with programmatic dependent launch: a kernel may
+ *     start while the kernel before it on the stream is finishing, and it waits for that
+ *     kernel before it reads X (or any activation data) and before it writes anything.  One
+ *     read comes before that wait: with M <= 8 (the one-launch decode route) each CTA starts
+ *     copying its rows of Wq at once.  So Wq must not be written by the kernel launched just
+ *     before the forward on the same stream.  Weights made by int8_quant_weight on the same
+ *     stream are safe to use at once: its kernel never lets the next launch start early.
  */
 #ifndef INT8MM_H
 #define INT8MM_H
@@ -152,6 +159,23 @@ int int8_activation_stats(const void *X, int M, int K, float *col_absmax, double
                           void *workspace, size_t ws_bytes, int8mm_stream_t stream);
 
 /*
+ * The outlier test of [P2] section 2.3 applied to column maxima gathered elsewhere, for a
+ * layer whose tokens are split across GPUs: every rank takes the column absmax of its own rows
+ * (int8_activation_stats), a MAX all-reduce makes them the maxima over all rows, and this call
+ * turns them into one extra activation row,
+ *   row[j] = binary16(col_absmax[j])  if col_absmax[j] > threshold,  0 otherwise,
+ * which the rank appends to its rows before int8_linear_forward.  That row exceeds the
+ * threshold in exactly the global outlier columns (the maxima are binary16 magnitudes, so the
+ * conversion is exact) and no real row's scale or codes change; its output row is dropped.
+ *   col_absmax [in]  float32 [K]
+ *   threshold  [in]  as for int8_linear_forward (negative acts as 0, +inf marks nothing,
+ *                    NaN is rejected)
+ *   row        [out] binary16 [K]
+ */
+int int8_outlier_row(const float *col_absmax, int K, float threshold, void *row,
+                     int8mm_stream_t stream);
+
+/*
  * The two halves of int8_linear_forward, for callers that time or schedule them apart:
  * int8_linear_forward is exactly int8_linear_quantize followed by int8_linear_matmul with
  * the same arguments, workspace and stream.  Arguments are as for int8_linear_forward.
@@ -221,6 +245,35 @@ int int8_gemm_i32(const int8_t *Xq, const int8_t *Wq, int M, int N, int K, int32
 int int8_outlier_weights(const int8_t *Wq, const float *w_scale, int N, int K,
                          const int32_t *outlier_cols, const int32_t *n_outliers, void *W_hat,
                          int8mm_stream_t stream);
+
+/*
+ * Diagnostic: int8_linear_forward_ex that also hands back what the forward's own kernels
+ * computed on the way to Y, so that every intermediate of the method can be compared with
+ * its definition: the outlier columns ([P2] section 2.3), the per-row (or per-tensor)
+ * activation scales and codes ([P5] section "LLM.int8() 是怎么做到几乎无损的", item 2) and
+ * the fp16 weights the outlier term multiplied ([P5] section "如何在 PyTorch 2.9 中启用
+ * LLM.int8 推理", has_fp16_weights).  The values come from the kernels that produce Y for
+ * this shape (the one-launch decode kernel, the few-token pair, the cluster kernel or the
+ * tiled passes), not from a separate computation.  Every output pointer may be NULL.
+ *   Xq           [out] int8 [M, K]: the codes, 0 in outlier columns
+ *   row_scale    [out] float32 [M]: the activation scale of each row
+ *   outlier_cols [out] int32 [K]: the outlier columns in ascending order, first *n_outliers
+ *                      entries valid
+ *   n_outliers   [out] int32 [1]
+ *   W_hat        [out] binary16 [N, K]: at every outlier column j, W_hat[n, j] is the weight
+ *                      the outlier term used (fp16(Wq[n,j] * w_scale[n]), or W16[n,j] when
+ *                      W16 is given); entries of the other columns are left untouched
+ * Every other argument, the workspace and the error codes are as for int8_linear_forward_ex;
+ * Y and acc get the same bits as from int8_linear_forward_ex.  Output pointers must be
+ * 16-byte aligned.  The extra writes make this call slower than the forward: it is meant for
+ * tests and debugging, not for the hot path.
+ */
+int int8_linear_forward_trace(const void *X, int M, int K, const int8_t *Wq,
+                              const float *w_scale, const void *W16, const void *bias, int N,
+                              float threshold, unsigned flags, void *Y, int32_t *acc, int8_t *Xq,
+                              float *row_scale, int32_t *outlier_cols, int32_t *n_outliers,
+                              void *W_hat, void *workspace, size_t ws_bytes,
+                              int8mm_stream_t stream);
 
 /*
  * int8_linear_forward without a workspace argument, for few-token (decode) shapes.

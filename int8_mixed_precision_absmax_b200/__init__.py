@@ -28,7 +28,8 @@ __all__ = [
     "int8_quantize_rows", "int8_gemm_i32", "int8_outlier_weights",
     "int8_read_device_status", "int8_status_string", "int8_linear_forward_noalloc",
     "int8_linear_forward_fp16w", "int8_linear_forward_ex", "PER_TENSOR_SCALE",
-    "int8_activation_stats", "Int8Linear", "DEFAULT_THRESHOLD",
+    "int8_activation_stats", "Int8Linear", "DEFAULT_THRESHOLD", "int8_linear_forward_trace",
+    "int8_outlier_row",
 ]
 
 DEFAULT_THRESHOLD = 6.0
@@ -77,14 +78,18 @@ def load_library():
         lib.int8_linear_forward_fp16w.argtypes = [p, i, i, p, p, p, p, i, f, p, p, sz, p]
         lib.int8_linear_forward_ex.argtypes = [p, i, i, p, p, p, p, i, f, ctypes.c_uint, p, p,
                                                p, sz, p]
+        lib.int8_linear_forward_trace.argtypes = [p, i, i, p, p, p, p, i, f, ctypes.c_uint, p,
+                                                  p, p, p, p, p, p, p, sz, p]
         lib.int8_activation_stats_workspace_size.argtypes = []
         lib.int8_activation_stats_workspace_size.restype = sz
         lib.int8_activation_stats.argtypes = [p, i, i, p, p, p, sz, p]
+        lib.int8_outlier_row.argtypes = [p, i, f, p, p]
         for name in ("int8_quant_weight", "int8_linear_forward", "int8_linear_quantize",
                      "int8_linear_matmul", "int8_linear_forward_acc", "int8_quantize_rows",
                      "int8_gemm_i32", "int8_outlier_weights", "int8_read_device_status",
                      "int8_linear_forward_noalloc", "int8_linear_forward_fp16w",
-                     "int8_linear_forward_ex", "int8_activation_stats"):
+                     "int8_linear_forward_ex", "int8_activation_stats",
+                     "int8_linear_forward_trace", "int8_outlier_row"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -241,6 +246,46 @@ def int8_linear_forward_ex(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Ten
     return Y
 
 
+def int8_linear_forward_trace(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                              bias: torch.Tensor | None, threshold: float = DEFAULT_THRESHOLD,
+                              W16: torch.Tensor | None = None, per_tensor: bool = False,
+                              workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """One forward that also returns what its own kernels computed on the way: a dict of
+    device tensors Y [M,N] fp16, acc [M,N] int32, Xq [M,K] int8, row_scale [M] f32,
+    outlier_cols [K] i32 (first n_outliers valid), n_outliers [1] i32 and W_hat [N,K] fp16
+    (valid at the outlier columns; zero elsewhere)."""
+    _need(X, torch.float16, "X", 2)
+    _need(Wq, torch.int8, "Wq", 2)
+    _need(w_scale, torch.float32, "w_scale", 1)
+    M, K = X.shape
+    N = Wq.shape[0]
+    dev = X.device
+    if W16 is not None:
+        _need(W16, torch.float16, "W16", 2)
+        if tuple(W16.shape) != (N, K):
+            raise ValueError(f"W16 must be [{N}, {K}], got {tuple(W16.shape)}")
+    if bias is not None:
+        _need(bias, torch.float16, "bias", 1)
+    out = {"Y": torch.empty((M, N), dtype=torch.float16, device=dev),
+           "acc": torch.empty((M, N), dtype=torch.int32, device=dev),
+           "Xq": torch.empty((M, K), dtype=torch.int8, device=dev),
+           "row_scale": torch.empty(M, dtype=torch.float32, device=dev),
+           "outlier_cols": torch.empty(K, dtype=torch.int32, device=dev),
+           "n_outliers": torch.zeros(1, dtype=torch.int32, device=dev),
+           "W_hat": torch.zeros((N, K), dtype=torch.float16, device=dev)}
+    if workspace is None:
+        workspace = new_workspace(M, N, K, dev)
+    _need(workspace, torch.uint8, "workspace", 1)
+    flags = PER_TENSOR_SCALE if per_tensor else 0
+    _check(load_library().int8_linear_forward_trace(
+        _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(W16), _ptr(bias), N, float(threshold),
+        flags, _ptr(out["Y"]), _ptr(out["acc"]), _ptr(out["Xq"]), _ptr(out["row_scale"]),
+        _ptr(out["outlier_cols"]), _ptr(out["n_outliers"]), _ptr(out["W_hat"]),
+        _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream, dev))),
+        "int8_linear_forward_trace")
+    return out
+
+
 def int8_activation_stats(X: torch.Tensor, stream=None):
     """Statistics of |X| for choosing the threshold: (max, q99, max / (q99 + 1e-6)) as a
     float64 tensor of 3 on the device, and the column absmax [K] (float32)."""
@@ -254,6 +299,21 @@ def int8_activation_stats(X: torch.Tensor, stream=None):
         _ptr(X), M, K, _ptr(col), _ptr(out), _ptr(ws), ws.numel(),
         ctypes.c_void_p(_stream(stream, X.device))), "int8_activation_stats")
     return out, col
+
+
+def int8_outlier_row(col_absmax: torch.Tensor, threshold: float, row: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """fp16 [K]: col_absmax[j] where it exceeds the threshold, 0 elsewhere (the extra row the
+    token split appends so that every rank finds the global outlier columns)."""
+    _need(col_absmax, torch.float32, "col_absmax", 1)
+    K = col_absmax.shape[0]
+    if row is None:
+        row = torch.empty(K, dtype=torch.float16, device=col_absmax.device)
+    _need(row, torch.float16, "row", 1)
+    _check(load_library().int8_outlier_row(_ptr(col_absmax), K, float(threshold), _ptr(row),
+                                           ctypes.c_void_p(_stream(stream, col_absmax.device))),
+           "int8_outlier_row")
+    return row
 
 
 def int8_linear_forward_noalloc(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,

@@ -111,7 +111,19 @@ namespace {
 struct LayerOpts {
   const void* W16 = nullptr;
   int per_tensor = 0;
+  TraceSink trace;  // diagnostic outputs written by the kernels themselves (all null normally)
 };
+
+// Which kernels a forward of this shape runs (the dispatch of run_quantize / run_matmul).
+enum class Route { kDecode, kGemv, kSmall, kTiled };
+Route route_of(int M, int N, int K) {
+  if (M <= kSmallMP) {
+    if (plan_decode(M, N, K).fits) return Route::kDecode;
+    if (plan_gemv(M, N, K, device_sm_count()).fits) return Route::kGemv;
+    if (small_path_fits(M, K)) return Route::kSmall;
+  }
+  return Route::kTiled;
+}
 
 struct ForwardPlan {
   WorkspaceLayout L;
@@ -167,6 +179,7 @@ GemvArgs gemv_args(const void* X, int M, int K, const int8_t* Wq, const float* w
   g.sx = at<float>(workspace, p.L.few_sx);
   g.cols = at<int32_t>(workspace, p.L.cols);
   g.n_out = p.header + 1;
+  g.trace = o.trace;
   g.status = p.header;
   return g;
 }
@@ -190,6 +203,7 @@ SmallArgs small_args(const void* X, int M, int K, const int8_t* Wq, const float*
   a.acc = acc;
   a.splits = sp.splits;
   a.stages = sp.stages;
+  a.trace = o.trace;
   a.status = p.header;
   return a;
 }
@@ -220,6 +234,7 @@ int run_decode(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   a.Y = static_cast<__half*>(Y);
   a.acc = acc;
   a.per_tensor = o.per_tensor;
+  a.trace = o.trace;
   a.status = status;
   return launch_status(launch_decode(map, a, dp, stream, pdl));
 }
@@ -376,6 +391,19 @@ int int8_activation_stats(const void* X, int M, int K, float* col_absmax, double
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int int8_outlier_row(const float* col_absmax, int K, float threshold, void* row,
+                     int8mm_stream_t stream) {
+  if (!col_absmax || !row) return INT8MM_ERR_NULL;
+  int rc = check_shape(1, 1, K);
+  if (rc) return rc;
+  if (!aligned16(col_absmax) || !aligned16(row)) return INT8MM_ERR_ALIGN;
+  if (std::isnan(threshold)) return INT8MM_ERR_THRESHOLD;
+  if ((rc = check_device())) return rc;
+  return launch_status(launch_outlier_row(col_absmax, K, effective_threshold(threshold),
+                                          static_cast<__half*>(row),
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int int8_linear_forward_ex(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
                            const void* W16, const void* bias, int N, float threshold,
                            unsigned flags, void* Y, int32_t* acc, void* workspace,
@@ -492,6 +520,67 @@ int int8_outlier_weights(const int8_t* Wq, const float* w_scale, int N, int K,
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int int8_linear_forward_trace(const void* X, int M, int K, const int8_t* Wq,
+                              const float* w_scale, const void* W16, const void* bias, int N,
+                              float threshold, unsigned flags, void* Y, int32_t* acc, int8_t* Xq,
+                              float* row_scale, int32_t* outlier_cols, int32_t* n_outliers,
+                              void* W_hat, void* workspace, size_t ws_bytes,
+                              int8mm_stream_t stream_) {
+  if (flags & ~static_cast<unsigned>(INT8MM_PER_TENSOR_SCALE)) return INT8MM_ERR_FLAGS;
+  if ((Xq && !aligned16(Xq)) || (row_scale && !aligned16(row_scale)) ||
+      (outlier_cols && !aligned16(outlier_cols)) || (n_outliers && !aligned16(n_outliers)) ||
+      (W_hat && !aligned16(W_hat)))
+    return INT8MM_ERR_ALIGN;
+  int rc = check_shape(M, N, K);
+  if (rc) return rc;
+  if (!workspace || !aligned256(workspace) || ws_bytes < workspace_layout(M, N, K).total)
+    return INT8MM_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const WorkspaceLayout L = workspace_layout(M, N, K);
+  uint32_t* mask = at<uint32_t>(workspace, L.mask);
+  const Route route = route_of(M, N, K);
+  LayerOpts o;
+  o.W16 = W16;
+  o.per_tensor = (flags & INT8MM_PER_TENSOR_SCALE) ? 1 : 0;
+  if (route == Route::kDecode || route == Route::kSmall) {
+    // these kernels keep codes, scales and outlier bits on chip: they write them out here
+    o.trace.xq = Xq;
+    o.trace.sx = row_scale;
+    o.trace.flags = reinterpret_cast<uint8_t*>(mask);
+  }
+  if (route != Route::kTiled) o.trace.what = static_cast<__half*>(W_hat);
+  if ((rc = forward_impl(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace, ws_bytes,
+                         stream, o)))
+    return rc;
+  int32_t* header = at<int32_t>(workspace, L.header);
+  if (route == Route::kDecode || route == Route::kSmall) {
+    if (outlier_cols || n_outliers)
+      return launch_status(launch_trace_cols(mask, K, outlier_cols, n_outliers, stream));
+    return INT8MM_OK;
+  }
+  // the other kernels left codes, scales and the outlier list in the workspace
+  const bool few = route == Route::kGemv;
+  const int8_t* src_xq = at<int8_t>(workspace, few ? L.few_xq : L.xq);
+  const size_t src_ld = few ? static_cast<size_t>((K + 255) / 256) * 256 : static_cast<size_t>(K);
+  cudaError_t e = cudaSuccess;
+  if (Xq)
+    e = cudaMemcpy2DAsync(Xq, K, src_xq, src_ld, K, M, cudaMemcpyDeviceToDevice, stream);
+  if (e == cudaSuccess && row_scale)
+    e = cudaMemcpyAsync(row_scale, at<float>(workspace, few ? L.few_sx : L.xscale),
+                        static_cast<size_t>(M) * sizeof(float), cudaMemcpyDeviceToDevice, stream);
+  if (e == cudaSuccess && outlier_cols)
+    e = cudaMemcpyAsync(outlier_cols, at<int32_t>(workspace, L.cols),
+                        static_cast<size_t>(K) * sizeof(int32_t), cudaMemcpyDeviceToDevice, stream);
+  if (e == cudaSuccess && n_outliers)
+    e = cudaMemcpyAsync(n_outliers, header + 1, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                        stream);
+  if (e == cudaSuccess && W_hat && !few)
+    e = launch_trace_what(at<__half>(workspace, L.wo), L.ldo, at<int32_t>(workspace, L.cols),
+                          header + 1, N, K, static_cast<__half*>(W_hat), stream);
+  return launch_status(e);
+}
+
 int int8_read_device_status(const int32_t* dev_status, int8mm_stream_t stream) {
   if (!dev_status) return INT8MM_ERR_NULL;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -585,14 +674,13 @@ int int8_linear_forward_noalloc(const void* X, int M, int K, const int8_t* Wq,
   const bool small = !gp.fits && small_path_fits(M, K);
   if (!gp.fits && !small) return INT8MM_ERR_SCRATCH;
   const WorkspaceLayout L = noalloc_layout(K);
-  if (L.total > INT8MM_NOALLOC_SCRATCH_BYTES) return INT8MM_ERR_SCRATCH;
   ForwardPlan p = {};
   p.L = L;
   p.header = at<int32_t>(scratch, L.header);
   // Nothing in the scratch has to start at zero: the quantization kernel writes the outlier
   // count, list and activations before the product kernel reads them, and the status goes to
   // the caller's word (or nowhere).
-  if (small) {
+  if (small) {  // the cluster kernel keeps everything on chip: no scratch, no size limit
     const SmallPlan sp = plan_small(M, N, K);
     SmallArgs a = small_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, p, sp);
     a.status = dev_status;
@@ -601,6 +689,7 @@ int int8_linear_forward_noalloc(const void* X, int M, int K, const int8_t* Wq,
       return INT8MM_ERR_CUDA;
     return launch_status(launch_small(map, a, sp, stream, true));
   }
+  if (L.total > INT8MM_NOALLOC_SCRATCH_BYTES) return INT8MM_ERR_SCRATCH;
   GemvArgs g = gemv_args(X, M, K, Wq, w_scale, bias, N, threshold, Y, nullptr, scratch, p, gp);
   g.status = dev_status;
   CUtensorMap map;

@@ -36,8 +36,8 @@
 // codes (the MMA's k positions are permuted the same way in both operands, which leaves the
 // dot product as it is); a fragment is one 8-byte shared-memory load.
 //
-// The weights and scales are read before the wait on the previous launch: they must not be
-// written by the launch just before this one on the stream while it can still be running.
+// Wq is read before the wait on the previous launch (everything else after it): it must not
+// be written by the launch just before this one on the stream while that can still be running.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -183,8 +183,10 @@ size_t decode_smem_bytes(int T, int K) {
   return 1024 + static_cast<size_t>(weight_area(T, K)) + static_cast<size_t>(kDTok) * (K + 16);
 }
 
-// T 16-channel tiles per CTA; each thread holds up to kItems 8-column chunks of X
-template <int T, int kItems>
+// T 16-channel tiles per CTA; each thread holds up to kItems 8-column chunks of X.  kTrace:
+// also write what the layer computed on the way (a.trace): CTA 0 the codes, the row scales
+// and the outlier bits, every CTA its channels' fp16 weights at the outlier columns.
+template <int T, int kItems, bool kTrace>
 __global__ void __launch_bounds__(kDThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap map_wq, const DecodeArgs a) {
   constexpr int kC = 16 * T;  // channels per CTA
@@ -222,6 +224,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
       tma_load_3d(&map_wq, wt + static_cast<size_t>(t) * tb, &sh.full[t], 0, n0 + 16 * t, 0);
     }
   }
+  grid_launch_dependents();
+  grid_dependency_wait();  // X (the previous layer's output) is complete from here on
   float swr[T][2];  // scales of the fragment rows g, g + 8 of each tile
 #pragma unroll
   for (int t = 0; t < T; ++t)
@@ -235,8 +239,6 @@ __global__ void __launch_bounds__(kDThreads, 1)
   const bool e_live = tid < kDTok * kC && ei < M && n0 + ec < N;
   const float e_sw = e_live ? a.w_scale[n0 + ec] : 0.0f;
   const float e_bias = (e_live && a.bias) ? __half2float(a.bias[n0 + ec]) : 0.0f;
-  grid_launch_dependents();
-  grid_dependency_wait();  // X (the previous layer's output) is complete from here on
 
   // ---- X: thread tid holds chunks c = tid + 512 u (8 columns x 8 tokens each) in registers
   const int chunks = K / 8;
@@ -277,6 +279,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
       }
       xkeep[it] = keep_masks(bits);
       sh.flags[c] = static_cast<uint8_t>(bits);
+      if (kTrace && blockIdx.x == 0 && a.trace.flags) a.trace.flags[c] = static_cast<uint8_t>(bits);
       if (bits != 0u) {  // keep the chunk's fp16 values for the outlier term
         const int slot = atomicAdd(&sh.n_ochunks, 1);
         sh.oslot[c] = static_cast<uint8_t>(slot < kDOutChunks ? slot : 0xFF);
@@ -337,6 +340,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
     sx_l = __fdiv_rn(mf, 127.0f);
     rcp_l = mf > 0.0f ? __frcp_rn(sx_l) : 0.0f;
     if (warp == 0) sh.sx[lane] = sx_l;
+    if (kTrace && warp == 0 && blockIdx.x == 0 && lane < M && a.trace.sx) a.trace.sx[lane] = sx_l;
   }
 
   // this warp's k-blocks and the k-steps among them holding an outlier column (bit
@@ -369,9 +373,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
       const int c = tid + it * kDThreads;
       if (c < chunks) {
 #pragma unroll
-        for (int i = 0; i < kDTok; ++i)
-          *reinterpret_cast<uint2*>(xq_s + i * xq_ld + c * 8) =
-              quantize8(xv[it][i], sxv[i], rcpv[i], xkeep[it]);
+        for (int i = 0; i < kDTok; ++i) {
+          const uint2 q = quantize8(xv[it][i], sxv[i], rcpv[i], xkeep[it]);
+          *reinterpret_cast<uint2*>(xq_s + i * xq_ld + c * 8) = q;
+          if (kTrace && blockIdx.x == 0 && i < M && a.trace.xq)
+            *reinterpret_cast<uint2*>(a.trace.xq + static_cast<size_t>(i) * K + 8 * c) = q;
+        }
       }
     }
   }
@@ -449,6 +456,19 @@ __global__ void __launch_bounds__(kDThreads, 1)
             ha[h][1] = what2(w.x, 1, swr[t][h]);
             ha[h][2] = what2(w.y, 0, swr[t][h]);
             ha[h][3] = what2(w.y, 1, swr[t][h]);
+          }
+        }
+        if (kTrace && a.trace.what && fb != 0u) {  // rows g, g + 8, the chunk's outlier columns
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int n = n0 + 16 * t + 8 * h + g;
+            if (n >= N) continue;
+            unsigned short* dst =
+                reinterpret_cast<unsigned short*>(a.trace.what) + static_cast<size_t>(n) * K + 8 * ch;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if ((fb >> e) & 1u)
+                dst[e] = static_cast<unsigned short>(ha[h][e / 2] >> (16 * (e & 1)));
           }
         }
         mma_f16_16816(pf[t], ha[0][0], ha[1][0], ha[0][1], ha[1][1], b0, b1);
@@ -532,8 +552,10 @@ cudaError_t launch_decode(const CUtensorMap& map_wq, const DecodeArgs& a, const 
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev != configured_device) {  // all the shared memory a CTA may have beside the static
-    for (const void* k : {reinterpret_cast<const void*>(decode_kernel<2, 1>),
-                          reinterpret_cast<const void*>(decode_kernel<1, 2>)}) {
+    for (const void* k : {reinterpret_cast<const void*>(decode_kernel<2, 1, false>),
+                          reinterpret_cast<const void*>(decode_kernel<1, 2, false>),
+                          reinterpret_cast<const void*>(decode_kernel<2, 1, true>),
+                          reinterpret_cast<const void*>(decode_kernel<1, 2, true>)}) {
       cudaFuncAttributes fa;
       e = cudaFuncGetAttributes(&fa, k);
       if (e == cudaSuccess)
@@ -554,8 +576,12 @@ cudaError_t launch_decode(const CUtensorMap& map_wq, const DecodeArgs& a, const 
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   // K <= 4096: two tiles, one chunk of X per thread; up to 8192: one tile, two chunks
-  return p.tiles == 2 ? cudaLaunchKernelEx(&cfg, decode_kernel<2, 1>, map_wq, a)
-                      : cudaLaunchKernelEx(&cfg, decode_kernel<1, 2>, map_wq, a);
+  const bool trace = a.trace.xq || a.trace.sx || a.trace.flags || a.trace.what;
+  if (trace)
+    return p.tiles == 2 ? cudaLaunchKernelEx(&cfg, decode_kernel<2, 1, true>, map_wq, a)
+                        : cudaLaunchKernelEx(&cfg, decode_kernel<1, 2, true>, map_wq, a);
+  return p.tiles == 2 ? cudaLaunchKernelEx(&cfg, decode_kernel<2, 1, false>, map_wq, a)
+                      : cudaLaunchKernelEx(&cfg, decode_kernel<1, 2, false>, map_wq, a);
 }
 
 }  // namespace i8mm

@@ -512,6 +512,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         wv = __half2float(__float2half_rn(static_cast<float>(q) * swn));
       }
+      if (i == 0 && a.trace.what) a.trace.what[static_cast<size_t>(n) * a.K + j] = __float2half_rn(wv);
       P += wv * __half2float(o < staged ? sh.xo[o][i] : a.xo[static_cast<size_t>(o) * kSmallMP + i]);
     }
     const float bb = sh.bias[c];

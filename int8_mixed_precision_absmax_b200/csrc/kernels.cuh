@@ -99,6 +99,28 @@ struct RowQuantArgs {
 };
 cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl);
 
+// What a forward's own kernels computed on the way to Y, for the diagnostic
+// int8_linear_forward_trace (every pointer nullable; all null on the normal path):
+//   xq     int8 [M, K]  the activation codes (0 in outlier columns)
+//   sx     f32 [M]      the row scales
+//   flags  u8 [K / 8]   outlier bits, one byte per 8 columns (byte c bit e: column 8 c + e),
+//                       the same bytes as the little-endian words of the workspace mask
+//   what   half [N, K]  at each outlier column j, the fp16 weight the outlier term used
+struct TraceSink {
+  int8_t* xq = nullptr;
+  float* sx = nullptr;
+  uint8_t* flags = nullptr;
+  __half* what = nullptr;
+};
+
+// trace.cu: the outlier list from outlier bits (bits of columns >= K ignored; cols and n_out
+// nullable), and the tiled path's compacted outlier weights scattered to their columns.
+cudaError_t launch_trace_cols(const uint32_t* mask, int K, int32_t* cols, int32_t* n_out,
+                              cudaStream_t stream);
+cudaError_t launch_trace_what(const __half* wo, int ldo, const int32_t* cols,
+                              const int32_t* n_out, int N, int K, __half* W_hat,
+                              cudaStream_t stream);
+
 struct SmallArgs {
   const __half* X;
   int M, K, N;
@@ -112,6 +134,7 @@ struct SmallArgs {
   int splits;            // CTAs per cluster, each owning a K-slice
   int stages;            // depth of the Wq ring
   int per_tensor;        // one activation scale for all rows (the largest row absmax)
+  TraceSink trace;       // diagnostic outputs (int8_linear_forward_trace)
   int32_t* status;
 };
 struct SmallPlan {
@@ -142,6 +165,7 @@ struct GemvArgs {
   int32_t* cols;         // [K] outlier columns, ascending
   int32_t* n_out;        // outlier count
   int per_tensor;        // one activation scale for all rows (the largest row absmax)
+  TraceSink trace;       // diagnostic outputs (int8_linear_forward_trace)
   int32_t* status;
 };
 struct GemvPlan {
@@ -157,6 +181,9 @@ int device_sm_count();
 // Statistics of |X| (stats.cu): column absmax (nullable), and out[3] = {max, q99, ratio}
 // (device doubles); workspace of stats_workspace_bytes() (the |x| histogram).
 size_t stats_workspace_bytes();
+// row[j] = fp16(col_absmax[j]) where it exceeds the threshold (already clamped to >= 0), else 0
+cudaError_t launch_outlier_row(const float* col_absmax, int K, float threshold, __half* row,
+                               cudaStream_t stream);
 cudaError_t launch_activation_stats(const __half* X, int M, int K, float* col_absmax,
                                     double* out, void* workspace, int num_sms,
                                     cudaStream_t stream);
@@ -173,6 +200,7 @@ struct DecodeArgs {
   __half* Y;
   int32_t* acc;          // nullable: also write the int32 accumulators
   int per_tensor;        // one activation scale for all rows (the largest row absmax)
+  TraceSink trace;       // diagnostic outputs (int8_linear_forward_trace)
   int32_t* status;
 };
 struct DecodePlan {

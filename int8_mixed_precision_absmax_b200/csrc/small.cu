@@ -282,6 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (__high2float(cm[e]) > a.threshold) bits |= 1u << (2 * e + 1);
       }
       sh.flags[c] = static_cast<uint8_t>(bits);
+      if (a.trace.flags && tile == 0 && kb_begin * 16 + c < 4 * ((a.K + 31) / 32))
+        a.trace.flags[kb_begin * 16 + c] = static_cast<uint8_t>(bits);
 #pragma unroll
       for (int i = 0; i < kSmallMP; ++i) {
         const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
@@ -357,6 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             w0 = g0 < a.N ? __half2float(a.W16[static_cast<size_t>(g0) * a.K + j]) : 0.0f;
             w1 = g1 < a.N ? __half2float(a.W16[static_cast<size_t>(g1) * a.K + j]) : 0.0f;
           }
+          if (a.trace.what) {  // the weights this term multiplies, as fp16
+            if (g0 < a.N) a.trace.what[static_cast<size_t>(g0) * a.K + j] = __float2half_rn(w0);
+            if (g1 < a.N) a.trace.what[static_cast<size_t>(g1) * a.K + j] = __float2half_rn(w1);
+          }
           const __half* xc = x_slice + (j - col_begin);
 #pragma unroll
           for (int i = 0; i < kSmallMP; ++i)
@@ -394,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sh.sx[tz] = (tz < a.M) ? sc : 0.0f;
         sh.rcp[tz] = (tz < a.M && m > 0.0f) ? __frcp_rn(sc) : 0.0f;
         sh.zero_row[tz] = (tz >= a.M) || m == 0.0f;
+        if (a.trace.sx && tile == 0 && split == 0 && tz < a.M) a.trace.sx[tz] = sc;
       }
       named_barrier(2, kQuantThreads);
       // thread tz quantizes chunk c (8 columns) for all 16 rows, independently per row;
@@ -438,6 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           *reinterpret_cast<uint2*>(tile + (i / 8) * 1024 + (i % 8) * 128 +
                                     (((kk / 16) ^ (i % 8)) * 16)) = q;
+          const int kg = col_begin + c * 8;  // the chunk's first column in X
+          if (a.trace.xq && blockIdx.x < static_cast<unsigned>(S) && i < a.M && kg < a.K)
+            *reinterpret_cast<uint2*>(a.trace.xq + static_cast<size_t>(i) * a.K + kg) = q;
         }
       }
       fence_async_shared();

@@ -160,4 +160,24 @@ cudaError_t launch_activation_stats(const __half* X, int M, int K, float* col_ab
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ the token split's row
+
+// row[j] = binary16(col_absmax[j]) where col_absmax[j] > threshold, else 0: one row that
+// exceeds the threshold in exactly the columns whose maximum over all rows does (the outlier
+// test of [P2] section 2.3, in float32 as in every kernel of the layer).
+__global__ void outlier_row_kernel(const float* __restrict__ col_absmax, int K, float threshold,
+                                   __half* __restrict__ row) {
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < K; j += gridDim.x * blockDim.x) {
+    const float c = col_absmax[j];
+    row[j] = c > threshold ? __float2half_rn(c) : __float2half_rn(0.0f);
+  }
+}
+
+cudaError_t launch_outlier_row(const float* col_absmax, int K, float threshold, __half* row,
+                               cudaStream_t stream) {
+  const int blocks = (K + 255) / 256;
+  outlier_row_kernel<<<blocks, 256, 0, stream>>>(col_absmax, K, threshold, row);
+  return cudaGetLastError();
+}
+
 }  // namespace i8mm

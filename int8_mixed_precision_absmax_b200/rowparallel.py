@@ -9,8 +9,8 @@ So a row split needs one exchange before the product, and only one:
   1. every rank takes the column maxima of |X| over its rows (the library's statistics kernel),
   2. one all-reduce with MAX makes them the maxima over all rows (K floats),
   3. every rank appends one row to its X holding, in each column whose maximum exceeds the
-     threshold, that maximum, and zero elsewhere, and runs the whole layer on it with the
-     library's kernels.
+     threshold, that maximum, and zero elsewhere (the library's int8_outlier_row), and runs
+     the whole layer on it with the library's kernels.
 
 The appended row makes the rank's own outlier set the global one (it exceeds the threshold
 exactly in the global outlier columns, and no real row exceeds it anywhere else), and it leaves
@@ -40,29 +40,25 @@ def _library_column_absmax(X: torch.Tensor) -> torch.Tensor:
     return i8.int8_activation_stats(X)[1]
 
 
-def outlier_row(col_max: torch.Tensor, threshold: float) -> torch.Tensor:
-    """The appended row: col_max[j] where it exceeds the threshold (a negative threshold acts
-    as 0, +inf selects nothing), 0 elsewhere, in binary16.  The comparison is in float32, as in
-    the kernels; the maxima are binary16 magnitudes, so the conversion back is exact."""
-    t = max(float(threshold), 0.0)
-    col = col_max.to(torch.float32)
-    return torch.where(col > t, col, torch.zeros_like(col)).to(torch.float16)
+def _library_outlier_row(col_max: torch.Tensor, threshold: float) -> torch.Tensor:
+    return i8.int8_outlier_row(col_max.to(torch.float32).contiguous(), threshold)
 
 
 class RowParallelInt8Linear:
     """An Int8Linear whose tokens are split across the ranks of `group`.
 
     Every rank passes the whole layer's `weight` and `bias` and its own rows of X (any number,
-    zero included).  `local_forward(X, Wq, w_scale, bias, threshold) -> Y` and
-    `column_absmax(X) -> float32 [K]` run on this rank; by default the library's kernels on the
-    current CUDA device.
+    zero included).  `local_forward(X, Wq, w_scale, bias, threshold) -> Y`,
+    `column_absmax(X) -> float32 [K]` and `outlier_row(col_max, threshold) -> float16 [K]` run
+    on this rank; by default the library's kernels on the current CUDA device.
     """
 
     def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None,
                  threshold: float = i8.DEFAULT_THRESHOLD, group=None,
                  local_forward: LocalForward | None = None,
                  quantize: Callable[[torch.Tensor], tuple[torch.Tensor, torch.Tensor]] | None = None,
-                 column_absmax: Callable[[torch.Tensor], torch.Tensor] | None = None):
+                 column_absmax: Callable[[torch.Tensor], torch.Tensor] | None = None,
+                 outlier_row: Callable[[torch.Tensor, float], torch.Tensor] | None = None):
         if math.isnan(threshold):
             raise ValueError("threshold is NaN")
         self.group = group
@@ -73,6 +69,7 @@ class RowParallelInt8Linear:
         self.bias = None if bias is None else bias.to(torch.float16).contiguous()
         self.local_forward = local_forward or _library_forward
         self.column_absmax = column_absmax or _library_column_absmax
+        self.outlier_row = outlier_row or _library_outlier_row
 
     def global_column_absmax(self, X2: torch.Tensor) -> torch.Tensor:
         """max over the rows of every rank of |X[:, j]| (the one exchange of the split)."""
@@ -87,7 +84,7 @@ class RowParallelInt8Linear:
         lead = X.shape[:-1]
         X2 = X.reshape(-1, self.in_features).to(torch.float16).contiguous()
         M = X2.shape[0]
-        extra = outlier_row(self.global_column_absmax(X2), self.threshold)
+        extra = self.outlier_row(self.global_column_absmax(X2), self.threshold)
         if M == 0:
             return X2.new_empty(*lead, self.out_features)
         Xa = torch.cat([X2, extra.to(X2.device).view(1, -1)], dim=0)

@@ -256,13 +256,14 @@ def test_forward_accumulators_and_y(M, K, N, n_out, t):
 
 @pytest.mark.parametrize("M,K,N,cols,t", [
     (8, 2048, 512, list(range(640, 704)), 6.0),       # 64 outlier columns in 8 chunks
-    (8, 2048, 512, list(range(640, 705)), 6.0),       # 65 columns: fp16 MMAs instead
-    (6, 4096, 384, list(range(3, 4096, 57)), 6.0),    # 72 chunks with an outlier
+    (8, 2048, 512, list(range(640, 705)), 6.0),       # 65 columns: a ninth, partial chunk
+    (6, 4096, 384, list(range(3, 4096, 57)), 6.0),    # 72 chunks: more than the 64 kept
     (7, 1024, 200, [0, 1, 2, 1023], 6.0),             # first and last columns
 ])
 def test_decode_outlier_term_routes(M, K, N, cols, t):
-    """The one-launch decode kernel computes the fp16 term on CUDA cores for up to 64 outlier
-    columns (all within 64 chunks of 8) and with fp16 MMAs beyond; both against the oracle."""
+    """The one-launch decode kernel keeps the fp16 activations of up to 64 chunks of 8 columns
+    that hold an outlier in shared memory and reads the others from X again; the fp16 term runs
+    on the warp-level fp16 MMA either way.  Both cases against the oracle."""
     rng = np.random.default_rng(M * K + N + len(cols))
     X = rng.standard_normal((M, K))
     X[:, cols] *= rng.uniform(10, 40, size=len(cols))
@@ -278,7 +279,7 @@ def test_decode_outlier_term_routes(M, K, N, cols, t):
 def test_decode_workload_full_forward():
     w, X, W, b, _ = workload_inputs("decode_q_proj")
     Y, acc = check_forward_acc(X, W, b, w.threshold)
-    # repeated calls reuse the split-K counters: same bits every time
+    # repeated calls: same bits every time
     Y2, acc2 = check_forward_acc(X, W, b, w.threshold)
     np.testing.assert_array_equal(acc, acc2)
     np.testing.assert_array_equal(f16_bits(Y), f16_bits(Y2))
@@ -319,3 +320,31 @@ def test_quantizer_ties_and_near_ties_exact(M):
     Xq, _ = oracle.quantize_rows(X, mask)
     np.testing.assert_array_equal(acc, 127 * Xq.astype(np.int32))
     assert Xq[0, 1] == 63
+
+
+@pytest.mark.parametrize("M,K,N", [(8, 4096, 1024), (16, 2048, 512), (64, 512, 520)])
+def test_weights_quantized_just_before_the_forward(M, K, N):
+    """int8_quant_weight immediately followed by the forward on one stream, with nothing
+    launched in between (buffers allocated up front), twice with different weights written into
+    the same Wq buffer: the forward (whose decode route starts reading Wq before its dependency
+    wait) must see the new weights each time."""
+    rng = np.random.default_rng(M + K + N)
+    X = rng.standard_normal((M, K))
+    X[:, rng.choice(K, size=3, replace=False)] *= 25.0
+    X = X.astype(np.float16)
+    Ws = [(rng.standard_normal((N, K)) * s).astype(np.float16) for s in (0.02, 0.05)]
+    Xd = to_dev(X)
+    Wds = [to_dev(W) for W in Ws]
+    Wq = torch.empty((N, K), dtype=torch.int8, device="cuda")
+    sw = torch.empty(N, dtype=torch.float32, device="cuda")
+    Ys = [torch.empty((M, N), dtype=torch.float16, device="cuda") for _ in Ws]
+    ws = i8.new_workspace(M, N, K, Xd.device)
+    torch.cuda.synchronize()
+    for Wd, Y in zip(Wds, Ys):
+        i8.int8_quant_weight(Wd, Wq=Wq, w_scale=sw)
+        i8.int8_linear_forward(Xd, Wq, sw, None, 6.0, Y=Y, workspace=ws)
+    torch.cuda.synchronize()
+    assert i8.int8_read_device_status(ws[:4].view(torch.int32)) == 0
+    for W, Y in zip(Ws, Ys):
+        Wq_ref, sw_ref = oracle.quant_weight(W)
+        assert_y_close(to_np(Y), oracle.linear_forward(X, Wq_ref, sw_ref, None, 6.0))

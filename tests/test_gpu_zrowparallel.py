@@ -10,6 +10,7 @@ import pytest
 import torch
 import torch.distributed as dist
 
+import int8_mixed_precision_absmax_b200 as i8
 import oracle
 from int8_mixed_precision_absmax_b200 import rowparallel as rp
 from tests.gpu_helpers import assert_y_close, to_dev, to_np
@@ -41,3 +42,19 @@ def test_one_rank_token_split_equals_the_layer(nccl_group, M, K, N):
     assert Y.shape == (M, N)
     Y_ref = oracle.linear_forward(X, to_np(layer.Wq), to_np(layer.w_scale), b, 6.0)
     assert_y_close(Y, Y_ref, f"token split {M}x{K}x{N}")
+
+
+def test_outlier_row_marks_exactly_the_columns_above_the_threshold():
+    # column maxima are binary16 magnitudes: 6 and its two binary16 neighbours
+    col = torch.tensor([0.0, 5.99609375, 6.0, 6.00390625, 60.0, 65504.0] + [1.0] * 10,
+                       dtype=torch.float32, device="cuda")
+    row = i8.int8_outlier_row(col, 6.0)
+    assert row.dtype == torch.float16
+    np.testing.assert_array_equal(to_np(row.float())[:6], [0, 0, 0, 6.00390625, 60, 65504])
+    assert not to_np(row.float())[6:].any()
+    # the kernels see the row exceed the threshold exactly in the marked columns
+    np.testing.assert_array_equal(to_np(row.float()) > 6.0, to_np(col) > 6.0)
+    assert not to_np(i8.int8_outlier_row(col, float("inf")).float()).any()
+    np.testing.assert_array_equal(to_np(i8.int8_outlier_row(col, -3.0).float()), to_np(col))
+    with pytest.raises(i8.Int8mmError):
+        i8.int8_outlier_row(col, float("nan"))

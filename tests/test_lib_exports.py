@@ -111,6 +111,10 @@ def test_extended_entry_points_check_their_arguments(lib):
     assert L.int8_activation_stats(FAKE, 4, 40, None, FAKE, FAKE, 1 << 20, None) == -3
     assert L.int8_activation_stats(FAKE, 4, 32, None, FAKE, FAKE, 16, None) == -5
     assert L.int8_activation_stats_workspace_size() == 32768 * 4
+    # the token split's outlier row
+    assert L.int8_outlier_row(None, 32, 6.0, FAKE, None) == -1
+    assert L.int8_outlier_row(FAKE, 40, 6.0, FAKE, None) == -3
+    assert L.int8_outlier_row(FAKE, 32, math.nan, FAKE, None) == -4
 
 
 def test_remaining_entry_points_check_their_arguments(lib):
@@ -136,11 +140,29 @@ def test_remaining_entry_points_check_their_arguments(lib):
     assert L.int8_outlier_weights(FAKE, FAKE, 8, 40, FAKE, FAKE, FAKE, None) == -3
 
 
+def test_trace_entry_point_checks_its_arguments(lib):
+    L = lib
+    # the diagnostic forward: unknown flags, a misaligned output, a short workspace
+    assert L.int8_linear_forward_trace(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 2, FAKE,
+                                       None, None, None, None, None, None, FAKE, 1 << 20,
+                                       None) == -11
+    assert L.int8_linear_forward_trace(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 0, FAKE,
+                                       None, ctypes.c_void_p(0x10004), None, None, None, None,
+                                       FAKE, 1 << 20, None) == -3
+    assert L.int8_linear_forward_trace(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 0, FAKE,
+                                       None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, None) == -5
+    assert L.int8_linear_forward_trace(FAKE, 4, 40, FAKE, FAKE, None, None, 8, 6.0, 0, FAKE,
+                                       None, None, None, None, None, None, FAKE, 1 << 20,
+                                       None) == -3
+
+
 def test_noalloc_entry_point_checks_before_touching_its_scratch(lib):
     L = lib
     # beyond the few-token kernels the static scratch serves: a clear error, no device work
     assert L.int8_linear_forward_noalloc(FAKE, 17, 256, FAKE, FAKE, None, 128, 6.0, FAKE, None,
                                          None) == -10
+    assert L.int8_linear_forward_noalloc(FAKE, 17, 12288, FAKE, FAKE, None, 128, 6.0, FAKE,
+                                         None, None) == -10
     assert L.int8_linear_forward_noalloc(None, 8, 256, FAKE, FAKE, None, 128, 6.0, FAKE, None,
                                          None) == -1
     # the optional status word must be 4-byte aligned
