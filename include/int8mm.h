@@ -58,6 +58,7 @@ typedef struct CUstream_st *int8mm_stream_t; /* the same type as cudaStream_t */
 
 /* flags of int8_linear_forward_ex */
 #define INT8MM_PER_TENSOR_SCALE 1u   /* one activation scale for the whole of X */
+#define INT8MM_PAIR_TILES 2u         /* M > 128: 256 x 256 product tiles on CTA pairs */
 
 /* Bytes of the static device scratch behind int8_linear_forward_noalloc (per device). */
 #define INT8MM_NOALLOC_SCRATCH_BYTES (512 * 1024)
@@ -134,7 +135,13 @@ int int8_linear_forward_fp16w(const void *X, int M, int K, const int8_t *Wq,
  *                sx = (max over every row i and regular column j of |X[i,j]|) / 127, every
  *                row quantized with it ([P5] section "LLM.int8() 是怎么做到几乎无损的", item 2,
  *                as its snippet is written; the default one-per-row scale follows the
- *                vector-wise reading of [P2]).  Other bits: INT8MM_ERR_FLAGS.
+ *                vector-wise reading of [P2]);
+ *                INT8MM_PAIR_TILES: for M > 128, compute the products in 256 x 256 tiles, each
+ *                shared by a pair of CTAs (tcgen05 cta_group::2: each CTA loads half of the
+ *                operands), instead of 128 x 256 tiles on single CTAs.  Same results, bit for
+ *                bit in the integer stages; it moves a third less operand data per multiply-add
+ *                but, measured under the 1 kW power cap, is not faster (the default is the
+ *                single-CTA tile).  Other bits: INT8MM_ERR_FLAGS.
  *   acc    [out] NULL, or int32 [M, N]: the int8 accumulators, as int8_linear_forward_acc
  * Every other argument, the workspace and the error codes are as for int8_linear_forward.
  */

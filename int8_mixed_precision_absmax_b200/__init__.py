@@ -29,11 +29,12 @@ __all__ = [
     "int8_read_device_status", "int8_status_string", "int8_linear_forward_noalloc",
     "int8_linear_forward_fp16w", "int8_linear_forward_ex", "PER_TENSOR_SCALE",
     "int8_activation_stats", "Int8Linear", "DEFAULT_THRESHOLD", "int8_linear_forward_trace",
-    "int8_outlier_row",
+    "int8_outlier_row", "PAIR_TILES",
 ]
 
 DEFAULT_THRESHOLD = 6.0
 PER_TENSOR_SCALE = 1  # int8_linear_forward_ex flag: one activation scale for the whole of X
+PAIR_TILES = 2        # int8_linear_forward_ex flag: M > 128 products on CTA pairs (256 x 256)
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libint8mm.so")
 _lib = None
@@ -215,9 +216,11 @@ def int8_linear_forward_ex(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Ten
                            bias: torch.Tensor | None, threshold: float = DEFAULT_THRESHOLD,
                            W16: torch.Tensor | None = None, per_tensor: bool = False,
                            Y: torch.Tensor | None = None, acc: torch.Tensor | None = None,
-                           workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                           workspace: torch.Tensor | None = None, stream=None,
+                           pair_tiles: bool = False) -> torch.Tensor:
     """The layer with every option: the kept fp16 weights W16 (or None), one activation scale
-    for the whole of X (per_tensor), and the int32 accumulators written to acc (or not)."""
+    for the whole of X (per_tensor), the int32 accumulators written to acc (or not), and the
+    products on CTA pairs (pair_tiles, for M > 128)."""
     _need(X, torch.float16, "X", 2)
     _need(Wq, torch.int8, "Wq", 2)
     _need(w_scale, torch.float32, "w_scale", 1)
@@ -238,7 +241,7 @@ def int8_linear_forward_ex(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Ten
         n = int8_linear_workspace_size(M, N, K)
         workspace = torch.zeros(max(n, 256), dtype=torch.uint8, device=X.device)
     _need(workspace, torch.uint8, "workspace", 1)
-    flags = PER_TENSOR_SCALE if per_tensor else 0
+    flags = (PER_TENSOR_SCALE if per_tensor else 0) | (PAIR_TILES if pair_tiles else 0)
     _check(load_library().int8_linear_forward_ex(
         _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(W16), _ptr(bias), N, float(threshold),
         flags, _ptr(Y), _ptr(acc), _ptr(workspace), workspace.numel(),
@@ -249,7 +252,8 @@ def int8_linear_forward_ex(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Ten
 def int8_linear_forward_trace(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
                               bias: torch.Tensor | None, threshold: float = DEFAULT_THRESHOLD,
                               W16: torch.Tensor | None = None, per_tensor: bool = False,
-                              workspace: torch.Tensor | None = None, stream=None) -> dict:
+                              workspace: torch.Tensor | None = None, stream=None,
+                              pair_tiles: bool = False) -> dict:
     """One forward that also returns what its own kernels computed on the way: a dict of
     device tensors Y [M,N] fp16, acc [M,N] int32, Xq [M,K] int8, row_scale [M] f32,
     outlier_cols [K] i32 (first n_outliers valid), n_outliers [1] i32 and W_hat [N,K] fp16
@@ -276,7 +280,7 @@ def int8_linear_forward_trace(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.
     if workspace is None:
         workspace = new_workspace(M, N, K, dev)
     _need(workspace, torch.uint8, "workspace", 1)
-    flags = PER_TENSOR_SCALE if per_tensor else 0
+    flags = (PER_TENSOR_SCALE if per_tensor else 0) | (PAIR_TILES if pair_tiles else 0)
     _check(load_library().int8_linear_forward_trace(
         _ptr(X), M, K, _ptr(Wq), _ptr(w_scale), _ptr(W16), _ptr(bias), N, float(threshold),
         flags, _ptr(out["Y"]), _ptr(out["acc"]), _ptr(out["Xq"]), _ptr(out["row_scale"]),

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libint8mm.so")
-SOURCES = ["api.cu", "quant.cu", "gemm.cu", "small.cu", "gemv.cu", "decode.cu", "stats.cu", "trace.cu"]
+SOURCES = ["api.cu", "quant.cu", "gemm.cu", "gemm2.cu", "small.cu", "gemv.cu", "decode.cu", "stats.cu", "trace.cu"]
 HEADERS = ["kernels.cuh", "ptx.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

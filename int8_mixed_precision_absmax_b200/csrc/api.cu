@@ -111,6 +111,7 @@ namespace {
 struct LayerOpts {
   const void* W16 = nullptr;
   int per_tensor = 0;
+  bool pair_tiles = false;  // M > 128: the products on CTA pairs (gemm2.cu)
   TraceSink trace;  // diagnostic outputs written by the kernels themselves (all null normally)
 };
 
@@ -311,13 +312,16 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
       return INT8MM_ERR_CUDA;
     return launch_status(launch_small(map, a, sp, stream, pdl));
   }
+  // on request, many rows: one 256 x 256 tile per CTA pair, each CTA loading 128 weight rows
+  const bool pair = o.pair_tiles && M > kPairMinRows;
+  const uint32_t wrows = pair ? kPairHalfRows : kBN;
   GemmMaps maps;
   if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.xq, K, M, K, kBKBytes, kBM) ||
-      !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kBN) ||
+      !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, wrows) ||
       !encode_tmap_2d(&maps.xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.xo, p.L.ldo, M,
                       p.L.ldo * 2ull, kBKBytes / 2, kBM) ||
       !encode_tmap_2d(&maps.wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.wo, p.L.ldo, N,
-                      p.L.ldo * 2ull, kBKBytes / 2, kBN))
+                      p.L.ldo * 2ull, kBKBytes / 2, wrows))
     return INT8MM_ERR_CUDA;
   GemmArgs g;
   g.M = M;
@@ -329,8 +333,10 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   g.Y = static_cast<__half*>(Y);
   g.C = acc;
   g.n_out = p.header + 1;
+  g.group_m = 0;
   g.status = p.header;
-  return launch_status(launch_gemm(maps, g, stream, pdl));
+  return launch_status(pair ? launch_gemm_pair(maps, g, stream, pdl)
+                            : launch_gemm(maps, g, stream, pdl));
 }
 
 int forward_impl(const void* X, int M, int K, const int8_t* Wq, const float* w_scale,
@@ -408,10 +414,12 @@ int int8_linear_forward_ex(const void* X, int M, int K, const int8_t* Wq, const 
                            const void* W16, const void* bias, int N, float threshold,
                            unsigned flags, void* Y, int32_t* acc, void* workspace,
                            size_t ws_bytes, int8mm_stream_t stream) {
-  if (flags & ~static_cast<unsigned>(INT8MM_PER_TENSOR_SCALE)) return INT8MM_ERR_FLAGS;
+  if (flags & ~static_cast<unsigned>(INT8MM_PER_TENSOR_SCALE | INT8MM_PAIR_TILES))
+    return INT8MM_ERR_FLAGS;
   LayerOpts o;
   o.W16 = W16;
   o.per_tensor = (flags & INT8MM_PER_TENSOR_SCALE) ? 1 : 0;
+  o.pair_tiles = (flags & INT8MM_PAIR_TILES) != 0;
   return forward_impl(X, M, K, Wq, w_scale, bias, N, threshold, Y, acc, workspace, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream), o);
 }
@@ -491,9 +499,11 @@ int int8_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K, int32
   if (rc) return rc;
   if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(C)) return INT8MM_ERR_ALIGN;
   if ((rc = check_device())) return rc;
+  const bool pair = false;  // the raw product runs on single-CTA tiles
   GemmMaps maps;
   if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K, M, K, kBKBytes, kBM) ||
-      !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, kBN))
+      !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes,
+                      pair ? kPairHalfRows : kBN))
     return INT8MM_ERR_CUDA;
   maps.xo = maps.xq;  // unused: no outlier columns
   maps.wo = maps.wq;
@@ -504,7 +514,9 @@ int int8_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K, int32
   g.C = C;
   g.n_out = nullptr;
   g.status = dev_status;
-  return launch_status(launch_gemm(maps, g, reinterpret_cast<cudaStream_t>(stream_), false));
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  return launch_status(pair ? launch_gemm_pair(maps, g, stream, false)
+                            : launch_gemm(maps, g, stream, false));
 }
 
 int int8_outlier_weights(const int8_t* Wq, const float* w_scale, int N, int K,
@@ -526,7 +538,8 @@ int int8_linear_forward_trace(const void* X, int M, int K, const int8_t* Wq,
                               float* row_scale, int32_t* outlier_cols, int32_t* n_outliers,
                               void* W_hat, void* workspace, size_t ws_bytes,
                               int8mm_stream_t stream_) {
-  if (flags & ~static_cast<unsigned>(INT8MM_PER_TENSOR_SCALE)) return INT8MM_ERR_FLAGS;
+  if (flags & ~static_cast<unsigned>(INT8MM_PER_TENSOR_SCALE | INT8MM_PAIR_TILES))
+    return INT8MM_ERR_FLAGS;
   if ((Xq && !aligned16(Xq)) || (row_scale && !aligned16(row_scale)) ||
       (outlier_cols && !aligned16(outlier_cols)) || (n_outliers && !aligned16(n_outliers)) ||
       (W_hat && !aligned16(W_hat)))
@@ -543,6 +556,7 @@ int int8_linear_forward_trace(const void* X, int M, int K, const int8_t* Wq,
   LayerOpts o;
   o.W16 = W16;
   o.per_tensor = (flags & INT8MM_PER_TENSOR_SCALE) ? 1 : 0;
+  o.pair_tiles = (flags & INT8MM_PAIR_TILES) != 0;
   if (route == Route::kDecode || route == Route::kSmall) {
     // these kernels keep codes, scales and outlier bits on chip: they write them out here
     o.trace.xq = Xq;

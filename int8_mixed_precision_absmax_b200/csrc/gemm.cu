@@ -36,6 +36,10 @@ constexpr int kBBytes = kBN * kBKBytes;  // 32 KB
 constexpr int kThreads = 320;
 constexpr int kEpiThreads = kThreads - 64;  // warps 2..9
 constexpr uint32_t kTmemCols = 512;
+#ifndef I8MM_EPI_SLEEP_NS
+#define I8MM_EPI_SLEEP_NS 500
+#endif
+constexpr uint32_t kEpiSleepNs = I8MM_EPI_SLEEP_NS;  // epilogue poll interval on a tile
 constexpr uint32_t kIdescI8 = idesc_i8_s32(kBM, kBN);
 constexpr uint32_t kIdescF16 = idesc_f16_f32(kBM, kBN);
 
@@ -54,11 +58,19 @@ struct GemmShared {
 };
 constexpr size_t kSmemBytes = sizeof(GemmShared) + 1024;  // + alignment slack
 
+// Tiles in groups of gm row tiles: inside a group the row tile varies fastest, so the CTAs
+// of one wave share each weight tile through L2 while the group's activation rows (sized by
+// the host to stay resident in L2) are reused by every wave of the group.
 struct TileSchedule {
-  int m_tiles, tiles;
+  int m_tiles, n_tiles, tiles, gm;
   __device__ void coords(int tile, int& m0, int& n0) const {
-    m0 = (tile % m_tiles) * kBM;  // consecutive blocks share the weight tile
-    n0 = (tile / m_tiles) * kBN;
+    const int per_group = gm * n_tiles;
+    const int g = tile / per_group;
+    const int first = g * gm;
+    const int rows = min(gm, m_tiles - first);
+    const int r = tile - g * per_group;
+    m0 = (first + r % rows) * kBM;
+    n0 = (r / rows) * kBN;
   }
 };
 
@@ -136,7 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nslots = both ? 1 : 2;
   TileSchedule sched;
   sched.m_tiles = (M + kBM - 1) / kBM;
-  sched.tiles = sched.m_tiles * ((N + kBN - 1) / kBN);
+  sched.n_tiles = (N + kBN - 1) / kBN;
+  sched.tiles = sched.m_tiles * sched.n_tiles;
+  sched.gm = (args.group_m > 0 && args.group_m < sched.m_tiles) ? args.group_m : sched.m_tiles;
   const uint32_t tmem = S.tmem_base;
   volatile int* abort = &S.abort;
 
@@ -238,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         S.bias[it & 1][et] = (et < kBN && n < N && args.bias) ? __half2float(args.bias[n]) : 0.0f;
         epi_sync();
       }
-      const bool landed = mbar_wait_bounded(&S.tmem_full[slot], use & 1u, abort);
+      const bool landed = mbar_wait_patient(&S.tmem_full[slot], use & 1u, abort, kEpiSleepNs);
       if (epi_any(!landed)) {  // every epilogue thread takes the same branch
         report(args.status, INT8MM_ERR_TIMEOUT);
         break;
@@ -457,7 +471,17 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t st
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  const int tiles = ((a.M + kBM - 1) / kBM) * ((a.N + kBN - 1) / kBN);
+  const int m_tiles = (a.M + kBM - 1) / kBM;
+  const int tiles = m_tiles * ((a.N + kBN - 1) / kBN);
+  // row tiles per group: as many as keep the group's int8 activations (gm x 128 rows x K
+  // bytes) within 32 MiB of L2, balanced over the groups
+  GemmArgs args = a;
+  const long long budget = 32ll << 20;
+  const long long row_tile_bytes = static_cast<long long>(kBM) * a.K;
+  const int gm_max = static_cast<int>(budget / row_tile_bytes) > 1
+                         ? static_cast<int>(budget / row_tile_bytes) : 1;
+  const int groups = (m_tiles + gm_max - 1) / gm_max;
+  args.group_m = (m_tiles + groups - 1) / groups;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles < num_sms ? tiles : num_sms);
   cfg.blockDim = dim3(kThreads);
@@ -468,7 +492,7 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t st
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel, maps.xq, maps.wq, maps.xo, maps.wo, a);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel, maps.xq, maps.wq, maps.xo, maps.wo, args);
 }
 
 }  // namespace i8mm

@@ -221,6 +221,7 @@ struct GemmArgs {
   __half* Y;             // fused epilogue output [M,N], or null
   int32_t* C;            // raw int32 accumulators [M,N], or null (at least one of Y, C)
   const int32_t* n_out;  // device outlier count, or null for none
+  int group_m;           // row tiles per group of the tile order (set by launch_gemm)
   int32_t* status;
 };
 struct GemmMaps {
@@ -236,6 +237,12 @@ bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
                     const uint64_t (&dims)[3], const uint64_t (&strides_bytes)[2],
                     const uint32_t (&box)[3], CUtensorMapSwizzle swizzle);
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream, bool pdl);
+// The same product with one 256 x 256 tile per CTA pair (gemm2.cu), for M > kPairMinRows; its
+// weight maps (wq, wo) take boxes of 128 rows, half of kBN.
+cudaError_t launch_gemm_pair(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream,
+                             bool pdl);
+constexpr int kPairMinRows = 128;
+constexpr int kPairHalfRows = 128;
 
 // GEMM tile shape (shared with the host for map boxes)
 constexpr int kBM = 128;

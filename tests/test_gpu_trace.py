@@ -30,7 +30,7 @@ def random_case(M, K, N, n_out, seed, factor=20.0, bias=True):
     return X.astype(np.float16), W.astype(np.float16), b
 
 
-def check_trace(X, W, b, t, per_tensor=False, keep_w16=False):
+def check_trace(X, W, b, t, per_tensor=False, keep_w16=False, pair_tiles=False):
     """Every output of the trace against the oracle; returns the trace (host arrays)."""
     Xd = to_dev(X)
     Wd = to_dev(W)
@@ -41,7 +41,7 @@ def check_trace(X, W, b, t, per_tensor=False, keep_w16=False):
     N = W.shape[0]
     ws = i8.new_workspace(M, N, K, Xd.device)
     tr = i8.int8_linear_forward_trace(Xd, Wq_d, sw_d, bd, t, W16=W16, per_tensor=per_tensor,
-                                      workspace=ws)
+                                      workspace=ws, pair_tiles=pair_tiles)
     assert i8.int8_read_device_status(ws[:4].view(torch.int32)) == 0
     g = {k: to_np(v) for k, v in tr.items()}
     Wq, sw = to_np(Wq_d), to_np(sw_d)
@@ -68,7 +68,7 @@ def check_trace(X, W, b, t, per_tensor=False, keep_w16=False):
     # the same bits as the forward without the trace
     acc2 = torch.empty((M, N), dtype=torch.int32, device=Xd.device)
     Y2 = i8.int8_linear_forward_ex(Xd, Wq_d, sw_d, bd, t, W16=W16, per_tensor=per_tensor,
-                                   acc=acc2, workspace=ws)
+                                   acc=acc2, workspace=ws, pair_tiles=pair_tiles)
     np.testing.assert_array_equal(f16_bits(to_np(Y2)), f16_bits(g["Y"]))
     np.testing.assert_array_equal(to_np(acc2), g["acc"])
     return g
@@ -143,3 +143,39 @@ def test_trace_planted_ties(M, K):
     X = X.astype(np.float16)
     W = (rng.standard_normal((64, K)) * 0.02).astype(np.float16)
     check_trace(X, W, None, 6.0)
+
+
+@pytest.mark.parametrize("M,K,N,n_out,t", [
+    (300, 1040, 600, 5, 6.0),     # ragged pair tiles in M, N and K
+    (129, 256, 257, 1, 6.0),      # one row past a single tile: a pair tile mostly empty
+    (512, 2048, 1000, 70, 6.0),   # more outliers than one fp16 k-block
+    (384, 512, 520, 0, math.inf), # no outlier term: two accumulator slots
+    (256, 384, 300, 0, 0.0),      # every column an outlier: fp16 product only
+])
+def test_trace_pair_tiles(M, K, N, n_out, t):
+    """The products on CTA pairs (256 x 256 tiles, tcgen05 cta_group::2) against the oracle, and
+    against the single-CTA tiles bit for bit in the integer stages."""
+    X, W, b = random_case(M, K, N, n_out, seed=5 * M + K + N)
+    g = check_trace(X, W, b, t, pair_tiles=True)
+    g1 = check_trace(X, W, b, t)
+    np.testing.assert_array_equal(g["acc"], g1["acc"])
+
+
+def test_pair_tiles_full_size_prefill():
+    w, X, W, b, _ = workload_inputs("prefill_up_proj")
+    Xd, Wd = to_dev(X), to_dev(W)
+    Wq_d, sw_d = i8.int8_quant_weight(Wd)
+    bd = to_dev(b)
+    ws = i8.new_workspace(w.M, w.N, w.K, Xd.device)
+    acc_p = torch.empty((w.M, w.N), dtype=torch.int32, device="cuda")
+    acc_1 = torch.empty((w.M, w.N), dtype=torch.int32, device="cuda")
+    Yp = i8.int8_linear_forward_ex(Xd, Wq_d, sw_d, bd, w.threshold, acc=acc_p, workspace=ws,
+                                   pair_tiles=True)
+    Y1 = i8.int8_linear_forward_ex(Xd, Wq_d, sw_d, bd, w.threshold, acc=acc_1, workspace=ws)
+    assert i8.int8_read_device_status(ws[:4].view(torch.int32)) == 0
+    assert torch.equal(acc_p, acc_1)
+    rows = np.array([0, 1, 777, w.M - 1])
+    Y_ref, A_ref = oracle.linear_forward_rows(X, to_np(Wq_d), to_np(sw_d), b, w.threshold, rows)
+    np.testing.assert_array_equal(to_np(acc_p)[rows], A_ref)
+    assert_y_close(to_np(Yp)[rows], Y_ref)
+    assert_y_close(to_np(Yp), to_np(Y1))

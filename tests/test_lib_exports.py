@@ -103,7 +103,7 @@ def test_fp16_weight_entry_point_checks_its_weights(lib):
 def test_extended_entry_points_check_their_arguments(lib):
     L = lib
     # unknown flag bits are rejected before anything else
-    assert L.int8_linear_forward_ex(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 2, FAKE, None,
+    assert L.int8_linear_forward_ex(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 4, FAKE, None,
                                     FAKE, 1 << 20, None) == -11
     assert L.int8_linear_forward_ex(None, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 1, FAKE, None,
                                     FAKE, 1 << 20, None) == -1
@@ -143,7 +143,7 @@ def test_remaining_entry_points_check_their_arguments(lib):
 def test_trace_entry_point_checks_its_arguments(lib):
     L = lib
     # the diagnostic forward: unknown flags, a misaligned output, a short workspace
-    assert L.int8_linear_forward_trace(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 2, FAKE,
+    assert L.int8_linear_forward_trace(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 4, FAKE,
                                        None, None, None, None, None, None, FAKE, 1 << 20,
                                        None) == -11
     assert L.int8_linear_forward_trace(FAKE, 4, 32, FAKE, FAKE, None, None, 8, 6.0, 0, FAKE,
