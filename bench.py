@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-per-config", action="store_true",
                     help="time only the headline workload")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--quick", action="store_true",
+                    help="few launches (for profilers): no clock sampling, short end-to-end "
+                         "and per-kernel timings; the line's numbers are indicative only")
     return ap.parse_args(argv)
 
 
@@ -322,7 +325,10 @@ def forward_path(M: int, N: int, K: int):
             "matmul": "gemm_kernel (int8 + fp16 tcgen05, fused epilogue)"}
 
 
-def graph_time_ms(fn, n: int, device, min_ms: float = 200.0) -> float:
+GRAPH_MIN_MS = 200.0  # replays per per-kernel timing (lowered by --quick)
+
+
+def graph_time_ms(fn, n: int, device, min_ms: float | None = None) -> float:
     """Average device time of fn() replayed back to back from one CUDA graph of n calls, over
     at least `min_ms` of replays (CUDA events on the launching stream)."""
     import torch
@@ -345,6 +351,7 @@ def graph_time_ms(fn, n: int, device, min_ms: float = 200.0) -> float:
     g.replay()
     b.record()
     torch.cuda.synchronize()
+    min_ms = GRAPH_MIN_MS if min_ms is None else min_ms
     reps = max(3, min(10000, int(min_ms / max(a.elapsed_time(b), 1e-3))))
     a.record()
     for _ in range(reps):
@@ -496,40 +503,74 @@ class Layer:
 
     def e2e(self, world: int, budget_s: float):
         """The same metric through the public call, with a pinned host->device copy of X and a
-        device->host copy of Y inside every step."""
+        device->host copy of Y inside every step.  The copies of neighbouring steps overlap the
+        forward on their own streams (X and Y double-buffered on the device, two pinned Y
+        buffers on the host), as a serving loop would run them: step i's Y goes back while
+        step i+1 computes and step i+2's X comes in."""
         import torch
         w = self.w
+        dev = self.device
         Xh = torch.from_numpy(self.X_h).pin_memory()
-        Yh = torch.empty((w.M, w.N), dtype=torch.float16).pin_memory()
-        c = self.copies
+        Yh = [torch.empty((w.M, w.N), dtype=torch.float16).pin_memory() for _ in range(2)]
+        Xd = [self.Xs[0], self.Xs[1] if self.copies > 1 else torch.empty_like(self.Xs[0])]
+        Yd = [self.Ys[0], self.Ys[1] if self.copies > 1 else torch.empty_like(self.Ys[0])]
+        s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        ev = lambda: torch.cuda.Event()
+        import int8_mixed_precision_absmax_b200 as i8
 
-        def one(i):
-            self.Xs[i % c].copy_(Xh, non_blocking=True)
-            self.step(i)
-            Yh.copy_(self.Ys[i % c], non_blocking=True)
-        for i in range(3):
-            one(i)
+        def run(n):
+            x_free = [None, None]   # forward done with Xd[b]
+            y_free = [None, None]   # Yd[b] copied out
+            for i in range(n):
+                b = i % 2
+                with torch.cuda.stream(s_in):
+                    if x_free[b] is not None:
+                        s_in.wait_event(x_free[b])
+                    Xd[b].copy_(Xh, non_blocking=True)
+                    x_in = ev(); x_in.record(s_in)
+                with torch.cuda.stream(s_run):
+                    s_run.wait_event(x_in)
+                    if y_free[b] is not None:
+                        s_run.wait_event(y_free[b])
+                    c = i % self.copies
+                    i8.int8_linear_forward(Xd[b], self.Wqs[c], self.sws[c], self.bs[c],
+                                           w.threshold, Y=Yd[b], workspace=self.wss[c],
+                                           stream=s_run)
+                    done = ev(); done.record(s_run)
+                    x_free[b] = done
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(done)
+                    Yh[b].copy_(Yd[b], non_blocking=True)
+                    out = ev(); out.record(s_out)
+                    y_free[b] = out
+            for s_ in (s_in, s_run, s_out):
+                torch.cuda.current_stream(dev).wait_stream(s_)
+        run(3)
         torch.cuda.synchronize()
-        e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e_a.record()
-        for i in range(3):
-            one(i)
-        e_b.record()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for s_ in (s_in, s_run, s_out):
+            s_.wait_stream(torch.cuda.current_stream(dev))
+        run(3)
+        t1.record()
         torch.cuda.synchronize()
-        est = e_a.elapsed_time(e_b) / 3
+        est = t0.elapsed_time(t1) / 3
         n_e = int(max(5, min(20000, budget_s * 1e3 / max(est, 1e-3))))
-        n_e = int(max_over_ranks(float(n_e), self.device))
-        barrier(self.device)
-        e_a.record()
-        for i in range(n_e):
-            one(i)
-        e_b.record()
+        n_e = int(max_over_ranks(float(n_e), dev))
+        barrier(dev)
+        t0.record()
+        for s_ in (s_in, s_run, s_out):  # no copy starts before t0
+            s_.wait_stream(torch.cuda.current_stream(dev))
+        run(n_e)
+        t1.record()
         torch.cuda.synchronize()
-        e2e_s = max_over_ranks(e_a.elapsed_time(e_b) / 1e3, self.device)
+        e2e_s = max_over_ranks(t0.elapsed_time(t1) / 1e3, dev)
         return {"value": whole_job_rate(w.ops, n_e, world, e2e_s) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
-                "d2h_bytes_per_step": int(Yh.numel() * Yh.element_size()), "steps": n_e,
-                "ms_per_step": e2e_s / n_e * 1e3}
+                "d2h_bytes_per_step": int(Yh[0].numel() * Yh[0].element_size()), "steps": n_e,
+                "ms_per_step": e2e_s / n_e * 1e3,
+                "overlap": "H2D of X, forward and D2H of Y on three streams, double-buffered"}
 
     def roofline(self, n_out: int, q_ms: float, g_ms: float, step_ms: float, peaks):
         """The product kernel against its roofline, and the whole step against the same."""
@@ -643,6 +684,10 @@ def run_ours(args):
     peaks["f16_tflops"] = peaks["bf16_tflops"]
     use_graph = not args.no_graph
     warm = max(args.warmup, 0)
+    global GRAPH_MIN_MS
+    if args.quick:
+        GRAPH_MIN_MS = 5.0
+    e2e_budget = 0.02 if args.quick else 2.0
     uuid = None
     try:
         uuid = "GPU-" + str(props.uuid)
@@ -655,8 +700,8 @@ def run_ours(args):
     est_ms = layer.estimate_ms()
     steps = args.steps if args.steps is not None else max(20, int(2000.0 / max(est_ms, 1e-3)))
     steps = int(max_over_ranks(float(steps), device))
-    sampler = ClockSampler(uuid) if rank == 0 else None
-    head = measure(layer, world, steps, warm, use_graph, peaks, sampler)
+    sampler = ClockSampler(uuid) if rank == 0 and not args.quick else None
+    head = measure(layer, world, steps, warm, use_graph, peaks, sampler, e2e_budget_s=e2e_budget)
     head["roofline"]["traffic"] = recorded_traffic(w.name, layer.path["kernel"])
 
     cpu = None
@@ -682,7 +727,8 @@ def run_ours(args):
             p_est = pl.estimate_ms()
             p_steps = int(max_over_ranks(float(max(20, int(PER_CONFIG_MIN_S * 1e3 / max(p_est, 1e-3)))),
                                          device))
-            r = measure(pl, world, p_steps, warm, use_graph, peaks, None, e2e_budget_s=1.0)
+            r = measure(pl, world, p_steps, warm, use_graph, peaks, None,
+                        e2e_budget_s=min(1.0, e2e_budget))
             r["roofline"]["traffic"] = recorded_traffic(pw.name, pl.path["kernel"])
             r.pop("clocks", None)
             per_config[name] = r
@@ -695,6 +741,8 @@ def run_ours(args):
         cfg["parallelism"] = f"{world} independent replica(s), one per GPU"
         cfg["clocks_window"] = ("nvidia-smi every 200 ms over about 1 s of the same steps run "
                                 "back to back just before the timed ones, and over the timed ones")
+        if args.quick:
+            cfg["quick"] = "profiling run: no clock sampling, short timings"
         line = {
             "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
             "steps": steps, "warmup": warm, "ms_per_step": head["ms_per_step"],

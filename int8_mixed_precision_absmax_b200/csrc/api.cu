@@ -314,7 +314,8 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   }
   // on request, many rows: one 256 x 256 tile per CTA pair, each CTA loading 128 weight rows
   const bool pair = o.pair_tiles && M > kPairMinRows;
-  const uint32_t wrows = pair ? kPairHalfRows : kBN;
+  const int bn = pair ? kBN : gemm_tile_width(M, N);  // channels per product tile
+  const uint32_t wrows = pair ? kPairHalfRows : static_cast<uint32_t>(bn);
   GemmMaps maps;
   if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.xq, K, M, K, kBKBytes, kBM) ||
       !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes, wrows) ||
@@ -334,6 +335,7 @@ int run_matmul(const void* X, int M, int K, const int8_t* Wq, const float* w_sca
   g.C = acc;
   g.n_out = p.header + 1;
   g.group_m = 0;
+  g.bn = bn;
   g.status = p.header;
   return launch_status(pair ? launch_gemm_pair(maps, g, stream, pdl)
                             : launch_gemm(maps, g, stream, pdl));
@@ -500,10 +502,11 @@ int int8_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K, int32
   if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(C)) return INT8MM_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   const bool pair = false;  // the raw product runs on single-CTA tiles
+  const int bn = gemm_tile_width(M, N);
   GemmMaps maps;
   if (!encode_tmap_2d(&maps.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K, M, K, kBKBytes, kBM) ||
       !encode_tmap_2d(&maps.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, kBKBytes,
-                      pair ? kPairHalfRows : kBN))
+                      static_cast<uint32_t>(bn)))
     return INT8MM_ERR_CUDA;
   maps.xo = maps.xq;  // unused: no outlier columns
   maps.wo = maps.wq;
@@ -513,6 +516,7 @@ int int8_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K, int32
   g.K = K;
   g.C = C;
   g.n_out = nullptr;
+  g.bn = bn;
   g.status = dev_status;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   return launch_status(pair ? launch_gemm_pair(maps, g, stream, false)

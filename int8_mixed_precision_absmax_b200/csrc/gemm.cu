@@ -40,8 +40,7 @@ constexpr uint32_t kTmemCols = 512;
 #define I8MM_EPI_SLEEP_NS 500
 #endif
 constexpr uint32_t kEpiSleepNs = I8MM_EPI_SLEEP_NS;  // epilogue poll interval on a tile
-constexpr uint32_t kIdescI8 = idesc_i8_s32(kBM, kBN);
-constexpr uint32_t kIdescF16 = idesc_f16_f32(kBM, kBN);
+
 
 struct GemmShared {
   uint8_t a[kStages][kABytes];
@@ -62,7 +61,7 @@ constexpr size_t kSmemBytes = sizeof(GemmShared) + 1024;  // + alignment slack
 // of one wave share each weight tile through L2 while the group's activation rows (sized by
 // the host to stay resident in L2) are reused by every wave of the group.
 struct TileSchedule {
-  int m_tiles, n_tiles, tiles, gm;
+  int m_tiles, n_tiles, tiles, gm, bn;
   __device__ void coords(int tile, int& m0, int& n0) const {
     const int per_group = gm * n_tiles;
     const int g = tile / per_group;
@@ -70,7 +69,7 @@ struct TileSchedule {
     const int rows = min(gm, m_tiles - first);
     const int r = tile - g * per_group;
     m0 = (first + r % rows) * kBM;
-    n0 = (r / rows) * kBN;
+    n0 = (r / rows) * bn;
   }
 };
 
@@ -146,9 +145,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kb_total = kb_i8 + kb_f16;
   const bool both = kb_i8 > 0 && kb_f16 > 0;
   const int nslots = both ? 1 : 2;
+  const int bn = args.bn > 0 ? args.bn : kBN;  // channels per tile
+  const uint32_t idesc_i8 = idesc_i8_s32(kBM, bn);
+  const uint32_t idesc_f16 = idesc_f16_f32(kBM, bn);
   TileSchedule sched;
+  sched.bn = bn;
   sched.m_tiles = (M + kBM - 1) / kBM;
-  sched.n_tiles = (N + kBN - 1) / kBN;
+  sched.n_tiles = (N + bn - 1) / bn;
   sched.tiles = sched.m_tiles * sched.n_tiles;
   sched.gm = (args.group_m > 0 && args.group_m < sched.m_tiles) ? args.group_m : sched.m_tiles;
   const uint32_t tmem = S.tmem_base;
@@ -165,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sched.coords(tile, m0, n0);
         for (int kb = 0; kb < kb_total; ++kb) {
           if (!mbar_wait_bounded(&S.empty[stage], phase ^ 1u, abort)) { ok = false; break; }
-          mbar_arrive_expect_tx(&S.full[stage], kABytes + kBBytes);
+          mbar_arrive_expect_tx(&S.full[stage], kABytes + bn * kBKBytes);
           if (kb < kb_i8) {
             tma_load_2d(&map_xq, S.a[stage], &S.full[stage], kb * kBKBytes, m0);
             tma_load_2d(&map_wq, S.b[stage], &S.full[stage], kb * kBKBytes, n0);
@@ -215,9 +218,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t ad = sw128_kmajor_desc(a0 + 32u * k);
             const uint64_t bd = sw128_kmajor_desc(b0 + 32u * k);
             if (kb < kb_i8)
-              mma_i8(d_i8, ad, bd, kIdescI8, (kb > 0 || k > 0) ? 1u : 0u);
+              mma_i8(d_i8, ad, bd, idesc_i8, (kb > 0 || k > 0) ? 1u : 0u);
             else
-              mma_f16(d_f32, ad, bd, kIdescF16, (kb > kb_i8 || k > 0) ? 1u : 0u);
+              mma_f16(d_f32, ad, bd, idesc_f16, (kb > kb_i8 || k > 0) ? 1u : 0u);
           }
           mma_commit(&S.empty[stage]);  // frees the stage once these MMAs have read it
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -234,7 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // -------------------------------------------------- epilogue (warps 2..9)
     const int quad = warp & 3;                // TMEM lanes 32 quad .. 32 quad + 31
-    const int half = (warp - 2) / 4;          // columns 128 half .. 128 half + 127
+    const int half = (warp - 2) / 4;          // the first or the second half of the tile's columns
+    // 16-column chunks: the first half takes ceil(chunks / 2) of them
+    const int c_split = (bn / 16 + 1) / 2 * 16;
+    const int c_begin = half ? c_split : 0, c_end = half ? bn : c_split;
     const int et = threadIdx.x - 64;          // 0 .. kEpiThreads - 1
     const bool vec_ok = (N % 8) == 0;
     int it = 0;
@@ -248,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const int n = n0 + et;
         // (the raw int32 product has neither: w_scale and bias are null there)
-        S.wscale[it & 1][et] = (et < kBN && n < N && args.w_scale) ? args.w_scale[n] : 0.0f;
-        S.bias[it & 1][et] = (et < kBN && n < N && args.bias) ? __half2float(args.bias[n]) : 0.0f;
+        S.wscale[it & 1][et] = (et < bn && n < N && args.w_scale) ? args.w_scale[n] : 0.0f;
+        S.bias[it & 1][et] = (et < bn && n < N && args.bias) ? __half2float(args.bias[n]) : 0.0f;
         epi_sync();
       }
       const bool landed = mbar_wait_patient(&S.tmem_full[slot], use & 1u, abort, kEpiSleepNs);
@@ -268,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* bsc = S.bias[it & 1];
       if (both) {
         // phase 1: Y in fp32 over the outlier accumulator, then the int32 columns are free
-        for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 16) {
+        for (int c = c_begin; c < c_end; c += 16) {
           uint32_t ra[16], rp[16];
           __syncwarp();
           tmem_ld16(t_i8 + c, ra);
@@ -308,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&S.tmem_empty[0]);
         // phase 2: Y out, then the fp32 columns are free
-        for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 16) {
+        for (int c = c_begin; c < c_end; c += 16) {
           uint32_t ry[16];
           __syncwarp();
           tmem_ld16(t_f32 + c, ry);
@@ -338,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&S.tmem_empty[1]);
         continue;
       }
-      for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 16) {
+      for (int c = c_begin; c < c_end; c += 16) {
         uint32_t ra[16], rp[16];
         __syncwarp();  // the tensor-memory loads are warp-collective
         if (kb_i8 > 0) tmem_ld16(t_i8 + c, ra);
@@ -457,6 +463,28 @@ bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int gemm_tile_width(int M, int N) {
+  // Measured: the widths that fill the last wave (224 for the 13B-shaped layer, 240 for
+  // prefill up_proj) ran 10% faster in an isolated launch of the 13B-shaped layer and within 1%
+  // under steps back to back at the 1 kW power cap (where a partly filled last wave costs
+  // less: the idle SMs let the busy ones clock higher).
+  const int ctas = device_sm_count();
+  const long long m_tiles = (M + kBM - 1) / kBM;
+  constexpr int kFixed = 32;  // per-tile cost beyond the MMA columns, in the same units
+  int best = kBN;
+  long long best_cost = -1;
+  for (int bn = kBN; bn >= 128; bn -= 16) {
+    const long long tiles = m_tiles * ((N + bn - 1) / bn);
+    const long long waves = (tiles + ctas - 1) / ctas;
+    const long long cost = waves * (bn + kFixed);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream, bool pdl) {
   static int configured_device = -1;
   static int num_sms = 0;
@@ -472,7 +500,8 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t st
     configured_device = dev;
   }
   const int m_tiles = (a.M + kBM - 1) / kBM;
-  const int tiles = m_tiles * ((a.N + kBN - 1) / kBN);
+  const int bn = a.bn > 0 ? a.bn : kBN;
+  const int tiles = m_tiles * ((a.N + bn - 1) / bn);
   // row tiles per group: as many as keep the group's int8 activations (gm x 128 rows x K
   // bytes) within 32 MiB of L2, balanced over the groups
   GemmArgs args = a;

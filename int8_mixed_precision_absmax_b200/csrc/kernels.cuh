@@ -222,6 +222,8 @@ struct GemmArgs {
   int32_t* C;            // raw int32 accumulators [M,N], or null (at least one of Y, C)
   const int32_t* n_out;  // device outlier count, or null for none
   int group_m;           // row tiles per group of the tile order (set by launch_gemm)
+  int bn;                // output channels per tile of the single-CTA product (multiple of 16,
+                         // 128..kBN; 0 means kBN), chosen by gemm_tile_width
   int32_t* status;
 };
 struct GemmMaps {
@@ -237,6 +239,11 @@ bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
                     const uint64_t (&dims)[3], const uint64_t (&strides_bytes)[2],
                     const uint32_t (&box)[3], CUtensorMapSwizzle swizzle);
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream, bool pdl);
+// Output channels per tile of the single-CTA product for an M x N output: the width (a multiple
+// of 16 from 128 to kBN) that minimises (waves of tiles over the persistent CTAs) x (width + a
+// fixed per-tile cost), preferring the widest on ties.  The weight maps take boxes of this
+// many rows.
+int gemm_tile_width(int M, int N);
 // The same product with one 256 x 256 tile per CTA pair (gemm2.cu), for M > kPairMinRows; its
 // weight maps (wq, wo) take boxes of 128 rows, half of kBN.
 cudaError_t launch_gemm_pair(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream,
