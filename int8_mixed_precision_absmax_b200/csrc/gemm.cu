@@ -36,10 +36,6 @@ constexpr int kBBytes = kBN * kBKBytes;  // 32 KB
 constexpr int kThreads = 320;
 constexpr int kEpiThreads = kThreads - 64;  // warps 2..9
 constexpr uint32_t kTmemCols = 512;
-#ifndef I8MM_EPI_SLEEP_NS
-#define I8MM_EPI_SLEEP_NS 500
-#endif
-constexpr uint32_t kEpiSleepNs = I8MM_EPI_SLEEP_NS;  // epilogue poll interval on a tile
 
 
 struct GemmShared {
@@ -258,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         S.bias[it & 1][et] = (et < bn && n < N && args.bias) ? __half2float(args.bias[n]) : 0.0f;
         epi_sync();
       }
-      const bool landed = mbar_wait_patient(&S.tmem_full[slot], use & 1u, abort, kEpiSleepNs);
+      const bool landed = mbar_wait_bounded(&S.tmem_full[slot], use & 1u, abort);
       if (epi_any(!landed)) {  // every epilogue thread takes the same branch
         report(args.status, INT8MM_ERR_TIMEOUT);
         break;

@@ -19,10 +19,9 @@
 // the ring is latency-bound: a stage is locked from its load until about 1700 cycles after its
 // MMAs finish (when their commit reaches the producer), so the tensor pipe only stays busy when
 // the ring holds more MMA work than load latency plus that round trip.  (Measured: 4, 6 and 7
-// stages ran within 1% of each other, and asking L2 for the boxes ahead of the loads
-// (kPrefetch > 0) doubled the L2 requests and slowed the kernel by a fifth, so it is off.)  The
-// epilogue reads the column scales from global memory (L1) and leaves the shared memory to the
-// ring.
+// stages ran within 1% of each other, and asking L2 for each stage's boxes eight k-blocks ahead
+// of its loads doubled the L2 requests and slowed the kernel by a fifth.)  The epilogue reads the
+// column scales from global memory (L1) and leaves the shared memory to the ring.
 //
 // Roles (320 threads per CTA): warp 0 issues TMA loads (both CTAs; completion is counted on
 // the leader's barrier), warp 1 allocates tensor memory (both CTAs, together) and issues the
@@ -38,18 +37,7 @@ namespace {
 constexpr int kPM = 256;                             // rows of a pair tile (128 per CTA)
 constexpr int kPN = 256;                             // output channels of a pair tile
 constexpr int kHalfRows = 128;                       // operand rows one CTA holds
-#ifndef I8MM_PAIR_STAGES
-#define I8MM_PAIR_STAGES 6
-#endif
-#ifndef I8MM_PAIR_PREFETCH
-#define I8MM_PAIR_PREFETCH 0
-#endif
-constexpr int kPStages = I8MM_PAIR_STAGES;
-constexpr int kPrefetch = I8MM_PAIR_PREFETCH;        // k-blocks between L2 prefetch and load
-#ifndef I8MM_EPI_SLEEP_NS
-#define I8MM_EPI_SLEEP_NS 500
-#endif
-constexpr uint32_t kEpiSleepNs = I8MM_EPI_SLEEP_NS;  // epilogue poll interval on a tile
+constexpr int kPStages = 6;
 constexpr int kOpBytes = kHalfRows * kBKBytes;       // 16 KB: 128 rows x 128 bytes
 constexpr int kPThreads = 320;
 constexpr int kPEpiThreads = kPThreads - 64;         // warps 2..9
@@ -209,22 +197,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------ producer (both CTAs)
       const uint32_t full0 = mapa_shared(smem_addr(&S.full[0]), 0);  // the leader's barriers
-      // L2 prefetch of this CTA's boxes of the t-th (tile, k-block) of the pair's sequence
-      auto prefetch = [&](int t) {
-        const int tile = pair + (t / kb_total) * pairs, kb = t % kb_total;
-        if (tile >= sched.tiles) return;
-        int m0, n0;
-        sched.coords(tile, m0, n0);
-        if (kb < kb_i8) {
-          tma_prefetch_2d(&map_xq, kb * kBKBytes, m0 + row_off);
-          tma_prefetch_2d(&map_wq, kb * kBKBytes, n0 + row_off);
-        } else {
-          tma_prefetch_2d(&map_xo, (kb - kb_i8) * 64, m0 + row_off);
-          tma_prefetch_2d(&map_wo, (kb - kb_i8) * 64, n0 + row_off);
-        }
-      };
-      if (kPrefetch > 0)
-        for (int t = 0; t < kPrefetch; ++t) prefetch(t);
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -232,7 +204,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
         int m0, n0;
         sched.coords(tile, m0, n0);
         for (int kb = 0; kb < kb_total; ++kb) {
-          if (kPrefetch > 0) prefetch(issued + kPrefetch);
           if (!mbar_wait_bounded(&S.empty[stage], phase ^ 1u, abort)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&S.full[stage], 4 * kOpBytes);  // both CTAs' A + B
           const uint32_t fb = full0 + static_cast<uint32_t>(stage * sizeof(uint64_t));
@@ -325,7 +296,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const uint32_t use = (nslots == 1) ? it : (it >> 1);
       int m0, n0;
       sched.coords(tile, m0, n0);
-      const bool landed = mbar_wait_patient(&S.tmem_full[slot], use & 1u, abort, kEpiSleepNs);
+      const bool landed = mbar_wait_bounded(&S.tmem_full[slot], use & 1u, abort);
       if (epi_any(!landed)) {  // every epilogue thread takes the same branch
         report(args.status, INT8MM_ERR_TIMEOUT);
         break;

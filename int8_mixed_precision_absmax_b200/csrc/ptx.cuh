@@ -81,27 +81,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
-// A wait for warps that have nothing else to do for a long time (an epilogue waiting for a
-// tile's accumulator): it sleeps from the first miss, `sleep_ns` between polls, so that the
-// polling does not take issue slots or barrier bandwidth from the producer and MMA threads of
-// the same SM.  Bounded like mbar_wait_bounded.
-__device__ __forceinline__ bool mbar_wait_patient(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort, uint32_t sleep_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(sleep_ns);
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 0) {
-      if (*abort) return false;
-      if (it >= kWaitIters || globaltimer_ns() - t0 > kWaitNs) {
-        *abort = 1;
-        return false;
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -116,14 +95,6 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, void* dst, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
       : "memory");
-}
-
-// Ask L2 to fetch the 2-D box at (x, y) of `map` (no shared memory, no completion signal).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
 }
 
 // 3-D tiled load into shared memory; completion is counted on `bar` in bytes.
