@@ -151,7 +151,7 @@ cudaError_t launch_quant_weight(const __half* W, int N, int K, int8_t* Wq, float
 //
 // A cluster of 8 CTAs owns a strip of 64 columns; CTA r of the cluster takes rows
 // r, r + 8, ...: thread (l, c) = (tid / 8, tid % 8) reads the 16-byte chunk c of the strip in
-// 16 of those rows at a time (all 16 loads in flight; one batch covers M <= 4096).  Each CTA reduces its column maxima
+// 8 of those rows at a time (all 8 loads in flight; one batch covers M <= 2048).  Each CTA reduces its column maxima
 // (fp16, exact) into its shared memory; after one cluster barrier CTA 0 takes the maximum over
 // the 8 CTAs through distributed shared memory and writes the strip's two mask words.  No two
 // clusters write the same word, so the mask needs no clearing.
@@ -287,34 +287,69 @@ cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint3
 }
 
 // ------------------------------------------------------------------ rows + outlier operands
+//
+// The row pass.  A block of 256 threads takes rpb rows at a time (rpb = 1, 2, 4 or 8, so that
+// a thread owns about 8 chunks of 8 columns or more) with tpr = 256 / rpb threads per row:
+// thread (row t / tpr, lane t % tpr) owns chunks lane + tpr j of its row.  It stages its own
+// chunks in shared memory with 16-byte asynchronous copies and is their only reader, so the
+// staging needs no block barrier and holds no registers; as soon as a chunk is quantized its
+// slot is refilled with the same chunk of the block's next row.  Blocks are persistent (up to
+// four per SM) and read the outlier mask and its prefix once.  Per row:
+//   1. outlier columns: their fp16 values to X_O at their compacted index, then 0 in the stage,
+//      so that the absolute maximum below is the regular columns' and their codes come out 0;
+//   2. the row's absolute maximum (fp16 maxima of the sign-cleared values, exact): shuffles,
+//      then one named barrier across the row's warps;
+//   3. codes rne(x * r) of 4 chunks at a time with packed fp32 FMAs; where x * r lies within
+//      2^-15 of a half-integer the chunk is redone with the IEEE quotient x / s (rare: the
+//      branch is taken by the warp only for a group of chunks in which some lane needs it).
+// The first row's copies go out before the wait on the column search: X is not written by that
+// kernel, and whatever wrote X had completed before the column search let this launch start.
+// Before their rows, all blocks write the fp16 outlier weights
+// W_hat[n, r] = fp16(Wq[n, col(r)] * w_scale[n]) (or the kept fp16 weight W16[n, col(r)]),
+// zero-padded to a multiple of 64, while their first rows land.
 
 constexpr int kRQThreads = 256;
-constexpr int kRQRegChunks = 8;                         // chunks of 8 halves kept per thread
-constexpr int kRQRegK = kRQThreads * 8 * kRQRegChunks;  // rows up to this length stay in registers
-constexpr int kRQMaxWords = INT8MM_MAX_K / 32;
+constexpr int kRQWarps = kRQThreads / 32;
+constexpr int kRQChunksPerThread = 8;  // rows share a block while a thread keeps this many chunks
+constexpr int kRQBlocksPerSM = 4;
+constexpr int kGatherCols = 256;       // outlier columns the weight gather lists at a time
 
-constexpr int kGatherSmemCols = 2048;  // outlier columns the weight gather lists in smem
-
-struct RowQuantShared {
-  uint32_t mask[kRQMaxWords];
-  int32_t prefix[kRQMaxWords];  // outliers in the words before this one
-  int32_t cols[kGatherSmemCols];  // the outlier columns (weight gather, n_out <= 2048)
-  int32_t warp_sum[kRQThreads / 32];
-  float red[kRQThreads / 32];
-  int32_t n_out;
+struct RowPassSmem {  // byte offsets into the dynamic shared memory
+  int words, tpr, rpb, mask, prefix, misc, red, cols, stage, total;
 };
 
-// Load the mask into shared memory and build the exclusive prefix of its popcounts.
-__device__ void load_mask_prefix(RowQuantShared& S, const uint32_t* __restrict__ mask, int words) {
+__host__ __device__ inline RowPassSmem row_pass_smem(int K) {
+  RowPassSmem L;
+  L.words = (K + 31) / 32;
+  const int chunks = K / 8;
+  int rpb = 1;
+  while (rpb < 8 && chunks * rpb * 2 <= kRQThreads * kRQChunksPerThread) rpb *= 2;
+  L.rpb = rpb;
+  L.tpr = kRQThreads / rpb;
+  const int wpad = (L.words + 3) / 4 * 4;
+  L.mask = 0;
+  L.prefix = wpad * 4;
+  L.misc = L.prefix + wpad * 4;  // int32 [0] outlier count, [8..15] per-warp sums
+  L.red = L.misc + 64;           // float [2][8] per-warp row maxima (two rows in flight)
+  L.cols = L.red + 64;           // int32 [kGatherCols]
+  L.stage = (L.cols + kGatherCols * 4 + 127) / 128 * 128;
+  L.total = L.stage + rpb * K * 2;
+  return L;
+}
+
+namespace {
+
+// Mask words into shared memory and the exclusive prefix of their popcounts; n_out = total.
+__device__ void stage_mask_prefix(const uint32_t* __restrict__ gmask, uint32_t* mask,
+                                  int32_t* prefix, int32_t* warp_sum, int32_t* n_out, int words) {
   const int per = (words + kRQThreads - 1) / kRQThreads;
   const int w0 = threadIdx.x * per;
   int local = 0;
   for (int w = w0; w < min(w0 + per, words); ++w) {
-    const uint32_t m = mask[w];
-    S.mask[w] = m;
+    const uint32_t m = gmask[w];
+    mask[w] = m;
     local += __popc(m);
   }
-  // exclusive scan of `local` over the block
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   int incl = local;
 #pragma unroll
@@ -322,173 +357,67 @@ __device__ void load_mask_prefix(RowQuantShared& S, const uint32_t* __restrict__
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
-  if (lane == 31) S.warp_sum[warp] = incl;
+  if (lane == 31) warp_sum[warp] = incl;
   __syncthreads();
   int warp_base = 0, total = 0;
 #pragma unroll
-  for (int w = 0; w < kRQThreads / 32; ++w) {
-    const int v = S.warp_sum[w];
+  for (int w = 0; w < kRQWarps; ++w) {
+    const int v = warp_sum[w];
     warp_base += (w < warp) ? v : 0;
     total += v;
   }
   int run = warp_base + incl - local;
   for (int w = w0; w < min(w0 + per, words); ++w) {
-    S.prefix[w] = run;
-    run += __popc(S.mask[w]);
+    prefix[w] = run;
+    run += __popc(mask[w]);
   }
-  if (threadIdx.x == 0) S.n_out = total;
+  if (threadIdx.x == 0) *n_out = total;
   __syncthreads();
 }
 
-// The row pass.  A block takes rpb = 256 / tpr rows (tpr = threads per row, 32..256): thread
-// (row t / tpr, lane t % tpr) holds chunks lane + u * tpr (u < 8) of its row in registers
-// (rows of up to kRQRegK columns), so the block keeps up to 32 KB of X in flight and shares
-// one mask prologue.  Longer rows (one per block) are read twice from global memory.
-
-// outlier bits (one per column) of chunk c: byte c % 4 of mask word c / 4
-__device__ __forceinline__ uint32_t chunk_bits(const RowQuantShared& S, int c) {
-  return (S.mask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-}
-
-__device__ __forceinline__ void absmax_chunk(const uint4& x, uint32_t bits, __half2& m2, float& mf) {
-  if (bits == 0) {
-    m2 = habs2_max(m2, x.x);
-    m2 = habs2_max(m2, x.y);
-    m2 = habs2_max(m2, x.z);
-    m2 = habs2_max(m2, x.w);
-  } else {
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (!((bits >> e) & 1u)) {
-        const uint32_t hb = (w[e / 2] >> (16 * (e & 1))) & 0xFFFFu;
-        mf = fmaxf(mf, fabsf(__half2float(__ushort_as_half(static_cast<unsigned short>(hb)))));
-      }
-  }
-}
-
-// the fp16 values of chunk c's outlier columns, at their places in the compacted row
-__device__ __forceinline__ void emit_outliers(const RowQuantShared& S, const uint4& x, int c,
-                                              uint32_t bits, __half* xo) {
+// The fp16 values of chunk c's outlier columns (bits), at their places in the compacted row.
+__device__ __forceinline__ void emit_outliers(const uint32_t* mask, const int32_t* prefix,
+                                              const uint4& x, int c, uint32_t bits, __half* xo) {
   const int word = c >> 2;
-  const uint32_t wm = S.mask[word];
+  const uint32_t wm = mask[word];
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
   for (int e = 0; e < 8; ++e)
     if ((bits >> e) & 1u) {
       const int bit = (c & 3) * 8 + e;
-      const int r = S.prefix[word] + __popc(wm & ((1u << bit) - 1u));
+      const int r = prefix[word] + __popc(wm & ((1u << bit) - 1u));
       const uint32_t hb = (w[e / 2] >> (16 * (e & 1))) & 0xFFFFu;
       xo[r] = __ushort_as_half(static_cast<unsigned short>(hb));
     }
 }
 
-// Row i of the block (tpr threads): absmax over the regular columns, scale, codes, outlier
-// activations.  In-register rows arrive in v.
-__device__ void quantize_rows_block(const RowQuantArgs& a, RowQuantShared& S, int tpr,
-                                    const uint4 (&v)[kRQRegChunks]) {
-  const int K = a.K;
-  const int chunks = K / 8;
-  const int rl = threadIdx.x / tpr, lr = threadIdx.x % tpr;
-  const int i = blockIdx.x * (kRQThreads / tpr) + rl;
-  const bool live = i < a.M;
-  const bool in_regs = K <= kRQRegK;
-  const uint4* row = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(live ? i : 0) * K);
-  __half2 m2 = __float2half2_rn(0.0f);
-  float mf = 0.0f;
-  uint32_t bits_r[kRQRegChunks];
-  if (in_regs) {
-#pragma unroll
-    for (int u = 0; u < kRQRegChunks; ++u) {
-      const int c = lr + u * tpr;
-      bits_r[u] = 0u;
-      if (live && c < chunks) {
-        bits_r[u] = chunk_bits(S, c);
-        absmax_chunk(v[u], bits_r[u], m2, mf);
-      }
-    }
-  } else if (live) {
-    for (int c = lr; c < chunks; c += tpr) absmax_chunk(__ldg(row + c), chunk_bits(S, c), m2, mf);
-  }
-  // maximum over the row's tpr threads: the warp, then the row's warps
-  float m = fmaxf(mf, half2_max_f(m2));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  const int warp = threadIdx.x / 32;
-  if ((threadIdx.x & 31) == 0) S.red[warp] = m;
-  __syncthreads();
-  float amax = 0.0f;
-  for (int w = rl * (tpr / 32); w < (rl + 1) * (tpr / 32); ++w) amax = fmaxf(amax, S.red[w]);
-  if (a.word_max) {  // one scale for all rows: the largest regular |x| of the whole tensor
-    const int lane = threadIdx.x & 31;
-    float g = 0.0f;
-    for (int w = lane; w < (K + 31) / 32; w += 32) g = fmaxf(g, __ldcg(a.word_max + w));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
-    amax = g;
-  }
-  if (!live) return;
-  const float s = __fdiv_rn(amax, 127.0f);
-  if (lr == 0) a.xscale[i] = s;
-  const bool zero_row = amax == 0.0f;
-  const float rcp = zero_row ? 0.0f : __frcp_rn(s);
-
-  uint2* out = reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(i) * K);
-  __half* xo = a.xo ? a.xo + static_cast<size_t>(i) * a.ldo : nullptr;
-  if (in_regs) {
-#pragma unroll
-    for (int u = 0; u < kRQRegChunks; ++u) {
-      const int c = lr + u * tpr;
-      if (c < chunks) {
-        out[c] = zero_row ? make_uint2(0u, 0u) : quantize_chunk_fast(v[u], s, rcp, bits_r[u]);
-        if (bits_r[u] != 0 && xo != nullptr) emit_outliers(S, v[u], c, bits_r[u], xo);
-      }
-    }
-  } else {
-    for (int c = lr; c < chunks; c += tpr) {
-      const uint4 x = __ldg(row + c);
-      const uint32_t bits = chunk_bits(S, c);
-      out[c] = zero_row ? make_uint2(0u, 0u) : quantize_chunk_fast(x, s, rcp, bits);
-      if (bits != 0 && xo != nullptr) emit_outliers(S, x, c, bits, xo);
-    }
-  }
-  if (xo != nullptr) {
-    const int n_out = S.n_out;
-    const int padded = (n_out + 63) / 64 * 64;
-    for (int r = n_out + lr; r < padded; r += tpr) xo[r] = __float2half_rn(0.0f);
-  }
-}
-
-// Extra blocks: W_hat[n, r] = fp16(float(Wq[n, col(r)]) * w_scale[n]), zero-padded to 64 (or
-// the kept fp16 weight W16[n, col(r)] when the layer has one).
-// The outliers are taken in windows of kGatherSmemCols: the block lists the window's columns
-// in shared memory, then thread u writes the 8 consecutive entries (one 16-byte store) of
-// channel u / groups, group u % groups of the window.
-__device__ void gather_weights(const RowQuantArgs& a, RowQuantShared& S, int words, int gb,
-                               int G) {
-  const int n_out = S.n_out;
+// Block gb of G: W_hat[n, r] for units (n, group of 8 outliers); the outliers are taken in
+// windows of kGatherCols columns listed in shared memory.
+__device__ void gather_weights(const RowQuantArgs& a, const uint32_t* mask,
+                               const int32_t* prefix, int n_out, int32_t* cols, int words,
+                               int gb, int G) {
   const int width = (n_out + 63) / 64 * 64;
-  for (int R0 = 0; R0 < width; R0 += kGatherSmemCols) {  // block-uniform
-    const int R1 = min(n_out, R0 + kGatherSmemCols);     // outliers of this window
+  for (int R0 = 0; R0 < width; R0 += kGatherCols) {  // block-uniform
+    const int R1 = min(n_out, R0 + kGatherCols);      // outliers of this window
     for (int w = threadIdx.x; w < words; w += kRQThreads) {
-      const int p0 = S.prefix[w];
-      uint32_t m = S.mask[w];
+      const int p0 = prefix[w];
+      uint32_t m = mask[w];
       if (p0 >= R1 || p0 + __popc(m) <= R0) continue;
       for (int r = p0; m; ++r, m &= m - 1)
-        if (r >= R0 && r < R1) S.cols[r - R0] = w * 32 + __ffs(m) - 1;
+        if (r >= R0 && r < R1) cols[r - R0] = w * 32 + __ffs(m) - 1;
     }
     __syncthreads();
-    const int groups = (min(width, R0 + kGatherSmemCols) - R0) / 8;
+    const int groups = (min(width, R0 + kGatherCols) - R0) / 8;  // <= 32
     const long long units = static_cast<long long>(a.N) * groups;
     for (long long u = static_cast<long long>(gb) * kRQThreads + threadIdx.x; u < units;
          u += static_cast<long long>(G) * kRQThreads) {
       const int n = static_cast<int>(u / groups);
-      const int r0 = R0 + static_cast<int>(u % groups) * 8;
+      const int r0 = R0 + static_cast<int>(u - static_cast<long long>(n) * groups) * 8;
       uint32_t h[4] = {0u, 0u, 0u, 0u};
       // eight outliers in consecutive columns from a multiple of 8 (every column, when the
       // threshold is 0): one vector load of the row instead of eight
-      const int c0 = r0 < n_out ? S.cols[r0 - R0] : 0;
-      const bool dense = r0 + 8 <= n_out && (c0 & 7) == 0 && S.cols[r0 + 7 - R0] == c0 + 7;
+      const int c0 = r0 < n_out ? cols[r0 - R0] : 0;
+      const bool dense = r0 + 8 <= n_out && (c0 & 7) == 0 && cols[r0 + 7 - R0] == c0 + 7;
       if (dense && a.W16 != nullptr) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.W16 + static_cast<size_t>(n) * a.K + c0));
         h[0] = v.x;
@@ -510,7 +439,7 @@ __device__ void gather_weights(const RowQuantArgs& a, RowQuantShared& S, int wor
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           if (r0 + e < n_out)
-            h[e / 2] |= static_cast<uint32_t>(hrow[S.cols[r0 + e - R0]]) << (16 * (e & 1));
+            h[e / 2] |= static_cast<uint32_t>(hrow[cols[r0 + e - R0]]) << (16 * (e & 1));
       } else if (r0 < n_out) {  // rebuilt from the int8 weights
         const float sc = a.w_scale[n];
         const int8_t* wrow = a.Wq + static_cast<size_t>(n) * a.K;
@@ -518,7 +447,7 @@ __device__ void gather_weights(const RowQuantArgs& a, RowQuantShared& S, int wor
         for (int e = 0; e < 8; ++e) {
           const int r = r0 + e;
           if (r < n_out) {
-            const float w = static_cast<float>(wrow[S.cols[r - R0]]) * sc;
+            const float w = static_cast<float>(wrow[cols[r - R0]]) * sc;
             h[e / 2] |= static_cast<uint32_t>(__half_as_ushort(__float2half_rn(w)))
                         << (16 * (e & 1));
           }
@@ -531,90 +460,239 @@ __device__ void gather_weights(const RowQuantArgs& a, RowQuantShared& S, int wor
   }
 }
 
-// (The row pass is capped at 64 registers, four 256-thread blocks per SM: measured 7% faster on
-// prefill up_proj than the 80 the compiler picks alone, equal on the longer rows.)
-
-// threads per row of the row pass: rows of up to 2048 / rpb chunks share a block
-__host__ __device__ inline int rowquant_tpr(int K) {
-  const int chunks = K / 8;
-  int rpb = 1;
-  while (rpb < 8 && chunks * rpb * 2 <= kRQThreads * kRQRegChunks) rpb *= 2;
-  return kRQThreads / rpb;
+// Packed fp32 (two lanes per 64-bit register; fma.rn.f32x2 rounds each lane like fmaf).
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t v, uint32_t& lo, uint32_t& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
 }
 
-__global__ void __launch_bounds__(kRQThreads, 4) rowquant_kernel(const RowQuantArgs a, int row_blocks) {
-  extern __shared__ __align__(16) uint8_t rq_smem[];
-  RowQuantShared& S = *reinterpret_cast<RowQuantShared*>(rq_smem);
-  const int words = (a.K + 31) / 32;
-  const int tpr = rowquant_tpr(a.K);
-  // The rows' loads go out before the wait on the column search: X is not written by that
-  // kernel, and whatever wrote X was complete before the column search (which waited for it)
-  // let this launch start.
-  const bool row_block = static_cast<int>(blockIdx.x) < row_blocks;
-  const int chunks = a.K / 8;
-  uint4 v[kRQRegChunks];
-  if (row_block && a.K <= kRQRegK) {
-    const int i = blockIdx.x * (kRQThreads / tpr) + threadIdx.x / tpr, lr = threadIdx.x % tpr;
-    const uint4* row = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * a.K);
+// Codes rne(x * r) of 8 halves, packed little-endian (the quantize_chunk_fast arithmetic, two
+// lanes per FMA); near = some |x * r - rne(x * r)| > 1/2 - 2^-15, where the caller must take
+// the IEEE quotient instead.
+__device__ __forceinline__ uint2 codes8_fast(const uint4& v, float rcp, bool& near) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kNear = 0.5f - 0x1p-15f;
+  const uint64_t r2 = f32x2_pack(rcp, rcp), k2 = f32x2_pack(kRound, kRound),
+                 m2 = f32x2_pack(-1.0f, -1.0f);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t qb[8];
+  bool nt = false;
 #pragma unroll
-    for (int u = 0; u < kRQRegChunks; ++u) {
-      const int c = lr + u * tpr;
-      v[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (i < a.M && c < chunks) v[u] = __ldg(row + c);
-    }
+  for (int p = 0; p < 4; ++p) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[p]));
+    const uint64_t x2 = f32x2_pack(f.x, f.y);
+    const uint64_t tb = f32x2_fma(x2, r2, k2);  // 1.5 * 2^23 + rne(x r), exactly
+    const uint64_t rn = f32x2_fma(tb, m2, k2);  // -rne(x r), exactly
+    const uint64_t d = f32x2_fma(x2, r2, rn);   // x r - rne(x r)
+    uint32_t d0, d1;
+    f32x2_unpack(d, d0, d1);
+    f32x2_unpack(tb, qb[2 * p], qb[2 * p + 1]);
+    nt |= fabsf(__uint_as_float(d0)) > kNear;
+    nt |= fabsf(__uint_as_float(d1)) > kNear;
   }
+  near = nt;
+  const uint32_t lo = __byte_perm(__byte_perm(qb[0], qb[1], 0x0040), __byte_perm(qb[2], qb[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(qb[4], qb[5], 0x0040), __byte_perm(qb[6], qb[7], 0x0040), 0x5410);
+  return make_uint2(lo, hi);
+}
+
+// The same codes with the IEEE quotient where it is needed (out of line: rarely called).
+__device__ __noinline__ uint2 codes8_exact(uint4 v, float s, float rcp) {
+  return quantize_chunk_fast(v, s, rcp, 0u);
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kRQThreads, kRQBlocksPerSM) rowquant_kernel(const RowQuantArgs a) {
+  extern __shared__ __align__(128) uint8_t rq_smem[];
+  const RowPassSmem L = row_pass_smem(a.K);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(rq_smem + L.mask);
+  int32_t* prefix = reinterpret_cast<int32_t*>(rq_smem + L.prefix);
+  int32_t* misc = reinterpret_cast<int32_t*>(rq_smem + L.misc);
+  float* red = reinterpret_cast<float*>(rq_smem + L.red);
+  const int K = a.K, M = a.M, chunks = K / 8, tpr = L.tpr, rpb = L.rpb;
+  const int rl = threadIdx.x / tpr, lr = threadIdx.x % tpr;
+  uint4* stage = reinterpret_cast<uint4*>(rq_smem + L.stage) + static_cast<size_t>(rl) * chunks;
+  const int step = gridDim.x * rpb;  // rows between a block's consecutive row groups
+  int i = blockIdx.x * rpb + rl;
+  if (i < M) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * K);
+    for (int c = lr; c < chunks; c += tpr) cp_async16(stage + c, src + c);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
   grid_dependency_wait();  // the outlier mask is complete from here on
-  load_mask_prefix(S, a.mask, words);
+  stage_mask_prefix(a.mask, mask, prefix, misc + 8, misc, L.words);
   grid_launch_dependents();
+  const int n_out = misc[0];
   if (blockIdx.x == 0) {
-    for (int w = threadIdx.x; w < words; w += kRQThreads) {
-      uint32_t m = S.mask[w];
-      int r = S.prefix[w];
+    for (int w = threadIdx.x; w < L.words; w += kRQThreads) {
+      uint32_t m = mask[w];
+      int r = prefix[w];
       while (m) {
-        const int b = __ffs(m) - 1;
-        a.cols[r++] = w * 32 + b;
+        a.cols[r++] = w * 32 + __ffs(m) - 1;
         m &= m - 1;
       }
     }
-    if (threadIdx.x == 0) *a.n_out = S.n_out;
+    if (threadIdx.x == 0) *a.n_out = n_out;
   }
-  if (row_block) {
-    quantize_rows_block(a, S, tpr, v);
-  } else if (a.wo != nullptr) {
-    gather_weights(a, S, words, blockIdx.x - row_blocks, gridDim.x - row_blocks);
+  if (a.wo != nullptr)
+    gather_weights(a, mask, prefix, n_out, reinterpret_cast<int32_t*>(rq_smem + L.cols), L.words,
+                   blockIdx.x, gridDim.x);
+  float tensor_max = -1.0f;  // one scale for all rows: the largest regular |x| of the tensor
+  if (a.word_max) {
+    float g = 0.0f;
+    for (int w = threadIdx.x % 32; w < L.words; w += 32) g = fmaxf(g, __ldcg(a.word_max + w));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
+    tensor_max = g;
+  }
+  const uint8_t* bits_of = reinterpret_cast<const uint8_t*>(mask);  // byte c: chunk c's outliers
+  const int warp = threadIdx.x / 32, wpr = tpr / 32;                // warps per row
+  // every thread of the block takes the same number of steps (rows past M idle)
+  for (int it = 0; blockIdx.x * rpb + it * step < M; ++it) {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    const bool live = i < M;
+    __half* xo = (a.xo && live) ? a.xo + static_cast<size_t>(i) * a.ldo : nullptr;
+    __half2 h0 = __float2half2_rn(0.0f), h1 = h0, h2 = h0, h3 = h0;
+    if (live) {
+#pragma unroll 4
+      for (int c = lr; c < chunks; c += tpr) {
+        uint4 x = stage[c];
+        const uint32_t bits = bits_of[c];
+        if (bits) {
+          if (xo) emit_outliers(mask, prefix, x, c, bits, xo);
+          uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if ((bits >> e) & 1u) w[e / 2] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+          x = make_uint4(w[0], w[1], w[2], w[3]);
+          stage[c] = x;
+        }
+        uint32_t b0 = x.x & 0x7FFF7FFFu, b1 = x.y & 0x7FFF7FFFu, b2 = x.z & 0x7FFF7FFFu,
+                 b3 = x.w & 0x7FFF7FFFu;
+        h0 = __hmax2(h0, *reinterpret_cast<const __half2*>(&b0));
+        h1 = __hmax2(h1, *reinterpret_cast<const __half2*>(&b1));
+        h2 = __hmax2(h2, *reinterpret_cast<const __half2*>(&b2));
+        h3 = __hmax2(h3, *reinterpret_cast<const __half2*>(&b3));
+      }
+      if (xo != nullptr) {
+        const int padded = (n_out + 63) / 64 * 64;
+        for (int r = n_out + lr; r < padded; r += tpr) xo[r] = __float2half_rn(0.0f);
+      }
+    }
+    float amax = half2_max_f(__hmax2(__hmax2(h0, h1), __hmax2(h2, h3)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (wpr > 1) {  // across the row's warps; two buffers, as a warp may be one row ahead
+      float* rd = red + (it & 1) * kRQWarps;
+      if ((threadIdx.x & 31) == 0) rd[warp] = amax;
+      named_barrier(1 + rl, tpr);
+      for (int w = rl * wpr; w < (rl + 1) * wpr; ++w) amax = fmaxf(amax, rd[w]);
+    }
+    if (tensor_max >= 0.0f) amax = tensor_max;
+    const int nx = i + step;
+    if (live) {
+      const float s = __fdiv_rn(amax, 127.0f);
+      if (lr == 0) a.xscale[i] = s;
+      const float rcp = amax == 0.0f ? 0.0f : __frcp_rn(s);
+      uint2* out = reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(i) * K);
+      const bool refill = nx < M;
+      const uint4* next = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(refill ? nx : i) * K);
+      for (int c0 = lr; c0 < chunks; c0 += 4 * tpr) {
+        uint4 x[4];
+        uint2 q[4];
+        bool near[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + tpr * u;
+          x[u] = c < chunks ? stage[c] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) q[u] = codes8_fast(x[u], rcp, near[u]);
+        if (near[0] | near[1] | near[2] | near[3]) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (near[u]) q[u] = codes8_exact(x[u], s, rcp);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + tpr * u;
+          if (c < chunks) {
+            out[c] = q[u];
+            if (refill) cp_async16(stage + c, next + c);  // x[u] is in registers
+          }
+        }
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    i = nx;
   }
 }
 
 cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl) {
-  static bool configured = false;
-  const int smem = static_cast<int>(sizeof(RowQuantShared));
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(rowquant_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // per device: shared memory of an SM, reserved per block, and the opt-in set on the kernel
+  constexpr int kMaxDevices = 64;
+  static int smem_per_sm[kMaxDevices] = {}, reserved[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (smem_per_sm[dev] == 0) {
+    int optin = 0, res = 0, per_sm_bytes = 0;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&res, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    if (e == cudaSuccess)
+      e = cudaDeviceGetAttribute(&per_sm_bytes, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(rowquant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e != cudaSuccess) return e;
-    configured = true;
+    reserved[dev] = res;
+    smem_per_sm[dev] = per_sm_bytes;
   }
-  int gather_blocks = 0;
-  if (a.wo != nullptr) {
-    const long long worst_units = static_cast<long long>(a.N) * (a.ldo / 8);
-    const long long want = (worst_units + kRQThreads - 1) / kRQThreads;
+  const RowPassSmem L = row_pass_smem(a.K);
+  int per_sm = smem_per_sm[dev] / (L.total + reserved[dev]);
+  if (per_sm > kRQBlocksPerSM) per_sm = kRQBlocksPerSM;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  long long want = (a.M + L.rpb - 1) / L.rpb;
+  if (a.wo != nullptr) {  // enough blocks for the weight gather (worst case: every column)
+    const long long units = static_cast<long long>(a.N) * (a.ldo / 8);
+    const long long gather = (units + kRQThreads - 1) / kRQThreads;
     const long long cap = 2LL * device_sm_count();
-    gather_blocks = static_cast<int>(want < cap ? want : cap);
-    if (gather_blocks < 1) gather_blocks = 1;
+    const long long g = gather < cap ? gather : cap;
+    if (g > want) want = g;
   }
-  const int rpb = kRQThreads / rowquant_tpr(a.K);
-  const int row_blocks = (a.M + rpb - 1) / rpb;
+  const long long resident = static_cast<long long>(per_sm) * device_sm_count();
+  const int blocks = static_cast<int>(want < resident ? want : resident);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(row_blocks + gather_blocks);
+  cfg.gridDim = dim3(blocks);
   cfg.blockDim = dim3(kRQThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = L.total;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, rowquant_kernel, a, row_blocks);
+  return cudaLaunchKernelEx(&cfg, rowquant_kernel, a);
 }
 
 // ------------------------------------------------------------------ diagnostic: W_hat alone
