@@ -10,9 +10,10 @@
 //                        row blocks, fp16(Wq*w_scale) weights by extra blocks)
 //                        [P5] item 2 and item 3; [P2] section 2.3
 //
-// Quantization arithmetic: scale = absmax / 127 and q = x / scale are IEEE float32
-// divisions (__fdiv_rn), q is rounded to nearest with ties to even (__float2int_rn) and
-// clamped to [-127, 127].  Absolute maxima are taken on the binary16 values (exact).
+// Quantization arithmetic: scale = absmax / 127 and q = x / scale are IEEE float32 quotients
+// (__fdiv_rn; in the row pass the quotient comes from one correction of x * RN(1/scale), equal
+// to it), q is rounded to nearest with ties to even and lies in [-127, 127].  Absolute maxima
+// are taken on the binary16 values (exact).
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -46,53 +47,6 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
-}
-
-// 8 halves -> 8 int8 codes q = rne(x / s) of a row whose regular columns satisfy
-// |x| <= absmax = 127 s, packed little-endian, outlier columns (bits) set to 0.
-// With r = 1/s rounded to nearest, the exact x * r is within 2^-17 of x / s (|x / s| <= 128)
-// and the rounded quotient within 2^-18, so rne(x * r) = rne(fl(x / s)) unless x * r lies
-// within 2^-15 of a half-integer; there the quotient itself (__fdiv_rn) is rounded.
-// tb = fl(x * r + 1.5 * 2^23) = 1.5 * 2^23 + rne(x * r) exactly, and as 1.5 * 2^23 has a zero
-// low byte, the low byte of tb's bits is the two's-complement code.  d = x * r - rne(x * r)
-// (one more FMA, rounding error <= 2^-25) has |d| <= 1/2, so "near a half-integer" is
-// |d| > 1/2 - 2^-15.  |x / s| <= 127 (1 + 2^-22) on regular columns: no clamp is needed.
-__device__ __forceinline__ uint32_t keep_mask(uint32_t bits4) {  // bit e set -> byte e = 0
-  return ~(((bits4 * 0x204081u) & 0x01010101u) * 0xFFu);
-}
-__device__ __forceinline__ uint2 quantize_chunk_fast(const uint4& v, float s, float rcp,
-                                                     uint32_t bits) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float kNear = 0.5f - 0x1p-15f;
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float x[8];
-  uint32_t qb[8];
-  bool near_tie = false;
-#pragma unroll
-  for (int e = 0; e < 8; e += 2) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e / 2]));
-    x[e] = f.x;
-    x[e + 1] = f.y;
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float tb = __fmaf_rn(x[e], rcp, kRound);
-    qb[e] = __float_as_uint(tb);
-    const float d = __fmaf_rn(x[e], rcp, -(tb - kRound));
-    near_tie |= fabsf(d) > kNear && !((bits >> e) & 1u);
-  }
-  if (near_tie) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float tb = __fmaf_rn(x[e], rcp, kRound);
-      const float d = __fmaf_rn(x[e], rcp, -(tb - kRound));
-      if (fabsf(d) > kNear && !((bits >> e) & 1u))
-        qb[e] = static_cast<uint32_t>(__float2int_rn(__fdiv_rn(x[e], s)));
-    }
-  }
-  const uint32_t lo = __byte_perm(__byte_perm(qb[0], qb[1], 0x0040), __byte_perm(qb[2], qb[3], 0x0040), 0x5410);
-  const uint32_t hi = __byte_perm(__byte_perm(qb[4], qb[5], 0x0040), __byte_perm(qb[6], qb[7], 0x0040), 0x5410);
-  return make_uint2(lo & keep_mask(bits & 0xFu), hi & keep_mask(bits >> 4));
 }
 
 // 8 halves (one 16-byte chunk) -> 8 int8 codes packed little-endian into 8 bytes.
@@ -299,9 +253,7 @@ cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint3
 //      so that the absolute maximum below is the regular columns' and their codes come out 0;
 //   2. the row's absolute maximum (fp16 maxima of the sign-cleared values, exact): shuffles,
 //      then one named barrier across the row's warps;
-//   3. codes rne(x * r) of 4 chunks at a time with packed fp32 FMAs; where x * r lies within
-//      2^-15 of a half-integer the chunk is redone with the IEEE quotient x / s (rare: the
-//      branch is taken by the warp only for a group of chunks in which some lane needs it).
+//   3. codes rne(x / s), the IEEE quotient from packed fp32 FMAs (codes8, no branch).
 // The first row's copies go out before the wait on the column search: X is not written by that
 // kernel, and whatever wrote X had completed before the column search let this launch start.
 // Before their rows, all blocks write the fp16 outlier weights
@@ -474,40 +426,45 @@ __device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 
-// Codes rne(x * r) of 8 halves, packed little-endian (the quantize_chunk_fast arithmetic, two
-// lanes per FMA); near = some |x * r - rne(x * r)| > 1/2 - 2^-15, where the caller must take
-// the IEEE quotient instead.
-__device__ __forceinline__ uint2 codes8_fast(const uint4& v, float rcp, bool& near) {
+// Codes rne(RN(x / s)) of 8 halves, packed little-endian (two lanes per packed operation).  The
+// IEEE quotient comes from one correction of x * r (r = RN(1 / s)), the method of P. Markstein
+// (IBM J. Res. Dev. 34(1), 1990; also his "IA-64 and Elementary Functions", 2000):
+// q0 = RN(x r), rho = x - q0 s (exact: one FMA), q1 = RN(q0 + rho r) = RN(x / s).  On this
+// pass's domain (x and absmax binary16, |x| <= absmax, s = RN(absmax / 127)) that equality was
+// checked for every pair (about 5 * 10^8, positive x; the steps are odd in x), and the GPU tests
+// check the codes through this pass against the oracle over every binade of absmax.
+// 1.5 * 2^23 + q1 rounded to an integer (ties to even) then holds rne(q1) in its low byte, in
+// two's complement.  |q1| <= 127 on regular columns, so no clamp is needed; s = 0 (a row whose
+// regular columns are all 0) gives r = 0 and code 0.
+__device__ __forceinline__ uint2 codes8(const uint4& v, float s, float rcp) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float kNear = 0.5f - 0x1p-15f;
-  const uint64_t r2 = f32x2_pack(rcp, rcp), k2 = f32x2_pack(kRound, kRound),
-                 m2 = f32x2_pack(-1.0f, -1.0f);
+  const uint64_t r2 = f32x2_pack(rcp, rcp), ns2 = f32x2_pack(-s, -s),
+                 k2 = f32x2_pack(kRound, kRound);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t qb[8];
-  bool nt = false;
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[p]));
     const uint64_t x2 = f32x2_pack(f.x, f.y);
-    const uint64_t tb = f32x2_fma(x2, r2, k2);  // 1.5 * 2^23 + rne(x r), exactly
-    const uint64_t rn = f32x2_fma(tb, m2, k2);  // -rne(x r), exactly
-    const uint64_t d = f32x2_fma(x2, r2, rn);   // x r - rne(x r)
-    uint32_t d0, d1;
-    f32x2_unpack(d, d0, d1);
-    f32x2_unpack(tb, qb[2 * p], qb[2 * p + 1]);
-    nt |= fabsf(__uint_as_float(d0)) > kNear;
-    nt |= fabsf(__uint_as_float(d1)) > kNear;
+    const uint64_t q0 = f32x2_mul(x2, r2);
+    const uint64_t rho = f32x2_fma(q0, ns2, x2);
+    const uint64_t q1 = f32x2_fma(rho, r2, q0);
+    f32x2_unpack(f32x2_add(q1, k2), qb[2 * p], qb[2 * p + 1]);
   }
-  near = nt;
   const uint32_t lo = __byte_perm(__byte_perm(qb[0], qb[1], 0x0040), __byte_perm(qb[2], qb[3], 0x0040), 0x5410);
   const uint32_t hi = __byte_perm(__byte_perm(qb[4], qb[5], 0x0040), __byte_perm(qb[6], qb[7], 0x0040), 0x5410);
   return make_uint2(lo, hi);
-}
-
-// The same codes with the IEEE quotient where it is needed (out of line: rarely called).
-__device__ __noinline__ uint2 codes8_exact(uint4 v, float s, float rcp) {
-  return quantize_chunk_fast(v, s, rcp, 0u);
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -617,30 +574,10 @@ __global__ void __launch_bounds__(kRQThreads, kRQBlocksPerSM) rowquant_kernel(co
       uint2* out = reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(i) * K);
       const bool refill = nx < M;
       const uint4* next = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(refill ? nx : i) * K);
-      for (int c0 = lr; c0 < chunks; c0 += 4 * tpr) {
-        uint4 x[4];
-        uint2 q[4];
-        bool near[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int c = c0 + tpr * u;
-          x[u] = c < chunks ? stage[c] : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) q[u] = codes8_fast(x[u], rcp, near[u]);
-        if (near[0] | near[1] | near[2] | near[3]) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (near[u]) q[u] = codes8_exact(x[u], s, rcp);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int c = c0 + tpr * u;
-          if (c < chunks) {
-            out[c] = q[u];
-            if (refill) cp_async16(stage + c, next + c);  // x[u] is in registers
-          }
-        }
+#pragma unroll 4
+      for (int c = lr; c < chunks; c += tpr) {
+        out[c] = codes8(stage[c], s, rcp);
+        if (refill) cp_async16(stage + c, next + c);  // the chunk is in registers
       }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
