@@ -111,9 +111,9 @@ def load_peaks():
 
 
 # the sources each timed kernel is built from (its own file and the shared headers)
-KERNEL_SOURCES = {"decode_kernel": "decode.cu", "gemm_kernel": "gemm.cu",
-                  "rowquant_kernel": "quant.cu", "colmask_kernel": "quant.cu",
-                  "gemv_kernel": "gemv.cu", "small_fused_kernel": "small.cu"}
+KERNEL_SOURCES = {"decode_kernel": ["decode.cu", "codes.cuh"], "gemm_kernel": ["gemm.cu"],
+                  "rowquant_kernel": ["quant.cu", "codes.cuh"], "colmask_kernel": ["quant.cu", "codes.cuh"],
+                  "gemv_kernel": ["gemv.cu", "codes.cuh"], "small_fused_kernel": ["small.cu", "codes.cuh"]}
 
 
 def kernel_source_hash(kernel: str | None = None) -> str:
@@ -121,7 +121,7 @@ def kernel_source_hash(kernel: str | None = None) -> str:
     h = hashlib.sha256()
     names = sorted(n for n in os.listdir(CSRC) if n.endswith((".cu", ".cuh")))
     if kernel in KERNEL_SOURCES:
-        names = sorted([KERNEL_SOURCES[kernel], "kernels.cuh", "ptx.cuh"])
+        names = sorted(KERNEL_SOURCES[kernel] + ["kernels.cuh", "ptx.cuh"])
     for name in names:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())

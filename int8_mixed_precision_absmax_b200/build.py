@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libint8mm.so")
 SOURCES = ["api.cu", "quant.cu", "gemm.cu", "gemm2.cu", "small.cu", "gemv.cu", "decode.cu", "stats.cu", "trace.cu"]
-HEADERS = ["kernels.cuh", "ptx.cuh"]
+HEADERS = ["codes.cuh", "kernels.cuh", "ptx.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

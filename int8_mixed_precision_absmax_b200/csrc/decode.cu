@@ -38,6 +38,7 @@
 //
 // Wq is read before the wait on the previous launch (everything else after it): it must not
 // be written by the launch just before this one on the stream while that can still be running.
+#include "codes.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -67,50 +68,11 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
 }
 
 // 8 codes of one row chunk, packed little-endian, then ANDed with `keep` (zero bytes in outlier
-// columns).  rne(x * r) with r = 1/sx rounded to nearest equals rne(fl(x / sx)) unless x * r
-// lies within 2^-15 of a half-integer (the exact x * r is within 2^-17 of x / sx for
-// |x / sx| <= 128, the rounded quotient within 2^-18); there the quotient itself (__fdiv_rn)
-// is rounded.  tb = fl(x * r + 1.5 * 2^23) = 1.5 * 2^23 + rne(x * r) exactly, and as
-// 1.5 * 2^23 has a zero low byte, the low byte of tb's bits is the two's-complement code.
-// d = x * r - rne(x * r) (one more FMA, rounding error <= 2^-25) has |d| <= 1/2, so "near a
-// half-integer" is |d| > 1/2 - 2^-15, tested once for the 8 values through max |d|.  A
-// regular column has |x| <= the row maximum, so |x / sx| <= 127 (1 + 2^-22) and the code needs
-// no clamp; an outlier column may take the exact route needlessly, and its code is masked.
-__device__ __forceinline__ uint2 keep_masks(uint32_t bits) {  // bit e set -> byte e = 0
-  const uint32_t lo = ~((((bits & 0xFu) * 0x204081u) & 0x01010101u) * 0xFFu);
-  const uint32_t hi = ~((((bits >> 4) * 0x204081u) & 0x01010101u) * 0xFFu);
-  return make_uint2(lo, hi);
-}
+// columns): the IEEE quotient's codes (codes.cuh).
+__device__ __forceinline__ uint2 keep_masks(uint32_t bits) { return keep_bytes(bits); }
 __device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, uint2 keep) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float kNear = 0.5f - 0x1p-15f;
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float x[8];
-  uint32_t qb[8];
-  float dmax = 0.0f;
-#pragma unroll
-  for (int e = 0; e < 8; e += 2) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e / 2]));
-    x[e] = f.x;
-    x[e + 1] = f.y;
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float tb = __fmaf_rn(x[e], rcp, kRound);
-    qb[e] = __float_as_uint(tb);
-    dmax = fmaxf(dmax, fabsf(__fmaf_rn(x[e], rcp, -(tb - kRound))));
-  }
-  if (dmax > kNear) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float tb = __fmaf_rn(x[e], rcp, kRound);
-      if (fabsf(__fmaf_rn(x[e], rcp, -(tb - kRound))) > kNear)
-        qb[e] = static_cast<uint32_t>(__float2int_rn(__fdiv_rn(x[e], sc)));
-    }
-  }
-  const uint32_t lo = __byte_perm(__byte_perm(qb[0], qb[1], 0x0040), __byte_perm(qb[2], qb[3], 0x0040), 0x5410);
-  const uint32_t hi = __byte_perm(__byte_perm(qb[4], qb[5], 0x0040), __byte_perm(qb[6], qb[7], 0x0040), 0x5410);
-  return make_uint2(lo & keep.x, hi & keep.y);
+  const uint2 q = codes8(v, sc, rcp);
+  return make_uint2(q.x & keep.x, q.y & keep.y);
 }
 
 // D(16 x 8, int32) += A(16 x 32, int8, row-major) * B(32 x 8, int8, column-major)

@@ -27,11 +27,8 @@
 //                     2.9 中启用 LLM.int8 推理": no fp16 weights are kept) comes from the
 //                     compact list, and Y = fp16(acc * sx * w_scale + P + bias).
 //
-// Quantization arithmetic, exact to the IEEE quotient.  With r = 1/sx rounded to nearest,
-// the exact product x*r is within 2^-17 of x/sx (|x/sx| <= 128) and the rounded quotient
-// fl(x/sx) within 2^-18, so rne(x*r) = rne(fl(x/sx)) unless x*r lies within 2^-15 of a
-// half-integer, where the quotient itself (__fdiv_rn) is rounded.  rne(x*r) is formed by one
-// fused multiply-add with 1.5*2^23, whose bits hold the integer.
+// Quantization arithmetic: the codes of the IEEE quotient x / sx (codes.cuh).
+#include "codes.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -84,34 +81,11 @@ __device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
   return v;
 }
 
-// 8 codes of one row chunk, packed little-endian (see the file comment for exactness)
+// 8 codes of one row chunk, packed little-endian, outlier columns (bits) 0 (codes.cuh)
 __device__ __forceinline__ uint2 quantize8(const uint4& v, float sc, float rcp, uint32_t bits) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float x[8];
-  int qv[8];
-  uint32_t near_tie = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    x[e] = h2f(w[e / 2], e & 1);
-    const float tb = __fmaf_rn(x[e], rcp, kRound);      // rne(x*r) + 1.5*2^23, exactly
-    qv[e] = __float_as_int(tb) - 0x4B400000;              // the integer rne(x*r)
-    const float d = fabsf(__fmaf_rn(x[e], rcp, -(tb - kRound)));  // |x*r - rne(x*r)|
-    near_tie |= (fabsf(d - 0.5f) <= 0x1p-15f ? 1u : 0u) << e;
-  }
-  if (near_tie) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if ((near_tie >> e) & 1u) qv[e] = __float2int_rn(__fdiv_rn(x[e], sc));
-  }
-  uint32_t p[2] = {0u, 0u};
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int qc = max(-127, min(127, qv[e]));
-    const uint32_t code = ((bits >> e) & 1u) ? 0u : (static_cast<uint32_t>(qc) & 0xFFu);
-    p[e / 4] |= code << (8 * (e & 3));
-  }
-  return make_uint2(p[0], p[1]);
+  const uint2 q = codes8(v, sc, rcp);
+  const uint2 keep = keep_bytes(bits);
+  return make_uint2(q.x & keep.x, q.y & keep.y);
 }
 
 // D(16 x 8, int32) += A(16 x 32, int8, row-major) * B(32 x 8, int8, column-major)

@@ -14,6 +14,7 @@
 // (__fdiv_rn; in the row pass the quotient comes from one correction of x * RN(1/scale), equal
 // to it), q is rounded to nearest with ties to even and lies in [-127, 127].  Absolute maxima
 // are taken on the binary16 values (exact).
+#include "codes.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -253,7 +254,7 @@ cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint3
 //      so that the absolute maximum below is the regular columns' and their codes come out 0;
 //   2. the row's absolute maximum (fp16 maxima of the sign-cleared values, exact): shuffles,
 //      then one named barrier across the row's warps;
-//   3. codes rne(x / s), the IEEE quotient from packed fp32 FMAs (codes8, no branch).
+//   3. codes rne(x / s), the IEEE quotient from packed fp32 FMAs (codes8 in codes.cuh).
 // The first row's copies go out before the wait on the column search: X is not written by that
 // kernel, and whatever wrote X had completed before the column search let this launch start.
 // Before their rows, all blocks write the fp16 outlier weights
@@ -410,61 +411,6 @@ __device__ void gather_weights(const RowQuantArgs& a, const uint32_t* mask,
     }
     __syncthreads();  // the list is rewritten for the next window
   }
-}
-
-// Packed fp32 (two lanes per 64-bit register; fma.rn.f32x2 rounds each lane like fmaf).
-__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
-  uint64_t d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-  return d;
-}
-__device__ __forceinline__ void f32x2_unpack(uint64_t v, uint32_t& lo, uint32_t& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-// Codes rne(RN(x / s)) of 8 halves, packed little-endian (two lanes per packed operation).  The
-// IEEE quotient comes from one correction of x * r (r = RN(1 / s)), the method of P. Markstein
-// (IBM J. Res. Dev. 34(1), 1990; also his "IA-64 and Elementary Functions", 2000):
-// q0 = RN(x r), rho = x - q0 s (exact: one FMA), q1 = RN(q0 + rho r) = RN(x / s).  On this
-// pass's domain (x and absmax binary16, |x| <= absmax, s = RN(absmax / 127)) that equality was
-// checked for every pair (about 5 * 10^8, positive x; the steps are odd in x), and the GPU tests
-// check the codes through this pass against the oracle over every binade of absmax.
-// 1.5 * 2^23 + q1 rounded to an integer (ties to even) then holds rne(q1) in its low byte, in
-// two's complement.  |q1| <= 127 on regular columns, so no clamp is needed; s = 0 (a row whose
-// regular columns are all 0) gives r = 0 and code 0.
-__device__ __forceinline__ uint2 codes8(const uint4& v, float s, float rcp) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t r2 = f32x2_pack(rcp, rcp), ns2 = f32x2_pack(-s, -s),
-                 k2 = f32x2_pack(kRound, kRound);
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t qb[8];
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[p]));
-    const uint64_t x2 = f32x2_pack(f.x, f.y);
-    const uint64_t q0 = f32x2_mul(x2, r2);
-    const uint64_t rho = f32x2_fma(q0, ns2, x2);
-    const uint64_t q1 = f32x2_fma(rho, r2, q0);
-    f32x2_unpack(f32x2_add(q1, k2), qb[2 * p], qb[2 * p + 1]);
-  }
-  const uint32_t lo = __byte_perm(__byte_perm(qb[0], qb[1], 0x0040), __byte_perm(qb[2], qb[3], 0x0040), 0x5410);
-  const uint32_t hi = __byte_perm(__byte_perm(qb[4], qb[5], 0x0040), __byte_perm(qb[6], qb[7], 0x0040), 0x5410);
-  return make_uint2(lo, hi);
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {

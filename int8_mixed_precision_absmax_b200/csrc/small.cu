@@ -27,10 +27,8 @@
 // No CTA waits on another except through the cluster's hardware barrier; the kernel keeps
 // no state in global memory between calls.
 //
-// Quantization arithmetic, exact to the IEEE quotient: v = x * r with r = 1/sx rounded to
-// nearest is within 2^-16 of x/sx (for |x/sx| <= 127), and the rounded quotient fl(x/sx) is
-// within 2^-18 of it, so round-to-nearest-even of v equals that of fl(x/sx) unless v lies
-// within 2^-15 of a half-integer; there the quotient itself (__fdiv_rn) is rounded.
+// Quantization arithmetic: the codes of the IEEE quotient x / sx (codes.cuh).
+#include "codes.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -416,32 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!sh.zero_row[i]) {
             const uint4 v =
                 *reinterpret_cast<const uint4*>(x_slice + static_cast<size_t>(i) * xs_ld + c * 8);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            const float sc = sh.sx[i], r = sh.rcp[i];
-            float x[8];
-            int qv[8];
-            uint32_t near_tie = 0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {  // 8 independent elements: no branch inside
-              x[e] = half_bits_to_float(w[e / 2], e & 1);
-              const float t = x[e] * r;
-              qv[e] = __float2int_rn(t);
-              const float d = fabsf(t - rintf(t));
-              near_tie |= (fabsf(d - 0.5f) <= 0x1p-15f ? 1u : 0u) << e;
-            }
-            if (near_tie) {  // rare: round the IEEE quotient itself
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                if ((near_tie >> e) & 1u) qv[e] = __float2int_rn(__fdiv_rn(x[e], sc));
-            }
-            uint32_t p[2] = {0u, 0u};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int qc = max(-127, min(127, qv[e]));
-              const uint32_t code = ((bits >> e) & 1u) ? 0u : (static_cast<uint32_t>(qc) & 0xFFu);
-              p[e / 4] |= code << (8 * (e & 3));
-            }
-            q = make_uint2(p[0], p[1]);
+            const uint2 c8 = codes8(v, sh.sx[i], sh.rcp[i]);
+            const uint2 keep = keep_bytes(bits);
+            q = make_uint2(c8.x & keep.x, c8.y & keep.y);
           }
           *reinterpret_cast<uint2*>(tile + (i / 8) * 1024 + (i % 8) * 128 +
                                     (((kk / 16) ^ (i % 8)) * 16)) = q;

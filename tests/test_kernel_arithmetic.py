@@ -7,14 +7,14 @@ LLM.int8()" section "LLM.int8() 是怎么做到几乎无损的", item 2: q = rou
 scale = absmax / 127; [P2] "8位量化实战：离群值处理与显存优化避坑指南" section 2.3: a column
 is an outlier when |x| exceeds the threshold):
 
-* the quantizer (quant.cu quantize_chunk_fast, decode.cu quantize8): q = rne(x * r) with
-  r = 1 / s rounded to nearest, read off the low byte of fl(x * r + 1.5 * 2^23), and the IEEE
-  quotient x / s only where x * r lies within 2^-15 of a half-integer;
+* the quantizer (codes.cuh codes8, used by every kernel): the IEEE quotient x / s from one
+  correction of x * r, r = 1 / s rounded to nearest (P. Markstein's method: q0 = RN(x r),
+  rho = x - q0 s exactly, q1 = RN(q0 + rho r)), the code read off the low byte of
+  fl(q1 + 1.5 * 2^23);
 * the threshold test on binary16 values against the threshold rounded down to binary16
   (decode.cu);
 * int8 codes to float through the bit pattern 0x4B0000vv (decode.cu code_to_float);
-* the byte masks that zero the codes of outlier columns (quant.cu keep_mask, decode.cu
-  keep_masks).
+* the byte masks that zero the codes of outlier columns (codes.cuh keep_bytes).
 
 None of this imports the CUDA library or the oracle.
 """
@@ -23,7 +23,6 @@ import pytest
 
 F16_POS = np.arange(0x0000, 0x7C00, dtype=np.uint16).view(np.float16)  # 0 and every finite > 0
 MAGIC = np.float32(12582912.0)  # 1.5 * 2^23
-NEAR = 0.5 - 2.0 ** -15
 
 
 def _absmax_sample(n_random: int, seed: int) -> np.ndarray:
@@ -37,36 +36,63 @@ def _absmax_sample(n_random: int, seed: int) -> np.ndarray:
     return np.array(sorted(bits), dtype=np.uint16).view(np.float16)
 
 
+def _round_to_f32(hi: np.ndarray, lo: np.ndarray) -> np.ndarray:
+    """RN to float32 of the exact sum hi + lo (float64, |lo| <= ulp(hi) / 2, from a two-sum)."""
+    f = hi.astype(np.float32)
+    f64 = f.astype(np.float64)
+    up = np.nextafter(f, np.float32(np.inf)).astype(np.float64)
+    down = np.nextafter(f, np.float32(-np.inf)).astype(np.float64)
+    # hi exactly halfway between f and a neighbour: the sign of lo decides (lo = 0: ties to even)
+    at_mid_up = (hi > f64) & (hi == (f64 + up) / 2)
+    at_mid_down = (hi < f64) & (hi == (f64 + down) / 2)
+    out = f.copy()
+    out = np.where(at_mid_up & (lo > 0), up.astype(np.float32), out)
+    out = np.where(at_mid_down & (lo < 0), down.astype(np.float32), out)
+    return out
+
+
+def _corrected_quotient(x: np.ndarray, s: np.float32, r: np.float32) -> np.ndarray:
+    """q0 = RN(x r); rho = RN(x - q0 s) (exact when done by one FMA); q1 = RN(q0 + rho r),
+    each fused operation emulated exactly in float64 (products of two float32 values have at
+    most 48 significant bits; the last sum goes through a two-sum)."""
+    x64 = x.astype(np.float64)
+    q0 = (x64 * np.float64(r)).astype(np.float32)
+    rho = (x64 - q0.astype(np.float64) * np.float64(s)).astype(np.float32)
+    p = rho.astype(np.float64) * np.float64(r)
+    a = q0.astype(np.float64)
+    hi = a + p
+    bb = hi - a
+    lo = (a - (hi - bb)) + (p - bb)
+    return _round_to_f32(hi, lo)
+
+
 @pytest.mark.parametrize("seed", [0, 1])
-def test_fast_quantizer_equals_the_ieee_quotient_outside_the_near_tie_window(seed):
-    """Wherever |x * r - rne(x * r)| <= 1/2 - 2^-15 (with 2^-24 to spare for the kernel's rounded
-    residual), rne(x * r) equals rne(fl(x / s)); the codes fit in [-127, 127] without a clamp;
-    and the low byte of fl(x * r + 1.5 * 2^23) is the code in two's complement."""
-    flagged = total = wrong_fast = 0
+def test_corrected_quotient_equals_the_ieee_quotient(seed):
+    """For every binary16 x with |x| <= a, over ~300 sampled binary16 row maxima a: Markstein's
+    corrected quotient q1 equals fl(x / s) (bit for bit, but for the sign of a zero quotient,
+    which no code sees), its codes fit in [-127, 127], and the
+    low byte of fl(q1 + 1.5 * 2^23) is the code in two's complement.  rne(x * r) alone, the
+    uncorrected product, differs from the code somewhere in the sample."""
+    total = wrong_uncorrected = 0
     for a in _absmax_sample(150, seed):
         s = np.float32(a) / np.float32(127.0)          # IEEE float32 division
         r = np.float32(1.0) / s                         # reciprocal rounded to nearest
         x = F16_POS[F16_POS <= a].astype(np.float32)
         x = np.concatenate([x, -x])
-        q_ref = np.rint(x / s)                          # fl(x / s), then ties to even
-        assert np.abs(q_ref).max() <= 127
-        t = x.astype(np.float64) * np.float64(r)        # exact: 11 x 24 significant bits
-        q_fast = np.rint(t)
-        d = t - q_fast                                  # exact
-        safe = np.abs(d) <= NEAR + 2.0 ** -24
-        np.testing.assert_array_equal(q_fast[safe], q_ref[safe])
-        # the low byte of fl(x * r + 1.5 * 2^23): the float32 sum of the exact product
-        tb = (t + np.float64(MAGIC)).astype(np.float32)
-        assert np.array_equal(tb.astype(np.float64) - np.float64(MAGIC), q_fast)
+        ref = x / s                                     # fl(x / s)
+        q1 = _corrected_quotient(x, s, r)
+        # equal as values: for x = -0 the correction gives +0 where the quotient is -0
+        np.testing.assert_array_equal(q1, ref, err_msg=f"row maximum {float(a)!r}")
+        nz = ref != 0
+        np.testing.assert_array_equal(q1[nz].view(np.uint32), ref[nz].view(np.uint32))
+        code = np.rint(ref.astype(np.float64))
+        assert np.abs(code).max() <= 127
+        tb = (q1.astype(np.float64) + np.float64(MAGIC)).astype(np.float32)
         low = (tb.view(np.uint32) & 0xFF).astype(np.uint8)
-        np.testing.assert_array_equal(low, q_fast.astype(np.int64).astype(np.int8).view(np.uint8))
-        flagged += int((~safe).sum())
+        np.testing.assert_array_equal(low, code.astype(np.int64).astype(np.int8).view(np.uint8))
         total += x.size
-        wrong_fast += int((q_fast != q_ref).sum())
-    # the exact route is taken for a small fraction of the values, never for most of them, and
-    # it is needed: rne(x * r) alone differs from rne(fl(x / s)) somewhere in the sample
-    assert 0 < flagged < total // 50
-    assert wrong_fast > 0
+        wrong_uncorrected += int((np.rint(x.astype(np.float64) * np.float64(r)) != code).sum())
+    assert total > 1_000_000 and wrong_uncorrected > 0
 
 
 def test_magic_constant_low_byte_for_every_int8_code_and_beyond():
