@@ -244,11 +244,11 @@ cudaError_t launch_colmask(const __half* X, int M, int K, float threshold, uint3
 // ------------------------------------------------------------------ rows + outlier operands
 //
 // The row pass.  A block of 256 threads takes rpb rows at a time (rpb = 1, 2, 4 or 8, so that
-// a thread owns about 8 chunks of 8 columns or more) with tpr = 256 / rpb threads per row:
-// thread (row t / tpr, lane t % tpr) owns chunks lane + tpr j of its row.  It stages its own
-// chunks in shared memory with 16-byte asynchronous copies and is their only reader, so the
-// staging needs no block barrier and holds no registers; as soon as a chunk is quantized its
-// slot is refilled with the same chunk of the block's next row.  Blocks are persistent (up to
+// a thread owns about 8 chunks of 8 columns or more) with tpr = 256 / rpb threads per row (a
+// template parameter): thread (row t / tpr, lane t % tpr) owns chunks lane + tpr j of its row.
+// It stages its own chunks in shared memory with 16-byte asynchronous copies and is their only
+// reader, so the staging needs no block barrier and holds no registers; as soon as a chunk is
+// quantized its slot is refilled with the same chunk of the block's next row.  Blocks are persistent (up to
 // four per SM) and read the outlier mask and its prefix once.  Per row:
 //   1. outlier columns: their fp16 values to X_O at their compacted index, then 0 in the stage,
 //      so that the absolute maximum below is the regular columns' and their codes come out 0;
@@ -413,8 +413,21 @@ __device__ void gather_weights(const RowQuantArgs& a, const uint32_t* mask,
   }
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)),
+// Shared memory through 32-bit shared-window addresses.
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
                "l"(reinterpret_cast<uint64_t>(src))
                : "memory");
 }
@@ -425,21 +438,25 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
 
 }  // namespace
 
+// TPR = threads per row (256, 128, 64 or 32: the block takes 256 / TPR rows at a time).
+template <int TPR>
 __global__ void __launch_bounds__(kRQThreads, kRQBlocksPerSM) rowquant_kernel(const RowQuantArgs a) {
+  constexpr int kRpb = kRQThreads / TPR, kWpr = TPR / 32;  // rows per block, warps per row
   extern __shared__ __align__(128) uint8_t rq_smem[];
   const RowPassSmem L = row_pass_smem(a.K);
   uint32_t* mask = reinterpret_cast<uint32_t*>(rq_smem + L.mask);
   int32_t* prefix = reinterpret_cast<int32_t*>(rq_smem + L.prefix);
   int32_t* misc = reinterpret_cast<int32_t*>(rq_smem + L.misc);
   float* red = reinterpret_cast<float*>(rq_smem + L.red);
-  const int K = a.K, M = a.M, chunks = K / 8, tpr = L.tpr, rpb = L.rpb;
-  const int rl = threadIdx.x / tpr, lr = threadIdx.x % tpr;
-  uint4* stage = reinterpret_cast<uint4*>(rq_smem + L.stage) + static_cast<size_t>(rl) * chunks;
-  const int step = gridDim.x * rpb;  // rows between a block's consecutive row groups
-  int i = blockIdx.x * rpb + rl;
+  const int K = a.K, M = a.M, chunks = K / 8;
+  const int rl = threadIdx.x / TPR, lr = threadIdx.x % TPR;
+  // this thread's row stage: chunk c at stage + 16 c (it owns c = lr + TPR j)
+  const uint32_t stage = smem_addr(rq_smem + L.stage) + static_cast<uint32_t>(rl * chunks) * 16u;
+  const int step = gridDim.x * kRpb;  // rows between a block's consecutive row groups
+  int i = blockIdx.x * kRpb + rl;
   if (i < M) {
     const uint4* src = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(i) * K);
-    for (int c = lr; c < chunks; c += tpr) cp_async16(stage + c, src + c);
+    for (int c = lr; c < chunks; c += TPR) cp_async16(stage + 16u * c, src + c);
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
   grid_dependency_wait();  // the outlier mask is complete from here on
@@ -469,27 +486,35 @@ __global__ void __launch_bounds__(kRQThreads, kRQBlocksPerSM) rowquant_kernel(co
     tensor_max = g;
   }
   const uint8_t* bits_of = reinterpret_cast<const uint8_t*>(mask);  // byte c: chunk c's outliers
-  const int warp = threadIdx.x / 32, wpr = tpr / 32;                // warps per row
+  // bit j: this thread's chunk lr + TPR j holds an outlier column (at most 32 chunks a thread:
+  // K <= 65536 with TPR = 256, and narrower rows have fewer)
+  uint32_t ochunks = 0u;
+  for (int j = 0, c = lr; c < chunks; ++j, c += TPR)
+    if (bits_of[c]) ochunks |= 1u << j;
+  const int warp = threadIdx.x / 32;
   // every thread of the block takes the same number of steps (rows past M idle)
-  for (int it = 0; blockIdx.x * rpb + it * step < M; ++it) {
+  for (int it = 0; blockIdx.x * kRpb + it * step < M; ++it) {
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     const bool live = i < M;
     __half* xo = (a.xo && live) ? a.xo + static_cast<size_t>(i) * a.ldo : nullptr;
     __half2 h0 = __float2half2_rn(0.0f), h1 = h0, h2 = h0, h3 = h0;
     if (live) {
-#pragma unroll 4
-      for (int c = lr; c < chunks; c += tpr) {
-        uint4 x = stage[c];
-        const uint32_t bits = bits_of[c];
-        if (bits) {
+      if (ochunks) {  // the outlier columns: to X_O, then 0 in the stage
+        for (int j = 0, c = lr; c < chunks; ++j, c += TPR) {
+          if (!((ochunks >> j) & 1u)) continue;
+          const uint32_t bits = bits_of[c];
+          const uint4 x = lds128(stage + 16u * c);
           if (xo) emit_outliers(mask, prefix, x, c, bits, xo);
           uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             if ((bits >> e) & 1u) w[e / 2] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
-          x = make_uint4(w[0], w[1], w[2], w[3]);
-          stage[c] = x;
+          sts128(stage + 16u * c, make_uint4(w[0], w[1], w[2], w[3]));
         }
+      }
+#pragma unroll 4
+      for (int c = lr; c < chunks; c += TPR) {
+        const uint4 x = lds128(stage + 16u * c);
         uint32_t b0 = x.x & 0x7FFF7FFFu, b1 = x.y & 0x7FFF7FFFu, b2 = x.z & 0x7FFF7FFFu,
                  b3 = x.w & 0x7FFF7FFFu;
         h0 = __hmax2(h0, *reinterpret_cast<const __half2*>(&b0));
@@ -499,17 +524,18 @@ __global__ void __launch_bounds__(kRQThreads, kRQBlocksPerSM) rowquant_kernel(co
       }
       if (xo != nullptr) {
         const int padded = (n_out + 63) / 64 * 64;
-        for (int r = n_out + lr; r < padded; r += tpr) xo[r] = __float2half_rn(0.0f);
+        for (int r = n_out + lr; r < padded; r += TPR) xo[r] = __float2half_rn(0.0f);
       }
     }
     float amax = half2_max_f(__hmax2(__hmax2(h0, h1), __hmax2(h2, h3)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (wpr > 1) {  // across the row's warps; two buffers, as a warp may be one row ahead
+    if constexpr (kWpr > 1) {  // across the row's warps; two buffers, as a warp may be one row ahead
       float* rd = red + (it & 1) * kRQWarps;
       if ((threadIdx.x & 31) == 0) rd[warp] = amax;
-      named_barrier(1 + rl, tpr);
-      for (int w = rl * wpr; w < (rl + 1) * wpr; ++w) amax = fmaxf(amax, rd[w]);
+      named_barrier(1 + rl, TPR);
+#pragma unroll
+      for (int w = 0; w < kWpr; ++w) amax = fmaxf(amax, rd[rl * kWpr + w]);
     }
     if (tensor_max >= 0.0f) amax = tensor_max;
     const int nx = i + step;
@@ -518,12 +544,17 @@ __global__ void __launch_bounds__(kRQThreads, kRQBlocksPerSM) rowquant_kernel(co
       if (lr == 0) a.xscale[i] = s;
       const float rcp = amax == 0.0f ? 0.0f : __frcp_rn(s);
       uint2* out = reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(i) * K);
-      const bool refill = nx < M;
-      const uint4* next = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(refill ? nx : i) * K);
+      if (nx < M) {  // each slot is refilled with the next row's chunk once its codes are out
+        const uint4* next = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(nx) * K);
 #pragma unroll 4
-      for (int c = lr; c < chunks; c += tpr) {
-        out[c] = codes8(stage[c], s, rcp);
-        if (refill) cp_async16(stage + c, next + c);  // the chunk is in registers
+        for (int c = lr; c < chunks; c += TPR) {
+          const uint4 x = lds128(stage + 16u * c);
+          out[c] = codes8(x, s, rcp);
+          cp_async16(stage + 16u * c, next + c);
+        }
+      } else {
+#pragma unroll 4
+        for (int c = lr; c < chunks; c += TPR) out[c] = codes8(lds128(stage + 16u * c), s, rcp);
       }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -545,8 +576,11 @@ cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&res, cudaDevAttrReservedSharedMemoryPerBlock, dev);
     if (e == cudaSuccess)
       e = cudaDeviceGetAttribute(&per_sm_bytes, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(rowquant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    for (const void* k : {reinterpret_cast<const void*>(rowquant_kernel<256>),
+                          reinterpret_cast<const void*>(rowquant_kernel<128>),
+                          reinterpret_cast<const void*>(rowquant_kernel<64>),
+                          reinterpret_cast<const void*>(rowquant_kernel<32>)})
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e != cudaSuccess) return e;
     reserved[dev] = res;
     smem_per_sm[dev] = per_sm_bytes;
@@ -575,7 +609,12 @@ cudaError_t launch_rowquant(const RowQuantArgs& a, cudaStream_t stream, bool pdl
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, rowquant_kernel, a);
+  switch (L.tpr) {
+    case 256: return cudaLaunchKernelEx(&cfg, rowquant_kernel<256>, a);
+    case 128: return cudaLaunchKernelEx(&cfg, rowquant_kernel<128>, a);
+    case 64: return cudaLaunchKernelEx(&cfg, rowquant_kernel<64>, a);
+    default: return cudaLaunchKernelEx(&cfg, rowquant_kernel<32>, a);
+  }
 }
 
 // ------------------------------------------------------------------ diagnostic: W_hat alone

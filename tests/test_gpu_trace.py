@@ -96,6 +96,9 @@ SHAPES = [
     (17, 512, 300, 3, 6.0),       # tiled path, one row past the few-token routes
     (200, 1040, 600, 5, 6.0),     # tiled path, ragged tiles
     (70, 384, 300, 0, 0.0),       # tiled path, every column an outlier
+    (40, 65536, 64, 7, 6.0),      # tiled path, the longest rows: one 128 KB row stage per block
+    (33, 24576, 96, 5, 6.0),      # tiled path, rows longer than 16K columns, ragged row groups
+    (23, 64, 40, 1, 6.0),         # tiled path, one warp per row (eight rows per block)
 ]
 
 
