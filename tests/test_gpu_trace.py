@@ -132,8 +132,9 @@ def test_trace_workloads(name):
 @pytest.mark.parametrize("M,K", [(4, 256), (8, 1024), (13, 2048), (16, 256), (40, 256),
                                  (3, 1040)])
 def test_trace_planted_ties(M, K):
-    """Values on and next to half-integer quotients x / s = k + 1/2, on every route: the
-    kernels' reciprocal quantizer must fall back to the IEEE quotient exactly there."""
+    """Values on and next to half-integer quotients x / s = k + 1/2, on every route: there the
+    codes of the IEEE quotient differ from those of the uncorrected product x * RN(1/s), and
+    the kernels must give the former."""
     rng = np.random.default_rng(100 + M + K)
     X = rng.standard_normal((M, K)) * 0.05
     for i in range(M):
