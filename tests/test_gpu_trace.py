@@ -99,6 +99,7 @@ SHAPES = [
     (40, 65536, 64, 7, 6.0),      # tiled path, the longest rows: one 128 KB row stage per block
     (33, 24576, 96, 5, 6.0),      # tiled path, rows longer than 16K columns, ragged row groups
     (23, 64, 40, 1, 6.0),         # tiled path, one warp per row (eight rows per block)
+    (41, 6144, 96, 4, 6.0),       # tiled path, 128 threads per row (two rows per block)
 ]
 
 
