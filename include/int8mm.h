@@ -93,7 +93,8 @@ size_t int8_linear_workspace_size(int M, int N, int K);
  * The LLM.int8() linear layer, [P2] section 2.3 with [P5] items 1-3:
  *   O   = { j : max_i |X[i,j]| > threshold }          (outlier feature columns)
  *   sx  = per row i, max over j not in O of |X[i,j]|, divided by 127 (float32)
- *   Xq  = round(X / sx) on the regular columns, 0 on O   (ties to even, [-127,127])
+ *   Xq  = round(X / sx) on the regular columns, 0 on O   (X / sx the float32 IEEE quotient,
+ *         rounded to nearest, ties to even; [-127,127])
  *   Y   = fp16( (Xq . Wq^T)[i,n] * sx[i] * w_scale[n]         (int8 x int8 -> int32)
  *               + sum_{j in O} X[i,j] * W_hat[n,j]             (fp16 operands, fp32 sum)
  *               + bias[n] )
